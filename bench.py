@@ -1,0 +1,367 @@
+#!/usr/bin/env python
+"""QSA forward + backward benchmark on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one full pass of the hot path on one sequence of the seq32k workload
+(T = 32768 tokens, 24 query heads / 2 KV heads, d = 256, 128 four-token blocks
+= 512 unique routed keys per query, 564 route slots with 10% duplicates):
+route sort/dedup + forward + route transpose + dQ + dK/dV, every kernel of the
+library, inputs resident in HBM.  The metric is selected (query, key) token
+pairs per second, N = sum_t |R_t| per step (the two KV groups share the routes).
+
+With N GPUs (torchrun), every rank runs its own sequence (independent problems,
+no collective on the data path) and the reported value is the sum over ranks of
+pairs / the slowest rank's time (weak scaling).
+
+``--impl reference`` times the FP64 CPU oracle on the host cores (each step a
+bounded sample of query rows of the same workload) and prints the same line
+with ``"impl": "reference"``.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = 4
+METRIC = "QSA fwd+bwd selected pairs/s and TFLOP/s at T=32K, 512 sel/query; % roofline"
+UNIT = "pairs/s"
+FWD_FLOPS_PER_PAIR_HEAD = 4 * 256      # QK^T + PV
+BWD_FLOPS_PER_PAIR_HEAD = 10 * 256     # S recompute, dP, dV, dQ, dK
+DKDV_FLOPS_PER_PAIR_HEAD = 4 * 256     # dK = dS^T Q, dV = P^T dO
+FWD_STAGES = ["fwd_route_rows", "fwd_attention"]
+BWD_STAGES = ["bwd_route_rows", "bwd_quad_scan", "bwd_quad_fill", "bwd_quad_sort", "bwd_dq", "bwd_dkdv"]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def workload_config(wl):
+    return {"workload": f"{wl.name}: T={wl.T}, T_kv={wl.T_kv}, {wl.H}Q/{wl.G}KV, d=256, "
+                        f"{wl.blocks} four-token blocks (512 unique keys)/query, {wl.W} route slots "
+                        f"with 10% duplicates, scale=1/16",
+            "T": wl.T, "T_kv": wl.T_kv, "H": wl.H, "G": wl.G, "n_sel": wl.W, "seed": wl.seed}
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample_step(wl, routes, tens, rows):
+    """One oracle fwd+bwd over the given query rows; returns (seconds, pairs)."""
+    import oracle
+    q, k, v, do = tens
+    t0 = time.perf_counter()
+    oracle.forward_rows(q, k, v, routes, wl.scale, rows)
+    oracle.backward_rows(do, q, k, v, routes, wl.scale, rows)
+    dt = time.perf_counter() - t0
+    pairs = sum(len(s) for s in oracle.row_route_sets(routes[rows], wl.T_kv))
+    return dt, pairs
+
+
+def oracle_inputs(wl):
+    from token_indexed_sparse_b200 import workloads as W
+    routes = W.make_routes(wl)
+    q, k, v, do = W.make_tensors(wl)
+    f = lambda x: x.float().numpy().astype(np.float64)  # noqa: E731
+    return routes, (f(q), f(k), f(v), f(do))
+
+
+def cpu_baseline(wl, budget_s=15.0, seed=0):
+    """Oracle (as it stands) on a bounded random sample of query rows."""
+    routes, tens = oracle_inputs(wl)
+    rng = np.random.default_rng(seed)
+    dt, pairs = oracle_sample_step(wl, routes, tens, np.sort(rng.choice(wl.T, 16, replace=False)))
+    n_rows = int(min(wl.T, max(16, 16 * budget_s / max(dt, 1e-3))))
+    rows = np.sort(rng.choice(wl.T, n_rows, replace=False))
+    dt, pairs = oracle_sample_step(wl, routes, tens, rows)
+    return {"value": pairs / dt, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"FP64 row-gather oracle, forward+backward over {n_rows} random query rows "
+                      f"({pairs} pairs) of the same workload, {dt:.1f} s"}
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle, a bounded row sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from token_indexed_sparse_b200 import workloads as W
+    wl = W.CONFIGS[WORKLOAD]
+    routes, tens = oracle_inputs(wl)
+    rng = np.random.default_rng(1)
+    rows_per_step = args.reference_rows
+    for _ in range(args.warmup):
+        oracle_sample_step(wl, routes, tens, np.sort(rng.choice(wl.T, rows_per_step, replace=False)))
+    total_t, total_p = 0.0, 0
+    for _ in range(args.steps):
+        dt, p = oracle_sample_step(wl, routes, tens, np.sort(rng.choice(wl.T, rows_per_step, replace=False)))
+        total_t += dt
+        total_p += p
+    value = total_p / total_t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                             "sample": f"FP64 row-gather oracle, forward+backward over {rows_per_step} random "
+                                       f"query rows per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from token_indexed_sparse_b200 import qsa
+    from token_indexed_sparse_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    wl = W.CONFIGS[args.workload]
+    routes_np = np.array(W.make_routes(wl), dtype=np.int32)
+    q_h, k_h, v_h, do_h = W.make_tensors(wl)
+    pairs = W.pair_count(routes_np, wl.T_kv)
+    flops = (FWD_FLOPS_PER_PAIR_HEAD + BWD_FLOPS_PER_PAIR_HEAD) * wl.H * pairs
+    routes_h = torch.from_numpy(routes_np)
+    host_in = [t.pin_memory() for t in (q_h, k_h, v_h, do_h, routes_h)]
+    q, k, v, do, routes = (t.to(dev) for t in host_in)
+    out = torch.empty_like(q)
+    lse = torch.empty(wl.T, wl.H, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_f = torch.empty(qsa.forward_workspace_size(wl.T, wl.T_kv, wl.H, wl.G, wl.W), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(qsa.backward_workspace_size(wl.T, wl.T_kv, wl.H, wl.G, wl.W), dtype=torch.uint8,
+                       device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    stream = torch.cuda.current_stream(dev)
+
+    def step(fwd_ev=None, bwd_ev=None):
+        qsa.forward(q, k, v, routes, wl.scale, out=out, lse=lse, workspace=ws_f, stage_events=fwd_ev)
+        qsa.backward(do, q, k, v, out, lse, routes, wl.scale, dq=dq, dk=dk, dv=dv, workspace=ws_b,
+                     stage_events=bwd_ev)
+
+    for _ in range(args.warmup):
+        step()
+        flush.zero_()
+    torch.cuda.synchronize()
+
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    starts = [mk() for _ in range(args.steps)]
+    fwd_ev = [[mk() for _ in FWD_STAGES] for _ in range(args.steps)]
+    bwd_ev = [[mk() for _ in BWD_STAGES] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()                 # L2 flushed before every timed step (outside its events)
+        starts[i].record(stream)
+        step(fwd_ev[i], bwd_ev[i])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+
+    stage_ms = {n: [] for n in FWD_STAGES + BWD_STAGES}
+    step_ms = []
+    for i in range(args.steps):
+        prev = starts[i]
+        for n, e in zip(FWD_STAGES + BWD_STAGES, fwd_ev[i] + bwd_ev[i]):
+            stage_ms[n].append(prev.elapsed_time(e))
+            prev = e
+        step_ms.append(starts[i].elapsed_time(bwd_ev[i][-1]))
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * pairs * args.steps / (total_ms * 1e-3)
+
+    if args.no_e2e:
+        if rank == 0:
+            print(json.dumps({"workload": wl.name, "ms_per_step": ms_per_step,
+                              "stage_ms": {n: float(np.mean(v)) for n, v in stage_ms.items()}}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
+    # end to end through the public API: pinned host inputs -> device, fwd+bwd, results -> pinned host
+    res_h = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (out, lse, dq, dk, dv)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in res_h)
+
+    def e2e_step():
+        ins = [t.to(dev, non_blocking=True) for t in host_in]
+        o, l_ = qsa.forward(ins[0], ins[1], ins[2], ins[4], wl.scale, workspace=ws_f)
+        g = qsa.backward(ins[3], ins[0], ins[1], ins[2], o, l_, ins[4], wl.scale, workspace=ws_b)
+        for dst, src in zip(res_h, (o, l_, *g)):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_steps = max(3, args.steps // 4)
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = mk(), mk()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * pairs * e2e_steps / (e2e_ms * 1e-3)
+
+    peaks = load_peaks()
+    avg = {n: float(np.mean(v)) for n, v in stage_ms.items()}
+    dominant = max(avg, key=avg.get)
+    # algorithmic work of the dominant kernel per launch
+    if dominant == "bwd_dkdv":
+        work = DKDV_FLOPS_PER_PAIR_HEAD * wl.H * pairs
+    elif dominant == "bwd_dq":
+        work = (BWD_FLOPS_PER_PAIR_HEAD - DKDV_FLOPS_PER_PAIR_HEAD) * wl.H * pairs
+    elif dominant == "fwd_attention":
+        work = FWD_FLOPS_PER_PAIR_HEAD * wl.H * pairs
+    else:
+        work = None
+    roofline = None
+    if work is not None:
+        achieved = work / (avg[dominant] * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)"}
+    step_tflops = flops / (ms_per_step * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**workload_config(wl), "pairs_per_step": pairs, "flops_per_step": flops,
+                   "l2": "flushed (256 MiB write) before every timed step, outside its events",
+                   "parallelism": f"{world} independent sequences (one per GPU)" if world > 1 else "1 GPU"},
+        "tflops": step_tflops * world,
+        "step_roofline": {"flops": flops, "t_roof_ms": flops / (peaks["bf16_tflops_sustained"] * 1e12) * 1e3,
+                          "frac": step_tflops / peaks["bf16_tflops_sustained"],
+                          "peak": peaks["bf16_tflops_sustained"], "peak_source": peaks["source"]},
+        "stage_ms": avg,
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": args.steps * (len(FWD_STAGES) + len(BWD_STAGES)),
+        "clocks": clk,
+    }
+    if world > 1:
+        dist.barrier()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true",
+                    help="time the device-resident steps only and print the stage breakdown (profiling runs)")
+    ap.add_argument("--workload", type=int, default=WORKLOAD, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--reference-rows", type=int, default=96)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

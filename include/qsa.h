@@ -1,0 +1,166 @@
+/*
+ * qsa.h -- C ABI of the B200 (sm_100a) exact route-set Query Sparse Attention
+ * library (libqsa_b200.so).
+ *
+ * What it computes.  Each query token t attends to the set R_t of K/V rows named
+ * by its route IDs (cuDNN-Frontend "Query Sparse Attention (QSA)" page, sections
+ * "Tensors" and "Selection and components"; "flex_qsa" page, module description
+ * and `_routes_to_membership`; "fa4_qsa" page, `fa4_sparse_gqa_attention`):
+ *   - a route ID r is valid iff 0 <= r < T_kv; every other value (-1, negative,
+ *     >= T_kv) is padding;
+ *   - duplicate IDs select a key once (route membership is a set);
+ *   - no causal or other mask is added: the routes alone decide visibility;
+ *   - grouped-query attention, 12 query heads per KV head: query head h reads KV
+ *     head h / 12 (contiguous head groups, "cudnn_qsa" page, `_CudnnQSA`);
+ *   - head dimension 256, BF16 inputs and outputs, FP32 accumulation.
+ * Forward:  S = scale * Q_h K_g^T over R_t, P = softmax(S), out = P V_g,
+ *           lse = natural-log softmax normaliser.  A row with empty R_t gives
+ *           out = 0 and lse = -inf.
+ * Backward: the equations of the "Selection and components" section:
+ *           P = exp(S - lse), delta = rowsum(dO * out), dP = dO V^T,
+ *           dS = P * (dP - delta), dQ = scale dS K, dK = scale dS^T Q,
+ *           dV = P^T dO, dK/dV summed over the 12 query heads of each group.
+ *           Empty rows give dQ = 0 and contribute nothing to dK/dV.  dK/dV are
+ *           bitwise reproducible run to run (no floating-point atomics).
+ *
+ * Conventions for every entry point.
+ *   - BF16 tensors are passed as `const void*` / `void*` holding IEEE bfloat16
+ *     bit patterns.  All tensors are dense, contiguous, row-major, on the device
+ *     that is current when the call is made.
+ *       q, out, grad_out, dq : [T, H, 256] BF16        (H = 12 * G)
+ *       k, v, dk, dv         : [T_kv, G, 256] BF16
+ *       routes               : [T, n_sel] int32
+ *       lse                  : [T, H] float32 (natural log)
+ *   - BF16 tensors must be 16-byte aligned, int32/float32 tensors 4-byte aligned,
+ *     the workspace 256-byte aligned.
+ *   - The caller owns every buffer, including the workspace (size from the
+ *     matching *_workspace_size function).  The library allocates no device
+ *     memory and keeps no state between calls.  The workspace contents are
+ *     scratch: nothing needs to be initialised, nothing survives the call.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without synchronising.  Route values are never
+ *     read on the host.
+ *   - Errors: arguments are checked on the host before anything is launched;
+ *     a failed check returns its status and launches nothing.  A failed kernel
+ *     launch returns QSA_ERR_CUDA.  Route values are never errors (invalid IDs
+ *     are padding).
+ *   - Limits: T, T_kv, n_sel >= 1; n_sel <= 16384; T * n_sel <= 2^31 - 1;
+ *     T_kv <= 2^31 - 1; H = 12 * G, G >= 1; 0 < scale < inf.
+ */
+#ifndef QSA_B200_H
+#define QSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* qsa_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  QSA_OK = 0,
+  QSA_ERR_INVALID_ARGUMENT = 1,   /* null pointer, size out of range, bad scale */
+  QSA_ERR_UNSUPPORTED = 2,        /* head geometry other than 12 query heads per KV head */
+  QSA_ERR_MISALIGNED = 3,         /* a pointer violates the alignment rules above */
+  QSA_ERR_WORKSPACE_TOO_SMALL = 4,
+  QSA_ERR_CUDA = 5                /* a CUDA runtime call or kernel launch failed */
+} qsa_status_t;
+
+/* Human-readable name of a status; never NULL, static storage. */
+const char* qsa_status_string(qsa_status_t status);
+
+/* Library version string, static storage. */
+const char* qsa_version(void);
+
+/*
+ * Workspace bytes needed by qsa_forward / qsa_backward for these sizes.  Returns
+ * 0 when the sizes are outside the limits above (the matching call would return
+ * QSA_ERR_INVALID_ARGUMENT or QSA_ERR_UNSUPPORTED).
+ */
+size_t qsa_forward_workspace_size(int64_t T, int64_t T_kv, int H, int G, int n_sel);
+size_t qsa_backward_workspace_size(int64_t T, int64_t T_kv, int H, int G, int n_sel);
+
+/*
+ * Forward pass.  Cites: "Query Sparse Attention (QSA)" page, "Selection and
+ * components" (forward: scaled QK, softmax, PV; FP32 output cast to BF16;
+ * natural-log LSE; empty rows zero output and -inf LSE).
+ *   in : q, k, v, routes, sizes, scale (finite, > 0; normally 1/16)
+ *   out: out [T, H, 256] BF16, lse [T, H] float32
+ */
+qsa_status_t qsa_forward(const void* q, const void* k, const void* v, const int32_t* routes,
+                         int64_t T, int64_t T_kv, int H, int G, int n_sel, float scale,
+                         void* out, float* lse,
+                         void* workspace, size_t workspace_bytes, qsa_stream_t stream);
+
+/*
+ * Backward pass.  Cites: "Query Sparse Attention (QSA)" page, "Selection and
+ * components" (the backward equations; delta from the forward output; FP32
+ * accumulation, BF16 gradients; dK/dV summed over query heads).
+ *   in : grad_out, q, k, v, out and lse from qsa_forward with the same q, k, v,
+ *        routes and scale; routes, sizes, scale
+ *   out: dq [T, H, 256], dk and dv [T_kv, G, 256] (BF16).  Every row of dk/dv is
+ *        written; keys no query routes to get exact zeros.
+ */
+qsa_status_t qsa_backward(const void* grad_out, const void* q, const void* k, const void* v,
+                          const void* out, const float* lse, const int32_t* routes,
+                          int64_t T, int64_t T_kv, int H, int G, int n_sel, float scale,
+                          void* dq, void* dk, void* dv,
+                          void* workspace, size_t workspace_bytes, qsa_stream_t stream);
+
+/*
+ * Same as qsa_forward / qsa_backward, and in addition records caller-created
+ * CUDA events (cudaEvent_t, passed as qsa_event_t) on `stream` after each stage,
+ * for per-kernel timing.  Stage i's event is recorded right after stage i is
+ * enqueued; only the first min(n_stage_events, stage count) are recorded.
+ * `stage_events` may be NULL when n_stage_events is 0.  The paper has no
+ * counterpart: this is an instrumentation hook of this library.
+ *   forward stages : 0 route rows (sort/dedup), 1 attention forward
+ *   backward stages: 0 route rows + quad counts, 1 quad scan, 2 quad fill,
+ *                    3 quad sort, 4 dQ (+ delta, P/dS records), 5 dK/dV
+ * A failed eventRecord returns QSA_ERR_CUDA.
+ */
+typedef struct CUevent_st* qsa_event_t; /* same type as cudaEvent_t */
+#define QSA_FORWARD_STAGES 2
+#define QSA_BACKWARD_STAGES 6
+
+qsa_status_t qsa_forward_ex(const void* q, const void* k, const void* v, const int32_t* routes,
+                            int64_t T, int64_t T_kv, int H, int G, int n_sel, float scale,
+                            void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, qsa_stream_t stream,
+                            const qsa_event_t* stage_events, int n_stage_events);
+qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k, const void* v,
+                             const void* out, const float* lse, const int32_t* routes,
+                             int64_t T, int64_t T_kv, int H, int G, int n_sel, float scale,
+                             void* dq, void* dk, void* dv,
+                             void* workspace, size_t workspace_bytes, qsa_stream_t stream,
+                             const qsa_event_t* stage_events, int n_stage_events);
+
+/*
+ * Route preprocessing on its own, exposing the index structures the attention
+ * kernels consume.  Cites: "fa4_qsa" page, `_preprocess` (duplicates collapse,
+ * invalid IDs discarded; forward and reverse lists).
+ *   row_cnt  [T] int32       : |R_t|
+ *   row_cols [T, n_sel] int32: R_t ascending in the first row_cnt[t] slots; the
+ *                              remaining slots are left unspecified
+ *   quad_ptr [ceil(T_kv/4)+1] int32 : CSR offsets of the key-quad lists
+ *   quad_ent [T * n_sel] int64 : for quad b (keys 4b..4b+3), entries
+ *       quad_ent[quad_ptr[b] .. quad_ptr[b+1]) in ascending query order, each
+ *       (t << 32) | (i0 << 4) | mask, where t is a query whose R_t meets the
+ *       quad, mask bit j is set iff key 4b+j is in R_t, and i0 is the position in
+ *       row_cols[t, :] of the quad's first key in R_t.  Slots past quad_ptr[last]
+ *       are left unspecified.
+ *   scratch: qsa_route_plan_scratch_size(T, T_kv) bytes, 256-byte aligned.
+ */
+size_t qsa_route_plan_scratch_size(int64_t T, int64_t T_kv);
+qsa_status_t qsa_route_plan(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel,
+                            int32_t* row_cnt, int32_t* row_cols, int32_t* quad_ptr,
+                            int64_t* quad_ent, void* scratch, size_t scratch_bytes,
+                            qsa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QSA_B200_H */

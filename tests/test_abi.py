@@ -1,0 +1,97 @@
+"""The C-ABI library builds, loads and exports what include/qsa.h declares;
+host-side argument checks reject bad calls before any CUDA work (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from token_indexed_sparse_b200 import build, qsa
+    build.build()
+    return qsa.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b(qsa_[a-z_0-9]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("qsa_forward", "qsa_backward", "qsa_forward_workspace_size",
+                     "qsa_backward_workspace_size", "qsa_status_string", "qsa_route_plan"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in enumerate(["QSA_OK", "QSA_ERR_INVALID_ARGUMENT", "QSA_ERR_UNSUPPORTED",
+                                 "QSA_ERR_MISALIGNED", "QSA_ERR_WORKSPACE_TOO_SMALL", "QSA_ERR_CUDA"]):
+        assert lib.qsa_status_string(code).decode() == name
+    assert b"sm_100a" in lib.qsa_version()
+
+
+def test_workspace_sizes(lib):
+    fw = lib.qsa_forward_workspace_size(32768, 32768, 24, 2, 564)
+    bw = lib.qsa_backward_workspace_size(32768, 32768, 24, 2, 564)
+    assert fw >= 32768 * 564 * 4 and bw > fw
+    assert fw % 256 == 0 and bw % 256 == 0
+    # outside the supported envelope -> 0
+    assert lib.qsa_forward_workspace_size(16, 16, 8, 1, 4) == 0        # 8 heads per KV head
+    assert lib.qsa_forward_workspace_size(0, 16, 12, 1, 4) == 0
+    assert lib.qsa_forward_workspace_size(16, 16, 12, 1, 16385) == 0
+    assert lib.qsa_backward_workspace_size(2**30, 16, 12, 1, 4) == 0   # T * n_sel > INT32_MAX
+
+
+def _fwd(lib, q=256, k=256, v=256, routes=256, T=16, T_kv=16, H=12, G=1, n_sel=4, scale=0.0625,
+         out=256, lse=256, ws=256, ws_bytes=1 << 20):
+    P = ctypes.c_void_p
+    return lib.qsa_forward(P(q), P(k), P(v), P(routes), T, T_kv, H, G, n_sel, scale, P(out), P(lse),
+                           P(ws), ws_bytes, None)
+
+
+def test_host_validation_before_any_launch(lib):
+    # These return before touching CUDA, so they run without a GPU.
+    assert _fwd(lib, q=0) == 1                       # null pointer
+    assert _fwd(lib, T=0) == 1
+    assert _fwd(lib, n_sel=0) == 1
+    assert _fwd(lib, scale=0.0) == 1
+    assert _fwd(lib, scale=float("inf")) == 1
+    assert _fwd(lib, scale=float("nan")) == 1
+    assert _fwd(lib, scale=-1.0) == 1
+    assert _fwd(lib, H=16, G=1) == 2                 # 16 query heads per KV head
+    assert _fwd(lib, H=13, G=2) == 2
+    assert _fwd(lib, q=264) == 3                     # 8-byte aligned BF16 tensor
+    assert _fwd(lib, routes=258) == 3
+    assert _fwd(lib, ws=4096 + 16) == 3
+    assert _fwd(lib, ws_bytes=16) == 4
+    P = ctypes.c_void_p
+    st = lib.qsa_backward(P(256), P(256), P(256), P(256), P(256), P(256), P(256), 16, 16, 12, 1, 4,
+                          0.0625, P(256), P(256), P(0), P(256), 1 << 30, None)
+    assert st == 1                                   # null dv
+    st = lib.qsa_backward(P(256), P(256), P(256), P(256), P(256), P(256), P(256), 16, 16, 12, 1, 4,
+                          0.0625, P(256), P(256), P(256), P(256), 8, None)
+    assert st == 4
+    st = lib.qsa_route_plan(P(256), 16, 16, 4, P(256), P(256), P(256), P(260), P(256), 1 << 20, None)
+    assert st == 3                                   # int64 entries need 8-byte alignment
+
+
+def test_no_cpu_fallback_without_library(monkeypatch, tmp_path):
+    from token_indexed_sparse_b200 import qsa
+    monkeypatch.setattr(qsa, "_lib", None)
+    monkeypatch.setattr(qsa, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        qsa.library()

@@ -1,0 +1,218 @@
+// C ABI of the QSA library: host-side argument checks, workspace layout and the
+// launch sequences of the forward, backward and route-plan calls.  Nothing here
+// reads device memory or synchronises; every launch goes to the caller's stream.
+#include <climits>
+#include <cmath>
+#include <cstdint>
+
+#include "qsa.h"
+#include "qsa_device.cuh"
+#include "qsa_internal.h"
+
+namespace {
+
+constexpr int kMaxSel = 16384;
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+qsa_status_t check_sizes(int64_t T, int64_t T_kv, int H, int G, int n_sel) {
+  if (T < 1 || T_kv < 1 || n_sel < 1 || n_sel > kMaxSel || G < 1 || H < 1) return QSA_ERR_INVALID_ARGUMENT;
+  if (T_kv > INT32_MAX || T > INT32_MAX / n_sel) return QSA_ERR_INVALID_ARGUMENT;
+  if (H % G != 0 || H / G != qsa::kHeadsPerGroup) return QSA_ERR_UNSUPPORTED;
+  if (T > INT32_MAX / G || (T_kv + 3) / 4 > INT32_MAX / G) return QSA_ERR_INVALID_ARGUMENT;
+  return QSA_OK;
+}
+
+struct Layout {
+  size_t row_cnt = 0, row_cols = 0, quad_cnt = 0, quad_ptr = 0, quad_fill = 0, quad_ent = 0, delta = 0,
+         pds = 0, total = 0;
+};
+
+Layout make_layout(int64_t T, int64_t T_kv, int H, int G, int n_sel, bool backward) {
+  Layout L;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  const size_t nq = static_cast<size_t>((T_kv + 3) / 4);
+  const size_t pairs = static_cast<size_t>(T) * static_cast<size_t>(n_sel);
+  L.row_cnt = take(static_cast<size_t>(T) * 4);
+  L.row_cols = take(pairs * 4);
+  if (backward) {
+    L.quad_cnt = take(nq * 4);
+    L.quad_ptr = take((nq + 1) * 4);
+    L.quad_fill = take(nq * 4);
+    L.quad_ent = take(pairs * 8);
+    L.delta = take(static_cast<size_t>(T) * H * 4);
+    L.pds = take(pairs * G * 48);
+  }
+  L.total = off;
+  return L;
+}
+
+template <typename P>
+P* at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<uint8_t*>(ws) + off);
+}
+
+#define QSA_TRY(expr)                         \
+  do {                                        \
+    cudaError_t e_ = (expr);                  \
+    if (e_ != cudaSuccess) return QSA_ERR_CUDA; \
+  } while (0)
+
+// Records stage event i (if supplied) on the stream.
+struct StageEvents {
+  const qsa_event_t* ev;
+  int n;
+  cudaStream_t s;
+  cudaError_t mark(int i) const {
+    if (ev == nullptr || i >= n || ev[i] == nullptr) return cudaSuccess;
+    return cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[i]), s);
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+const char* qsa_status_string(qsa_status_t status) {
+  switch (status) {
+    case QSA_OK: return "QSA_OK";
+    case QSA_ERR_INVALID_ARGUMENT: return "QSA_ERR_INVALID_ARGUMENT";
+    case QSA_ERR_UNSUPPORTED: return "QSA_ERR_UNSUPPORTED";
+    case QSA_ERR_MISALIGNED: return "QSA_ERR_MISALIGNED";
+    case QSA_ERR_WORKSPACE_TOO_SMALL: return "QSA_ERR_WORKSPACE_TOO_SMALL";
+    case QSA_ERR_CUDA: return "QSA_ERR_CUDA";
+  }
+  return "QSA_ERR_UNKNOWN";
+}
+
+const char* qsa_version(void) { return "qsa_b200 0.1 (sm_100a)"; }
+
+size_t qsa_forward_workspace_size(int64_t T, int64_t T_kv, int H, int G, int n_sel) {
+  if (check_sizes(T, T_kv, H, G, n_sel) != QSA_OK) return 0;
+  return make_layout(T, T_kv, H, G, n_sel, false).total;
+}
+
+size_t qsa_backward_workspace_size(int64_t T, int64_t T_kv, int H, int G, int n_sel) {
+  if (check_sizes(T, T_kv, H, G, n_sel) != QSA_OK) return 0;
+  return make_layout(T, T_kv, H, G, n_sel, true).total;
+}
+
+qsa_status_t qsa_forward(const void* q, const void* k, const void* v, const int32_t* routes, int64_t T,
+                         int64_t T_kv, int H, int G, int n_sel, float scale, void* out, float* lse,
+                         void* workspace, size_t workspace_bytes, qsa_stream_t stream) {
+  return qsa_forward_ex(q, k, v, routes, T, T_kv, H, G, n_sel, scale, out, lse, workspace, workspace_bytes, stream,
+                        nullptr, 0);
+}
+
+qsa_status_t qsa_forward_ex(const void* q, const void* k, const void* v, const int32_t* routes, int64_t T,
+                            int64_t T_kv, int H, int G, int n_sel, float scale, void* out, float* lse,
+                            void* workspace, size_t workspace_bytes, qsa_stream_t stream,
+                            const qsa_event_t* stage_events, int n_stage_events) {
+  if (!q || !k || !v || !routes || !out || !lse || !workspace) return QSA_ERR_INVALID_ARGUMENT;
+  const qsa_status_t st = check_sizes(T, T_kv, H, G, n_sel);
+  if (st != QSA_OK) return st;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return QSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(routes, 4) ||
+      !aligned(lse, 4) || !aligned(workspace, 256))
+    return QSA_ERR_MISALIGNED;
+  const Layout L = make_layout(T, T_kv, H, G, n_sel, false);
+  if (workspace_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* row_cnt = at<int32_t>(workspace, L.row_cnt);
+  int32_t* row_cols = at<int32_t>(workspace, L.row_cols);
+  const StageEvents ev{stage_events, n_stage_events, s};
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, s));
+  QSA_TRY(ev.mark(0));
+  QSA_TRY(qsa::launch_forward(q, k, v, row_cnt, row_cols, T, G, n_sel, scale, out, lse, s));
+  QSA_TRY(ev.mark(1));
+  return QSA_OK;
+}
+
+qsa_status_t qsa_backward(const void* grad_out, const void* q, const void* k, const void* v, const void* out,
+                          const float* lse, const int32_t* routes, int64_t T, int64_t T_kv, int H, int G,
+                          int n_sel, float scale, void* dq, void* dk, void* dv, void* workspace,
+                          size_t workspace_bytes, qsa_stream_t stream) {
+  return qsa_backward_ex(grad_out, q, k, v, out, lse, routes, T, T_kv, H, G, n_sel, scale, dq, dk, dv, workspace,
+                         workspace_bytes, stream, nullptr, 0);
+}
+
+qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k, const void* v, const void* out,
+                             const float* lse, const int32_t* routes, int64_t T, int64_t T_kv, int H, int G,
+                             int n_sel, float scale, void* dq, void* dk, void* dv, void* workspace,
+                             size_t workspace_bytes, qsa_stream_t stream, const qsa_event_t* stage_events,
+                             int n_stage_events) {
+  if (!grad_out || !q || !k || !v || !out || !lse || !routes || !dq || !dk || !dv || !workspace)
+    return QSA_ERR_INVALID_ARGUMENT;
+  const qsa_status_t st = check_sizes(T, T_kv, H, G, n_sel);
+  if (st != QSA_OK) return st;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return QSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(grad_out, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(routes, 4) ||
+      !aligned(workspace, 256))
+    return QSA_ERR_MISALIGNED;
+  const Layout L = make_layout(T, T_kv, H, G, n_sel, true);
+  if (workspace_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t nq = (T_kv + 3) / 4;
+  int32_t* row_cnt = at<int32_t>(workspace, L.row_cnt);
+  int32_t* row_cols = at<int32_t>(workspace, L.row_cols);
+  int32_t* quad_cnt = at<int32_t>(workspace, L.quad_cnt);
+  int32_t* quad_ptr = at<int32_t>(workspace, L.quad_ptr);
+  int32_t* quad_fill = at<int32_t>(workspace, L.quad_fill);
+  int64_t* quad_ent = at<int64_t>(workspace, L.quad_ent);
+  float* delta = at<float>(workspace, L.delta);
+  uint16_t* pds = at<uint16_t>(workspace, L.pds);
+  const StageEvents ev{stage_events, n_stage_events, s};
+  QSA_TRY(cudaMemsetAsync(quad_cnt, 0, static_cast<size_t>(nq) * 4, s));
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, quad_cnt, s));
+  QSA_TRY(ev.mark(0));
+  QSA_TRY(qsa::launch_quad_scan(quad_cnt, nq, quad_ptr, quad_fill, s));
+  QSA_TRY(ev.mark(1));
+  QSA_TRY(qsa::launch_quad_fill(row_cnt, row_cols, T, n_sel, quad_fill, quad_ent, s));
+  QSA_TRY(ev.mark(2));
+  QSA_TRY(qsa::launch_quad_sort(quad_ptr, nq, quad_ent, s));
+  QSA_TRY(ev.mark(3));
+  QSA_TRY(qsa::launch_backward_dq(grad_out, q, k, v, out, lse, row_cnt, row_cols, T, G, n_sel, scale, dq, delta,
+                                  pds, s));
+  QSA_TRY(ev.mark(4));
+  QSA_TRY(qsa::launch_backward_dkdv(grad_out, q, pds, quad_ptr, quad_ent, T, T_kv, G, n_sel, scale, dk, dv, s));
+  QSA_TRY(ev.mark(5));
+  return QSA_OK;
+}
+
+size_t qsa_route_plan_scratch_size(int64_t T, int64_t T_kv) {
+  if (T < 1 || T_kv < 1 || T_kv > INT32_MAX) return 0;
+  const size_t nq = static_cast<size_t>((T_kv + 3) / 4);
+  return 2 * align256(nq * 4);
+}
+
+qsa_status_t qsa_route_plan(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel, int32_t* row_cnt,
+                            int32_t* row_cols, int32_t* quad_ptr, int64_t* quad_ent, void* scratch,
+                            size_t scratch_bytes, qsa_stream_t stream) {
+  if (!routes || !row_cnt || !row_cols || !quad_ptr || !quad_ent || !scratch) return QSA_ERR_INVALID_ARGUMENT;
+  const qsa_status_t st = check_sizes(T, T_kv, qsa::kHeadsPerGroup, 1, n_sel);
+  if (st != QSA_OK) return st;
+  if (!aligned(routes, 4) || !aligned(row_cnt, 4) || !aligned(row_cols, 4) || !aligned(quad_ptr, 4) ||
+      !aligned(quad_ent, 8) || !aligned(scratch, 256))
+    return QSA_ERR_MISALIGNED;
+  if (scratch_bytes < qsa_route_plan_scratch_size(T, T_kv)) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t nq = (T_kv + 3) / 4;
+  int32_t* quad_cnt = static_cast<int32_t*>(scratch);
+  int32_t* quad_fill = at<int32_t>(scratch, align256(static_cast<size_t>(nq) * 4));
+  QSA_TRY(cudaMemsetAsync(quad_cnt, 0, static_cast<size_t>(nq) * 4, s));
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, quad_cnt, s));
+  QSA_TRY(qsa::launch_quad_scan(quad_cnt, nq, quad_ptr, quad_fill, s));
+  QSA_TRY(qsa::launch_quad_fill(row_cnt, row_cols, T, n_sel, quad_fill, quad_ent, s));
+  QSA_TRY(qsa::launch_quad_sort(quad_ptr, nq, quad_ent, s));
+  return QSA_OK;
+}
+
+}  // extern "C"

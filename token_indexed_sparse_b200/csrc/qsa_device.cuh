@@ -1,0 +1,86 @@
+// Device-side building blocks shared by the QSA kernels (sm_100a).
+//
+// Warp-level BF16 tensor-core MMA (m16n8k16, FP32 accumulate) and the shared
+// memory / async-copy primitives the kernels stage gathered rows with.
+//
+// Fragment conventions for mma.m16n8k16.row.col (g = lane / 4, c = lane % 4):
+//   A (16x16, row-major)  a0: (g, 2c..2c+1)   a1: (g+8, 2c..)   a2: (g, 2c+8..)  a3: (g+8, 2c+8..)
+//   B (16x8, k-by-n)      b0: (k 2c..2c+1, n g)                  b1: (k 2c+8.., n g)
+//   C (16x8, fp32)        c0: (g, 2c)  c1: (g, 2c+1)  c2: (g+8, 2c)  c3: (g+8, 2c+1)
+// In a packed register the lower 16 bits hold the lower k (or column) index.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace qsa {
+
+constexpr int kHeadDim = 256;       // d
+constexpr int kHeadsPerGroup = 12;  // query heads sharing one KV head
+constexpr int kRowTile = 16;        // MMA M tile: 12 heads padded to 16
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16-byte global->shared async copy; when `pred` is false the 16 destination
+// bytes are zero-filled and nothing is read from `src`.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool pred) {
+  const int n = pred ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+
+// d += a * b  (bf16 inputs, fp32 accumulate)
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Round two floats to bf16 (round-to-nearest-even) and pack: lo -> bits 0..15.
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
+// Select 16-bit halves of two registers: result = {lo: half of a, hi: half of b}.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;\n" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+constexpr uint32_t kLoLo = 0x5410;  // {a.lo, b.lo}
+constexpr uint32_t kHiHi = 0x7632;  // {a.hi, b.hi}
+
+// Byte offset of 16-byte chunk `c` (0..31) of row `r` in a [rows][256] bf16 tile
+// whose rows are 512 bytes: chunks are XOR-swizzled within each 128-byte group so
+// that eight consecutive rows read at the same logical chunk hit distinct banks.
+__device__ __forceinline__ uint32_t swz512(int r, int c) {
+  return static_cast<uint32_t>(r * 512 + ((c ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+}  // namespace qsa

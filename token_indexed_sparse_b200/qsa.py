@@ -1,0 +1,197 @@
+"""Thin Python binding of libqsa_b200.so (argument marshalling only).
+
+Every step of the computation runs in the CUDA library; this module passes
+device pointers of PyTorch tensors and the current CUDA stream through the C ABI
+declared in ``include/qsa.h``.  There is no fallback: if the library is missing
+or the tensors are not on a CUDA device, the call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libqsa_b200.so")
+_lib = None
+
+QSA_OK = 0
+
+
+class QSAError(RuntimeError):
+    """A QSA C-ABI call returned a non-OK status."""
+
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+def library() -> ctypes.CDLL:
+    """Load the shared library (once); raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise RuntimeError(
+            f"QSA CUDA library not found at {_LIB_PATH}; build it with "
+            "`python -m token_indexed_sparse_b200.build` (there is no CPU fallback)")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i64, i32, f32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.qsa_status_string.restype = ctypes.c_char_p
+    lib.qsa_status_string.argtypes = [i32]
+    lib.qsa_version.restype = ctypes.c_char_p
+    lib.qsa_version.argtypes = []
+    for name in ("qsa_forward_workspace_size", "qsa_backward_workspace_size"):
+        f = getattr(lib, name)
+        f.restype = sz
+        f.argtypes = [i64, i64, i32, i32, i32]
+    lib.qsa_forward.restype = i32
+    lib.qsa_forward.argtypes = [vp, vp, vp, vp, i64, i64, i32, i32, i32, f32, vp, vp, vp, sz, vp]
+    lib.qsa_backward.restype = i32
+    lib.qsa_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, f32,
+                                 vp, vp, vp, vp, sz, vp]
+    lib.qsa_forward_ex.restype = i32
+    lib.qsa_forward_ex.argtypes = lib.qsa_forward.argtypes + [vp, i32]
+    lib.qsa_backward_ex.restype = i32
+    lib.qsa_backward_ex.argtypes = lib.qsa_backward.argtypes + [vp, i32]
+    lib.qsa_route_plan_scratch_size.restype = sz
+    lib.qsa_route_plan_scratch_size.argtypes = [i64, i64]
+    lib.qsa_route_plan.restype = i32
+    lib.qsa_route_plan.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp, vp, sz, vp]
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return library().qsa_status_string(int(status)).decode()
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != QSA_OK:
+        raise QSAError(status, what)
+
+
+def _prep(x: torch.Tensor, dtype, name: str) -> torch.Tensor:
+    if not x.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if x.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {x.dtype}")
+    return x.contiguous()
+
+
+def _sizes(q, k, routes):
+    if q.dim() != 3 or k.dim() != 3 or routes.dim() != 2:
+        raise ValueError("expected q [T,H,256], k/v [T_kv,G,256], routes [T,n_sel]")
+    T, H, D = q.shape
+    T_kv, G, Dk = k.shape
+    if D != 256 or Dk != 256:
+        raise ValueError("head dimension must be 256")
+    if routes.shape[0] != T:
+        raise ValueError("routes must have one row per query")
+    return T, T_kv, H, G, routes.shape[1]
+
+
+def forward_workspace_size(T, T_kv, H, G, n_sel) -> int:
+    return int(library().qsa_forward_workspace_size(T, T_kv, H, G, n_sel))
+
+
+def backward_workspace_size(T, T_kv, H, G, n_sel) -> int:
+    return int(library().qsa_backward_workspace_size(T, T_kv, H, G, n_sel))
+
+
+def _workspace(nbytes: int, device, given: torch.Tensor | None) -> torch.Tensor:
+    if given is not None:
+        return given
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def _events(stage_events):
+    """ctypes array of raw cudaEvent_t handles from torch.cuda.Event objects."""
+    if not stage_events:
+        return None, 0
+    handles = []
+    for e in stage_events:
+        if e.cuda_event == 0:          # torch creates events lazily
+            e.record()
+        handles.append(e.cuda_event)
+    return (ctypes.c_void_p * len(handles))(*handles), len(handles)
+
+
+def forward(q, k, v, routes, scale: float = 1.0 / 16.0, *, out=None, lse=None, workspace=None,
+            stage_events=None):
+    """qsa_forward: returns ``(out [T,H,256] bf16, lse [T,H] float32)``.
+
+    ``stage_events`` (optional list of torch.cuda.Event) are recorded after the
+    route-sort and attention stages (qsa_forward_ex)."""
+    lib = library()
+    q = _prep(q, torch.bfloat16, "q")
+    k = _prep(k, torch.bfloat16, "k")
+    v = _prep(v, torch.bfloat16, "v")
+    routes = _prep(routes, torch.int32, "routes")
+    T, T_kv, H, G, n_sel = _sizes(q, k, routes)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(T, H, dtype=torch.float32, device=q.device)
+    ws_bytes = lib.qsa_forward_workspace_size(T, T_kv, H, G, n_sel)
+    ws = _workspace(ws_bytes, q.device, workspace)
+    ev, n_ev = _events(stage_events)
+    st = lib.qsa_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(routes), T, T_kv, H, G, n_sel, float(scale),
+                            _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device), ev, n_ev)
+    _check(st, "qsa_forward")
+    return out, lse
+
+
+def backward(grad_out, q, k, v, out, lse, routes, scale: float = 1.0 / 16.0, *,
+             dq=None, dk=None, dv=None, workspace=None, stage_events=None):
+    """qsa_backward: returns ``(dq, dk, dv)`` (bf16, shapes of q, k, v).
+
+    ``stage_events`` (optional, up to 6 torch.cuda.Event) are recorded after
+    each backward stage (qsa_backward_ex)."""
+    lib = library()
+    grad_out = _prep(grad_out, torch.bfloat16, "grad_out")
+    q = _prep(q, torch.bfloat16, "q")
+    k = _prep(k, torch.bfloat16, "k")
+    v = _prep(v, torch.bfloat16, "v")
+    out = _prep(out, torch.bfloat16, "out")
+    lse = _prep(lse, torch.float32, "lse")
+    routes = _prep(routes, torch.int32, "routes")
+    T, T_kv, H, G, n_sel = _sizes(q, k, routes)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws_bytes = lib.qsa_backward_workspace_size(T, T_kv, H, G, n_sel)
+    ws = _workspace(ws_bytes, q.device, workspace)
+    ev, n_ev = _events(stage_events)
+    st = lib.qsa_backward_ex(_ptr(grad_out), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(routes),
+                             T, T_kv, H, G, n_sel, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+                             _ptr(ws), ws.numel(), _stream(q.device), ev, n_ev)
+    _check(st, "qsa_backward")
+    return dq, dk, dv
+
+
+def route_plan(routes, T_kv: int):
+    """qsa_route_plan: ``(row_cnt, row_cols, quad_ptr, quad_ent)`` device tensors."""
+    lib = library()
+    routes = _prep(routes, torch.int32, "routes")
+    T, n_sel = routes.shape
+    dev = routes.device
+    nq = (T_kv + 3) // 4
+    row_cnt = torch.empty(T, dtype=torch.int32, device=dev)
+    row_cols = torch.empty(T, n_sel, dtype=torch.int32, device=dev)
+    quad_ptr = torch.empty(nq + 1, dtype=torch.int32, device=dev)
+    quad_ent = torch.empty(T * n_sel, dtype=torch.int64, device=dev)
+    scratch = torch.empty(max(256, lib.qsa_route_plan_scratch_size(T, T_kv)), dtype=torch.uint8, device=dev)
+    st = lib.qsa_route_plan(_ptr(routes), T, T_kv, n_sel, _ptr(row_cnt), _ptr(row_cols), _ptr(quad_ptr),
+                            _ptr(quad_ent), _ptr(scratch), scratch.numel(), _stream(dev))
+    _check(st, "qsa_route_plan")
+    return row_cnt, row_cols, quad_ptr, quad_ent
