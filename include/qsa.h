@@ -159,6 +159,39 @@ qsa_status_t qsa_route_plan(const int32_t* routes, int64_t T, int64_t T_kv, int 
                             int64_t* quad_ent, void* scratch, size_t scratch_bytes,
                             qsa_stream_t stream);
 
+/*
+ * Allocation-free forward, for callers that cannot allocate device memory: for
+ * example an extension running inside a host application that owns the device
+ * allocator and offers it no allocation hook, or a latency-critical path that
+ * must not call cudaMalloc (which can synchronise the device and has no bounded
+ * latency).  The paper has no counterpart: this is an interface convenience of
+ * this library.
+ *
+ * Same arguments and results as qsa_forward, minus the workspace.  The scratch
+ * the forward needs (the per-row sorted route lists) lives in a fixed array of
+ * QSA_NOALLOC_SCRATCH_BYTES (16 MiB) compiled into the library; every GPU on
+ * which the library runs this call holds that array until the process exits.
+ *   - Limit: qsa_forward_workspace_size(T, T_kv, H, G, n_sel) must not exceed
+ *     QSA_NOALLOC_SCRATCH_BYTES, roughly T * (n_sel + 1) * 4 bytes <= 16 MiB
+ *     (T = 4096 with n_sel = 256 fits; T = 16384 with n_sel = 512 does not).
+ *     Larger sizes return QSA_ERR_WORKSPACE_TOO_SMALL and launch nothing; call
+ *     qsa_forward with a workspace instead.  Other argument errors return the
+ *     same statuses as qsa_forward.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.  Later calls on the device reuse the address.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *   - All calls on one device share the array, and it keeps the last call's
+ *     contents; nothing in it has to start at zero, because each call overwrites
+ *     everything it later reads.  Calls whose GPU work overlaps (unordered
+ *     streams, several host threads) race on the array and produce wrong
+ *     results: order them on one stream or with events.
+ */
+#define QSA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+qsa_status_t qsa_forward_noalloc(const void* q, const void* k, const void* v, const int32_t* routes,
+                                 int64_t T, int64_t T_kv, int H, int G, int n_sel, float scale,
+                                 void* out, float* lse, qsa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
