@@ -196,6 +196,8 @@ def run_ours(args):
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
 
     wl = W.CONFIGS[args.workload]
+    if args.scale_T:
+        wl = wl.scaled(args.scale_T)
     routes_np = np.array(W.make_routes(wl), dtype=np.int32)
     q_h, k_h, v_h, do_h = W.make_tensors(wl)
     pairs = W.pair_count(routes_np, wl.T_kv)
@@ -354,6 +356,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true",
                     help="time the device-resident steps only and print the stage breakdown (profiling runs)")
     ap.add_argument("--workload", type=int, default=WORKLOAD, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--scale-T", type=int, default=0,
+                    help="run the workload's recipe at this many query rows (profiling of smaller cases)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--reference-rows", type=int, default=96)
     args = ap.parse_args()

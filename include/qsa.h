@@ -36,7 +36,12 @@
  *   - The caller owns every buffer, including the workspace (size from the
  *     matching *_workspace_size function).  The library allocates no device
  *     memory and keeps no state between calls.  The workspace contents are
- *     scratch: nothing needs to be initialised, nothing survives the call.
+ *     scratch: nothing needs to be initialised, nothing survives the call,
+ *     except the first int32 of the workspace, a status word: once the call's
+ *     work has completed on the stream it is 0, or nonzero if a kernel gave up
+ *     on a bounded wait (its outputs are then invalid).  Every wait inside the
+ *     kernels is bounded, so a fault in the pipeline ends the kernel instead of
+ *     hanging the GPU.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and the call returns without synchronising.  Route values are never
  *     read on the host.
@@ -45,7 +50,7 @@
  *     launch returns QSA_ERR_CUDA.  Route values are never errors (invalid IDs
  *     are padding).
  *   - Limits: T, T_kv, n_sel >= 1; n_sel <= 16384; T * n_sel <= 2^31 - 1;
- *     T_kv <= 2^31 - 1; H = 12 * G, G >= 1; 0 < scale < inf.
+ *     T <= 2^30; T_kv <= 2^31 - 1; H = 12 * G, G >= 1; 0 < scale < inf.
  */
 #ifndef QSA_B200_H
 #define QSA_B200_H

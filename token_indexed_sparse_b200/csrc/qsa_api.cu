@@ -19,15 +19,31 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 
 qsa_status_t check_sizes(int64_t T, int64_t T_kv, int H, int G, int n_sel) {
   if (T < 1 || T_kv < 1 || n_sel < 1 || n_sel > kMaxSel || G < 1 || H < 1) return QSA_ERR_INVALID_ARGUMENT;
-  if (T_kv > INT32_MAX || T > INT32_MAX / n_sel) return QSA_ERR_INVALID_ARGUMENT;
+  if (T_kv > INT32_MAX || T > INT32_MAX / n_sel || T > (int64_t{1} << 30)) return QSA_ERR_INVALID_ARGUMENT;
   if (H % G != 0 || H / G != qsa::kHeadsPerGroup) return QSA_ERR_UNSUPPORTED;
   if (T > INT32_MAX / G || (T_kv + 3) / 4 > INT32_MAX / G) return QSA_ERR_INVALID_ARGUMENT;
   return QSA_OK;
 }
 
+// Query phases of the dK/dV pass: each phase covers C consecutive queries, chosen
+// so that one phase's Q and dO rows (C * H * 1 KB) stay resident in L2 (48 MiB);
+// at most 64 phases.
+void dkdv_phases(int64_t T, int H, int* P, int* C) {
+  int64_t c = (int64_t{48} << 20) / (static_cast<int64_t>(H) * 1024);
+  c = c < 256 ? 256 : (c / 256) * 256;
+  int64_t p = (T + c - 1) / c;
+  if (p > 64) {
+    c = (((T + 63) / 64) + 255) / 256 * 256;
+    p = (T + c - 1) / c;
+  }
+  *P = static_cast<int>(p);
+  *C = static_cast<int>(c);
+}
+
 struct Layout {
-  size_t row_cnt = 0, row_cols = 0, quad_cnt = 0, quad_ptr = 0, quad_fill = 0, quad_ent = 0, delta = 0,
-         pds = 0, total = 0;
+  size_t status = 0, row_cnt = 0, row_cols = 0, quad_cnt = 0, quad_ptr = 0, quad_fill = 0, quad_ent = 0,
+         delta = 0, pds = 0, phase_ptr = 0, wl_cnt = 0, wl = 0, partial = 0, total = 0;
+  int P = 1, C = 1;
 };
 
 Layout make_layout(int64_t T, int64_t T_kv, int H, int G, int n_sel, bool backward) {
@@ -40,6 +56,7 @@ Layout make_layout(int64_t T, int64_t T_kv, int H, int G, int n_sel, bool backwa
   };
   const size_t nq = static_cast<size_t>((T_kv + 3) / 4);
   const size_t pairs = static_cast<size_t>(T) * static_cast<size_t>(n_sel);
+  L.status = take(4);
   L.row_cnt = take(static_cast<size_t>(T) * 4);
   L.row_cols = take(pairs * 4);
   if (backward) {
@@ -49,6 +66,11 @@ Layout make_layout(int64_t T, int64_t T_kv, int H, int G, int n_sel, bool backwa
     L.quad_ent = take(pairs * 8);
     L.delta = take(static_cast<size_t>(T) * H * 4);
     L.pds = take(pairs * G * 48);
+    dkdv_phases(T, H, &L.P, &L.C);
+    L.phase_ptr = take(nq * (L.P + 1) * 4);
+    L.wl_cnt = take(static_cast<size_t>(L.P) * 4);
+    L.wl = take(static_cast<size_t>(L.P) * nq * 16);
+    L.partial = take(nq * G * 2048 * 4);
   }
   L.total = off;
   return L;
@@ -125,12 +147,14 @@ qsa_status_t qsa_forward_ex(const void* q, const void* k, const void* v, const i
   const Layout L = make_layout(T, T_kv, H, G, n_sel, false);
   if (workspace_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* status = at<int>(workspace, L.status);
   int32_t* row_cnt = at<int32_t>(workspace, L.row_cnt);
   int32_t* row_cols = at<int32_t>(workspace, L.row_cols);
   const StageEvents ev{stage_events, n_stage_events, s};
-  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, s));
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, status, nullptr, nullptr,
+                                 nullptr, H, s));
   QSA_TRY(ev.mark(0));
-  QSA_TRY(qsa::launch_forward(q, k, v, row_cnt, row_cols, T, G, n_sel, scale, out, lse, s));
+  QSA_TRY(qsa::launch_forward(q, k, v, row_cnt, row_cols, T, G, n_sel, scale, out, lse, status, s));
   QSA_TRY(ev.mark(1));
   return QSA_OK;
 }
@@ -161,6 +185,7 @@ qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k,
   if (workspace_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t nq = (T_kv + 3) / 4;
+  int* status = at<int>(workspace, L.status);
   int32_t* row_cnt = at<int32_t>(workspace, L.row_cnt);
   int32_t* row_cols = at<int32_t>(workspace, L.row_cols);
   int32_t* quad_cnt = at<int32_t>(workspace, L.quad_cnt);
@@ -169,20 +194,29 @@ qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k,
   int64_t* quad_ent = at<int64_t>(workspace, L.quad_ent);
   float* delta = at<float>(workspace, L.delta);
   uint16_t* pds = at<uint16_t>(workspace, L.pds);
+  int32_t* phase_ptr = at<int32_t>(workspace, L.phase_ptr);
+  int32_t* wl_cnt = at<int32_t>(workspace, L.wl_cnt);
+  int4* wl = at<int4>(workspace, L.wl);
+  float* partial = at<float>(workspace, L.partial);
   const StageEvents ev{stage_events, n_stage_events, s};
   QSA_TRY(cudaMemsetAsync(quad_cnt, 0, static_cast<size_t>(nq) * 4, s));
-  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, quad_cnt, s));
+  QSA_TRY(cudaMemsetAsync(wl_cnt, 0, static_cast<size_t>(L.P) * 4, s));
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, quad_cnt, status, grad_out, out, delta,
+                                 H, s));
   QSA_TRY(ev.mark(0));
   QSA_TRY(qsa::launch_quad_scan(quad_cnt, nq, quad_ptr, quad_fill, s));
   QSA_TRY(ev.mark(1));
   QSA_TRY(qsa::launch_quad_fill(row_cnt, row_cols, T, n_sel, quad_fill, quad_ent, s));
   QSA_TRY(ev.mark(2));
-  QSA_TRY(qsa::launch_quad_sort(quad_ptr, nq, quad_ent, s));
+  QSA_TRY(qsa::launch_quad_sort(quad_ptr, nq, quad_ent, L.P, L.C, phase_ptr, s));
+  QSA_TRY(qsa::launch_quad_worklist(quad_ptr, phase_ptr, nq, T_kv, G, L.P, wl_cnt, wl, dk, dv, s));
   QSA_TRY(ev.mark(3));
-  QSA_TRY(qsa::launch_backward_dq(grad_out, q, k, v, out, lse, row_cnt, row_cols, T, G, n_sel, scale, dq, delta,
-                                  pds, s));
+  QSA_TRY(qsa::launch_backward_dq(grad_out, q, k, v, lse, delta, row_cnt, row_cols, T, G, n_sel, scale, dq, pds,
+                                  s));
   QSA_TRY(ev.mark(4));
-  QSA_TRY(qsa::launch_backward_dkdv(grad_out, q, pds, quad_ptr, quad_ent, T, T_kv, G, n_sel, scale, dk, dv, s));
+  for (int p = 0; p < L.P; ++p)
+    QSA_TRY(qsa::launch_backward_dkdv(grad_out, q, pds, quad_ent, wl_cnt, wl, p, nq, T_kv, G, n_sel, scale, partial,
+                                      dk, dv, s));
   QSA_TRY(ev.mark(5));
   return QSA_OK;
 }
@@ -190,7 +224,7 @@ qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k,
 size_t qsa_route_plan_scratch_size(int64_t T, int64_t T_kv) {
   if (T < 1 || T_kv < 1 || T_kv > INT32_MAX) return 0;
   const size_t nq = static_cast<size_t>((T_kv + 3) / 4);
-  return 2 * align256(nq * 4);
+  return 2 * align256(nq * 4) + align256(nq * 8);
 }
 
 qsa_status_t qsa_route_plan(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel, int32_t* row_cnt,
@@ -207,11 +241,13 @@ qsa_status_t qsa_route_plan(const int32_t* routes, int64_t T, int64_t T_kv, int 
   const int64_t nq = (T_kv + 3) / 4;
   int32_t* quad_cnt = static_cast<int32_t*>(scratch);
   int32_t* quad_fill = at<int32_t>(scratch, align256(static_cast<size_t>(nq) * 4));
+  int32_t* phase_ptr = at<int32_t>(scratch, 2 * align256(static_cast<size_t>(nq) * 4));
   QSA_TRY(cudaMemsetAsync(quad_cnt, 0, static_cast<size_t>(nq) * 4, s));
-  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, quad_cnt, s));
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, quad_cnt, nullptr, nullptr, nullptr,
+                                 nullptr, qsa::kHeadsPerGroup, s));
   QSA_TRY(qsa::launch_quad_scan(quad_cnt, nq, quad_ptr, quad_fill, s));
   QSA_TRY(qsa::launch_quad_fill(row_cnt, row_cols, T, n_sel, quad_fill, quad_ent, s));
-  QSA_TRY(qsa::launch_quad_sort(quad_ptr, nq, quad_ent, s));
+  QSA_TRY(qsa::launch_quad_sort(quad_ptr, nq, quad_ent, 1, static_cast<int>(T), phase_ptr, s));
   return QSA_OK;
 }
 

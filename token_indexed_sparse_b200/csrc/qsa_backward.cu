@@ -6,156 +6,178 @@
 //   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO  (dK/dV summed over heads).
 //
 // Two kernels, neither using floating-point atomics:
-//   * dq_kernel, one CTA per (query t, group g): recomputes S and dP over R_t
-//     (K/V rows gathered like the forward), forms P and dS, accumulates dQ, and
-//     stores delta and the BF16 P / dS of every routed pair (`pds`, one 48-byte
-//     record [P h0..h11 | dS h0..h11] per (t, g, position in R_t)).
+//   * dq_kernel, persistent over (query t, group g) items: recomputes S and dP
+//     over R_t (K/V rows gathered like the forward), forms P and dS with delta
+//     from the route kernel, accumulates dQ, and stores the BF16 P / dS of every
+//     routed pair (`pds`, one 48-byte record [P h0..h11 | dS h0..h11] per
+//     (t, g, position in R_t)).
 //   * dkdv_kernel, one CTA per (aligned key quad, group g): walks the quad's
 //     query list in ascending query order and accumulates dK^T = Q^T dS and
 //     dV^T = dO^T P on tensor cores.  Each warp owns 64 of the 256 dims and loads
 //     its Q / dO slices straight from global memory into A fragments, so the
 //     kernel uses no shared memory; the fixed list order makes dK/dV bitwise
 //     reproducible.
-#include "qsa_device.cuh"
 #include "qsa_internal.h"
+#include "qsa_pipe.cuh"
 
 namespace qsa {
 namespace {
 
 // ---------------------------------------------------------------------------
-// dQ (+ delta, P/dS records)
+// dQ (+ P/dS records): persistent, one CTA (8 warps) per SM
 // ---------------------------------------------------------------------------
-constexpr int kDqThreads = 128;
-constexpr int kChunk = 32;
-constexpr int kDsStride = 40;  // bf16 per row of the dS tile (80 B)
-constexpr int kTileBytes = kChunk * 512;
-constexpr int kRec = 24;       // bf16 per (t, g, key) record: 12 P + 12 dS
-constexpr int kOffDO = 16 * 512;
-constexpr int kOffK = kOffDO + 16 * 512;
-constexpr int kOffV = kOffK + 2 * kTileBytes;
-constexpr int kOffDS = kOffV + 2 * kTileBytes;
+// Same pipeline as the forward kernel (qsa_pipe.cuh): 64-key chunks of K and V
+// rows gathered two chunks ahead into a 3-stage ring of swizzled tiles (rows
+// past the end of R_t zero-filled: dQ multiplies their zero dS by their K rows).
+// Once per item the 12 Q and dO rows, the 12 LSE values and the 12 delta values
+// (delta = rowsum(dO * out), computed by the route kernel) go to one of two item
+// buffers.  Per chunk, warp w computes S = Q K^T and dP = dO V^T for keys
+// 8w..8w+7, P = exp2(S*scale*log2e - lse*log2e), dS = P (dP - delta), stores the
+// BF16 P / dS records and accumulates dQ[:, 32w:32w+32] += dS K.
+constexpr int kDqThreads = kPipeThreads;
+constexpr int kStages = 3;
+constexpr int kTile = kPipeKeys * 512;
+constexpr int kStageBytes = 2 * kTile;
+constexpr int kRec = 24;  // bf16 per (t, g, key) record: 12 P + 12 dS
+constexpr int kItemQ = 0, kItemDO = kHeadsPerGroup * 512, kItemLse = 2 * kHeadsPerGroup * 512;
+constexpr int kItemDelta = kItemLse + 64, kItemBytes = kItemDelta + 64;
+constexpr int kOffItem = kStages * kStageBytes;
+constexpr int kOffZero = kOffItem + 2 * kItemBytes;
+constexpr int kDsStride = 72;  // bf16 per dS row (144 B)
+constexpr int kOffDS = kOffZero + 512;
 constexpr int kOffRec = kOffDS + kRowTile * kDsStride * 2;
-constexpr int kOffDelta = kOffRec + kChunk * kRec * 2;
-constexpr int kOffLse = kOffDelta + kRowTile * 4;
-constexpr int kOffCols = kOffLse + kRowTile * 4;
+constexpr int kOffDesc = kOffRec + kPipeKeys * kRec * 2;
+constexpr int kSmemDq = kOffDesc + kStages * 16;
+static_assert(kSmemDq <= 232448, "shared memory per block");
+static_assert(kOffItem % 16 == 0 && kItemBytes % 16 == 0 && kOffZero % 16 == 0 && kOffDS % 16 == 0 &&
+                  kOffRec % 16 == 0 && kOffDesc % 16 == 0,
+              "alignment");
+constexpr int kFirst = 1, kLast = 2, kSlot = 4;
 
-__global__ void __launch_bounds__(kDqThreads, 2)
+__global__ void __launch_bounds__(kDqThreads, 1)
 dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ q,
           const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-          const __nv_bfloat16* __restrict__ out, const float* __restrict__ lse,
-          const int32_t* __restrict__ row_cnt, const int32_t* __restrict__ row_cols, int G, int n_sel,
-          float scale, float scale_log2, __nv_bfloat16* __restrict__ dq, float* __restrict__ delta_out,
-          uint16_t* __restrict__ pds) {
-  extern __shared__ __align__(128) uint8_t smem[];
+          const float* __restrict__ lse, const float* __restrict__ delta, const int32_t* __restrict__ row_cnt,
+          const int32_t* __restrict__ row_cols, int64_t n_items, int G, int n_sel, float scale, float scale_log2,
+          __nv_bfloat16* __restrict__ dq, uint16_t* __restrict__ pds) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, cq = lane & 3, mi = lane >> 3;
+  const int H = G * kHeadsPerGroup;
+  int4* desc = reinterpret_cast<int4*>(smem + kOffDesc);
   __nv_bfloat16* sDS = reinterpret_cast<__nv_bfloat16*>(smem + kOffDS);
   uint16_t* sRec = reinterpret_cast<uint16_t*>(smem + kOffRec);
-  float* sDelta = reinterpret_cast<float*>(smem + kOffDelta);
-  float* sLse = reinterpret_cast<float*>(smem + kOffLse);
-  int32_t* sCols = reinterpret_cast<int32_t*>(smem + kOffCols);
+  const uint32_t sDSa = smem_u32(sDS);
+  if (tid < 32) reinterpret_cast<uint4*>(smem + kOffZero)[tid] = make_uint4(0, 0, 0, 0);
 
-  const int H = G * kHeadsPerGroup;
-  const int64_t t = blockIdx.x / G;
-  const int g = static_cast<int>(blockIdx.x - t * G);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, cq = lane & 3;
-  const int cnt = row_cnt[t];
-  const int64_t qrow0 = t * H + g * kHeadsPerGroup;
-
-  if (cnt == 0) {  // padding query: dQ = 0, nothing else is read later
-    uint4* o = reinterpret_cast<uint4*>(dq + qrow0 * kHeadDim);
-    for (int i = tid; i < kHeadsPerGroup * 32; i += kDqThreads) o[i] = make_uint4(0, 0, 0, 0);
-    if (tid < kHeadsPerGroup) delta_out[qrow0 + tid] = 0.f;
-    return;
-  }
-
-  for (int i = tid; i < cnt; i += kDqThreads) sCols[i] = row_cols[t * n_sel + i];
-  const uint32_t sQa = smem_u32(smem), sDOa = smem_u32(smem + kOffDO);
-  const uint32_t sKa = smem_u32(smem + kOffK), sVa = smem_u32(smem + kOffV);
-  for (int i = tid; i < 2 * kRowTile * 32; i += kDqThreads) {
-    const int tensor = i >> 9, r = (i >> 5) & 15, c = i & 31;
-    const bool ok = r < kHeadsPerGroup;
-    const __nv_bfloat16* src = (tensor ? dout : q) + (qrow0 + (ok ? r : 0)) * kHeadDim + c * 8;
-    cp_async16((tensor ? sDOa : sQa) + swz512(r, c), src, ok);
-  }
-  cp_async_commit();
-  if (tid < kRowTile) sLse[tid] = tid < kHeadsPerGroup ? lse[qrow0 + tid] * kLog2e : INFINITY;
-  __syncthreads();
-
-  const int n_chunks = (cnt + kChunk - 1) / kChunk;
-  auto issue = [&](int ch) {
-    const int stage = ch & 1, base = ch * kChunk;
-    const int nk = min(kChunk, cnt - base);
-#pragma unroll 4
-    for (int i = tid; i < 2 * kChunk * 32; i += kDqThreads) {
-      const int tensor = i / (kChunk * 32);
-      const int r = (i >> 5) & (kChunk - 1), c = i & 31;
-      const bool ok = r < nk;
-      const int64_t key = ok ? sCols[base + r] : 0;
-      const __nv_bfloat16* src = (tensor ? v : k) + (key * G + g) * kHeadDim + c * 8;
-      cp_async16((tensor ? sVa : sKa) + stage * kTileBytes + swz512(r, c), src, ok);
+  Cursor cur;
+  cursor_init(cur, row_cnt, n_items, G);
+  int32_t key[8];
+  cursor_keys(key, cur, n_items, G, row_cols, n_sel);
+  int islot = 0;  // item buffer of the next non-empty item
+  auto issue = [&](int stage) {
+    const uint32_t st = sbase + stage * kStageBytes;
+    if (cur.it < n_items) {
+      const int64_t t = cur.it / G;
+      const int g = static_cast<int>(cur.it - t * G);
+      const int nk = cursor_nk(cur, n_items);
+      int flags = (cur.ch == 0 ? kFirst : 0) | (cur.ch == cur.nch - 1 ? kLast : 0);
+      if (nk > 0) {
+        gather_rows(st, st + kTile, k, v, key, g, G, nk);
+        if (cur.ch == 0) {
+          const int64_t qrow0 = t * H + g * kHeadsPerGroup;
+          const uint32_t ib = sbase + kOffItem + islot * kItemBytes;
+          gather_heads(ib + kItemQ, q + qrow0 * kHeadDim);
+          gather_heads(ib + kItemDO, dout + qrow0 * kHeadDim);
+          const int j = tid - kHeadsPerGroup * 16;  // threads 192..197
+          if (j >= 0 && j < 3) cp_async16(ib + kItemLse + 16 * j, lse + qrow0 + 4 * j, true);
+          if (j >= 3 && j < 6) cp_async16(ib + kItemDelta + 16 * (j - 3), delta + qrow0 + 4 * (j - 3), true);
+          flags |= islot ? kSlot : 0;
+          islot ^= 1;
+        } else {
+          flags |= islot ? 0 : kSlot;  // the item's slot was flipped at its first chunk
+        }
+      }
+      if (tid == 0) desc[stage] = make_int4(static_cast<int>(t), g, nk, flags | ((cur.ch) << 3));
+    } else if (tid == 0) {
+      desc[stage] = make_int4(0, 0, -1, 0);
     }
+    cp_async_commit();
+    cursor_next(cur, row_cnt, n_items, G);
+    cursor_keys(key, cur, n_items, G, row_cols, n_sel);
   };
   issue(0);
-  cp_async_commit();
-  if (n_chunks > 1) issue(1);
-  cp_async_commit();
-  cp_async_wait<2>();  // Q and dO tiles have landed
-  __syncthreads();
-
-  // delta = rowsum(dO * out) in fp32 from the BF16 forward output; warp w owns rows 3w..3w+2.
-  for (int r = warp * 3; r < warp * 3 + 3; ++r) {
-    const uint4 ov = *reinterpret_cast<const uint4*>(out + (qrow0 + r) * kHeadDim + lane * 8);
-    uint4 dv;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n"
-                 : "=r"(dv.x), "=r"(dv.y), "=r"(dv.z), "=r"(dv.w) : "r"(sDOa + swz512(r, lane)));
-    float acc = bf16_lo(ov.x) * bf16_lo(dv.x) + bf16_hi(ov.x) * bf16_hi(dv.x) +
-                bf16_lo(ov.y) * bf16_lo(dv.y) + bf16_hi(ov.y) * bf16_hi(dv.y) +
-                bf16_lo(ov.z) * bf16_lo(dv.z) + bf16_hi(ov.z) * bf16_hi(dv.z) +
-                bf16_lo(ov.w) * bf16_lo(dv.w) + bf16_hi(ov.w) * bf16_hi(dv.w);
-    acc = warp_sum(acc);
-    if (lane == 0) {
-      sDelta[r] = acc;
-      delta_out[qrow0 + r] = acc;
-    }
-  }
-  if (tid < kRowTile - kHeadsPerGroup) sDelta[kHeadsPerGroup + tid] = 0.f;
+  issue(1);
 
   uint32_t qa[16][4], da[16][4];
-#pragma unroll
-  for (int ks = 0; ks < 16; ++ks) {
-    const int mi = lane >> 3;
-    const uint32_t off = swz512(((mi & 1) << 3) + (lane & 7), 2 * ks + (mi >> 1));
-    ldsm_x4(qa[ks], sQa + off);
-    ldsm_x4(da[ks], sDOa + off);
-  }
-  __syncthreads();  // sDelta
-  const float dl0 = sDelta[gq], dl1 = sDelta[gq + 8];
-  const float ls0 = sLse[gq], ls1 = sLse[gq + 8];
+  float acc[4][4];
+  float ls0 = INFINITY, ls1 = INFINITY, dl0 = 0.f, dl1 = 0.f;
 
-  float acc[8][4];
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-  const uint32_t sDSa = smem_u32(sDS);
-  uint16_t* pds_row = pds + (t * G + g) * static_cast<int64_t>(n_sel) * kRec;
-
-  for (int ch = 0; ch < n_chunks; ++ch) {
-    const int stage = ch & 1, base = ch * kChunk;
-    const int nk = min(kChunk, cnt - base);
+  for (int c = 0;; ++c) {
+    const int stage = c % kStages;
+    const uint32_t st = sbase + stage * kStageBytes;
     cp_async_wait<1>();
-    __syncthreads();
-
-    float s[4] = {0.f, 0.f, 0.f, 0.f}, dp[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t kb = sKa + stage * kTileBytes, vb = sVa + stage * kTileBytes;
-#pragma unroll
-    for (int ks = 0; ks < 16; ks += 2) {
-      uint32_t b[4], c[4];
-      const uint32_t off = swz512(warp * 8 + (lane & 7), 2 * ks + (lane >> 3));
-      ldsm_x4(b, kb + off);
-      ldsm_x4(c, vb + off);
-      mma_16816(s, qa[ks], b[0], b[1]);
-      mma_16816(s, qa[ks + 1], b[2], b[3]);
-      mma_16816(dp, da[ks], c[0], c[1]);
-      mma_16816(dp, da[ks + 1], c[2], c[3]);
+    __syncthreads();  // chunk c has landed; every warp is done with chunk c - 1
+    const int4 d = desc[stage];
+    const int nk = d.z;
+    if (nk < 0) break;
+    const int64_t t = d.x;
+    const int g = d.y;
+    const int64_t qrow0 = t * H + g * kHeadsPerGroup;
+    if (nk == 0) {  // padding query: dQ = 0 (no item buffer is used)
+      issue((c + 2) % kStages);
+      uint4* orow = reinterpret_cast<uint4*>(dq + qrow0 * kHeadDim);
+      for (int i = tid; i < kHeadsPerGroup * 32; i += kDqThreads) orow[i] = make_uint4(0, 0, 0, 0);
+      continue;
     }
+    if (d.w & kFirst) {
+      const uint32_t ib = sbase + kOffItem + ((d.w & kSlot) ? kItemBytes : 0);
+#pragma unroll
+      for (int ks = 0; ks < 16; ++ks) {
+        const int r = ((mi & 1) << 3) + (lane & 7);
+        const int cc = 2 * ks + (mi >> 1);
+        const bool real = r < kHeadsPerGroup;
+        ldsm_x4(qa[ks], real ? ib + kItemQ + swz512(r, cc) : sbase + kOffZero + (cc << 4));
+        ldsm_x4(da[ks], real ? ib + kItemDO + swz512(r, cc) : sbase + kOffZero + (cc << 4));
+      }
+      const float* il = reinterpret_cast<const float*>(smem + (ib - sbase) + kItemLse);
+      const float* idl = reinterpret_cast<const float*>(smem + (ib - sbase) + kItemDelta);
+      ls0 = il[gq] * kLog2e;
+      dl0 = idl[gq];
+      ls1 = gq + 8 < kHeadsPerGroup ? il[gq + 8] * kLog2e : INFINITY;
+      dl1 = gq + 8 < kHeadsPerGroup ? idl[gq + 8] : 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+    }
+    // S = Q K^T and dP = dO V^T for this warp's 8 keys, two chains each
+    float s[4], dp[4];
+    {
+      float sa[2][4], pa[2][4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sa[j][i] = pa[j][i] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < 16; ks += 2) {
+        uint32_t b[4], e[4];
+        const uint32_t off = swz512(warp * 8 + (lane & 7), 2 * ks + mi);
+        ldsm_x4(b, st + off);
+        ldsm_x4(e, st + kTile + off);
+        mma_16816(sa[(ks >> 1) & 1], qa[ks], b[0], b[1]);
+        mma_16816(pa[(ks >> 1) & 1], da[ks], e[0], e[1]);
+        mma_16816(sa[(ks >> 1) & 1], qa[ks + 1], b[2], b[3]);
+        mma_16816(pa[(ks >> 1) & 1], da[ks + 1], e[2], e[3]);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        s[i] = sa[0][i] + sa[1][i];
+        dp[i] = pa[0][i] + pa[1][i];
+      }
+    }
+    __syncthreads();  // every warp has read this item's buffer: its slot may be refilled
+    issue((c + 2) % kStages);
+
     const int key0 = warp * 8 + 2 * cq;
     const bool v0 = key0 < nk, v1 = key0 + 1 < nk;
     const float p0 = v0 ? exp2f(s[0] * scale_log2 - ls0) : 0.f;
@@ -179,189 +201,288 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
       sRec[(key0 + 1) * kRec + 20 + gq] = static_cast<uint16_t>(D23 >> 16);
     }
     __syncthreads();
-
-    // records of this chunk: nk * 48 contiguous bytes
     {
+      const int base = (d.w >> 3) * kPipeKeys;
       const uint4* src = reinterpret_cast<const uint4*>(sRec);
-      uint4* dst = reinterpret_cast<uint4*>(pds_row + static_cast<int64_t>(base) * kRec);
+      uint4* dst = reinterpret_cast<uint4*>(pds + ((t * G + g) * n_sel + base) * kRec);
       for (int i = tid; i < nk * 3; i += kDqThreads) dst[i] = src[i];
     }
-    // dQ[:, 64w:64w+64] += dS K
+    // dQ[:, 32w:32w+32] += dS K over the chunk's 64 keys
 #pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
+    for (int ks = 0; ks < 4; ++ks) {
       uint32_t a[4];
-      const int mi = lane >> 3;
       ldsm_x4(a, sDSa + (((((mi & 1) << 3) + (lane & 7)) * kDsStride + 16 * ks + ((mi >> 1) << 3)) << 1));
 #pragma unroll
-      for (int nt = 0; nt < 8; nt += 2) {
+      for (int nt = 0; nt < 4; nt += 2) {
         uint32_t b[4];
-        ldsm_x4_t(b, kb + swz512(16 * ks + ((mi & 1) << 3) + (lane & 7), warp * 8 + nt + (mi >> 1)));
+        ldsm_x4_t(b, st + swz512(16 * ks + ((mi & 1) << 3) + (lane & 7), warp * 4 + nt + (mi >> 1)));
         mma_16816(acc[nt], a, b[0], b[1]);
         mma_16816(acc[nt + 1], a, b[2], b[3]);
       }
     }
-    __syncthreads();
-    if (ch + 2 < n_chunks) issue(ch + 2);
-    cp_async_commit();
+    if (d.w & kLast) {
+      __nv_bfloat16* drow = dq + qrow0 * kHeadDim;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const int dim = warp * 32 + nt * 8 + 2 * cq;
+        *reinterpret_cast<uint32_t*>(drow + gq * kHeadDim + dim) = pack_bf16(acc[nt][0] * scale, acc[nt][1] * scale);
+        if (gq + 8 < kHeadsPerGroup)
+          *reinterpret_cast<uint32_t*>(drow + (gq + 8) * kHeadDim + dim) =
+              pack_bf16(acc[nt][2] * scale, acc[nt][3] * scale);
+      }
+    }
   }
   cp_async_wait<0>();
-
-  __nv_bfloat16* drow = dq + qrow0 * kHeadDim;
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    const int dim = warp * 64 + nt * 8 + 2 * cq;
-    *reinterpret_cast<uint32_t*>(drow + gq * kHeadDim + dim) = pack_bf16(acc[nt][0] * scale, acc[nt][1] * scale);
-    if (gq + 8 < kHeadsPerGroup)
-      *reinterpret_cast<uint32_t*>(drow + (gq + 8) * kHeadDim + dim) =
-          pack_bf16(acc[nt][2] * scale, acc[nt][3] * scale);
-  }
 }
 
 // ---------------------------------------------------------------------------
-// dK / dV per key quad
+// dK / dV per key quad, one query phase per launch
 // ---------------------------------------------------------------------------
-constexpr int kKvThreads = 128;
-constexpr int kUnroll = 4;  // entries in flight per warp
+// Work item = (quad b, group g, entries [lo, hi) of b's ascending query list that
+// fall in the launch's query phase).  Items are dealt round-robin to persistent
+// CTAs (8 warps); each item's entries flow in chunks of 4 through a 4-stage ring:
+// all 12 Q rows and 12 dO rows of each entry (whole 512-byte rows, cp.async,
+// swizzled) and the entry's P/dS records placed by key slot (absent keys and
+// missing entries zero-filled).  Warp w owns dims [32w, 32w+32) and accumulates
+// dK^T += Q^T dS and dV^T += dO^T P with mma.sync: the A fragments come from
+// ldmatrix.trans of the staged rows and the K dimension packs head rows of
+// different entries of the same quad: k-step 0 = heads 0..7 of entries 0 and 1,
+// k-step 1 = the same for entries 2 and 3, k-step 2 = heads 8..11 of all four,
+// so no MMA slot or shared-memory read is spent on padding heads.  An item
+// starts from zero or from the FP32 partial of the previous phase and ends with
+// a partial or, on its last range, the BF16 result: the summation order is the
+// fixed list order, so dK/dV are bitwise reproducible.
+constexpr int kKvThreads = 256;
+constexpr int kKvStages = 4;
+constexpr int kEnt = 4;                                   // entries per chunk
+constexpr int kKvRows = kEnt * 2 * kHeadsPerGroup;        // 96 staged rows per chunk
+constexpr int kKvRecOff = kKvRows * 512;                  // records after the rows
+constexpr int kKvRecBytes = kEnt * 4 * kRec * 2;          // 4 entries x 4 key slots x 48 B
+constexpr int kKvStageBytes = kKvRecOff + kKvRecBytes;
+constexpr int kKvOffDesc = kKvStages * kKvStageBytes;
+constexpr int kKvSmem = kKvOffDesc + kKvStages * 16;
+static_assert(kKvSmem <= 232448, "shared memory per block");
+static_assert(kKvStageBytes % 128 == 0, "alignment");
+constexpr int kItemFirst = 1, kItemLast = 2, kChFirst = 4, kChLast = 8;
 
-// Loads this thread's slice of one query's 12 head rows for the A operand of
-// X^T (dims x heads): rows {2c, 2c+1, 2c+8, 2c+9} (rows >= 12 are zero), dims
-// [4g, 4g+4) and [32+4g, 32+4g+4) of the warp's 64-dim slice.
-struct RowSlice {
-  uint2 x[4], y[4];
+struct KvCursor {
+  int64_t w;        // work index (item = w / G, g = w % G); >= n_work when exhausted
+  int4 item;        // (quad, lo, hi, flags) of the current work index
+  int4 item_next;   // of the next one (prefetched)
+  int ch, nch;
 };
-__device__ __forceinline__ void load_slice(RowSlice& r, const __nv_bfloat16* base, int gq, int cq, bool live) {
-  const int rows[4] = {2 * cq, 2 * cq + 1, 2 * cq + 8, 2 * cq + 9};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (live && rows[i] < kHeadsPerGroup) {
-      const __nv_bfloat16* p = base + rows[i] * kHeadDim + 4 * gq;
-      r.x[i] = __ldg(reinterpret_cast<const uint2*>(p));
-      r.y[i] = __ldg(reinterpret_cast<const uint2*>(p + 32));
-    } else {
-      r.x[i] = make_uint2(0, 0);
-      r.y[i] = make_uint2(0, 0);
-    }
-  }
-}
-// A fragment of m-tile mt (dims 4g+mt and 32+4g+mt; k = head rows).
-__device__ __forceinline__ void slice_frag(uint32_t (&a)[4], const RowSlice& r, int mt) {
-  const uint32_t sel = (mt & 1) ? kHiHi : kLoLo;
-  const bool hiw = mt >= 2;
-  a[0] = prmt(hiw ? r.x[0].y : r.x[0].x, hiw ? r.x[1].y : r.x[1].x, sel);
-  a[1] = prmt(hiw ? r.y[0].y : r.y[0].x, hiw ? r.y[1].y : r.y[1].x, sel);
-  a[2] = prmt(hiw ? r.x[2].y : r.x[2].x, hiw ? r.x[3].y : r.x[3].x, sel);
-  a[3] = prmt(hiw ? r.y[2].y : r.y[2].x, hiw ? r.y[3].y : r.y[3].x, sel);
+
+__device__ __forceinline__ int4 kv_item(const int4* wl, int64_t w, int64_t n_work, int G) {
+  return w < n_work ? __ldg(wl + w / G) : make_int4(0, 0, 0, 0);
 }
 
-__global__ void __launch_bounds__(kKvThreads)
+__global__ void __launch_bounds__(kKvThreads, 1)
 dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ q,
-            const uint16_t* __restrict__ pds, const int32_t* __restrict__ quad_ptr,
-            const int64_t* __restrict__ quad_ent, int64_t T_kv, int G, int n_sel, float scale,
-            __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv) {
+            const uint16_t* __restrict__ pds, const int64_t* __restrict__ quad_ent,
+            const int32_t* __restrict__ wl_cnt, const int4* __restrict__ wl, int64_t T_kv, int G, int n_sel,
+            float scale, float* __restrict__ partial, __nv_bfloat16* __restrict__ dk,
+            __nv_bfloat16* __restrict__ dv) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, cq = lane & 3, mat = lane >> 3, rr = lane & 7;
   const int H = G * kHeadsPerGroup;
-  const int64_t b = blockIdx.x / G;
-  const int g = static_cast<int>(blockIdx.x - b * G);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, cq = lane & 3;
-  const int e0 = quad_ptr[b], e1 = quad_ptr[b + 1];
+  int4* desc = reinterpret_cast<int4*>(smem + kKvOffDesc);
+  const int64_t n_work = static_cast<int64_t>(__ldg(wl_cnt)) * G;
 
-  float ak[4][4], av[4][4];
+  KvCursor cur;
+  cur.w = blockIdx.x;
+  cur.item = kv_item(wl, cur.w, n_work, G);
+  cur.item_next = kv_item(wl, cur.w + gridDim.x, n_work, G);
+  cur.ch = 0;
+  cur.nch = (cur.item.z - cur.item.y + kEnt - 1) / kEnt;
+  int64_t ent[kEnt];
+  auto load_ents = [&]() {
+    const int e0 = cur.item.y + cur.ch * kEnt;
 #pragma unroll
-  for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) ak[mt][j] = av[mt][j] = 0.f;
+    for (int u = 0; u < kEnt; ++u) ent[u] = (cur.w < n_work && e0 + u < cur.item.z) ? __ldg(quad_ent + e0 + u) : -1;
+  };
+  load_ents();
+  // ent[u] for a runtime u without dynamic register indexing
+  auto ent_at = [&](int u) { return u == 0 ? ent[0] : u == 1 ? ent[1] : u == 2 ? ent[2] : ent[3]; };
 
-  for (int base = e0; base < e1; base += 32) {
-    const int64_t my_ent = base + lane < e1 ? quad_ent[base + lane] : -1;
-    const int n_here = min(32, e1 - base);
-    for (int u0 = 0; u0 < n_here; u0 += kUnroll) {
-      RowSlice sq[kUnroll], sd[kUnroll];
-      uint32_t pb[kUnroll][2], sb[kUnroll][2];
+  auto issue = [&](int stage) {
+    const uint32_t st = sbase + stage * kKvStageBytes;
+    if (cur.w < n_work) {
+      const int g = static_cast<int>(cur.w % G);
+      const int n_ent = min(kEnt, cur.item.z - (cur.item.y + cur.ch * kEnt));
+      // rows: index i = u * 24 + tensor * 12 + head; warp w copies the 12 rows
+      // (one contiguous 6 KB block) of entry w / 2, tensor w % 2
+      {
+        const int u = warp >> 1, tn = warp & 1;
+        const int64_t eu = ent_at(u);
+        const int64_t t = eu >= 0 ? (eu >> 32) : 0;
+        const __nv_bfloat16* src = (tn ? dout : q) + ((t * H + g * kHeadsPerGroup) * kHeadDim + lane * 8);
+        const int i0 = u * 24 + tn * kHeadsPerGroup;
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t ent = __shfl_sync(0xffffffffu, my_ent, (u0 + u) & 31);
-        const bool live = u0 + u < n_here;
-        const int64_t t = live ? (ent >> 32) : 0;
-        const int i0 = static_cast<int>((ent >> 4) & 0x0fffffff);
-        const int mask = static_cast<int>(ent & 15);
-        const int64_t row0 = (t * H + g * kHeadsPerGroup) * kHeadDim + warp * 64;
-        load_slice(sq[u], q + row0, gq, cq, live);
-        load_slice(sd[u], dout + row0, gq, cq, live);
-        pb[u][0] = pb[u][1] = sb[u][0] = sb[u][1] = 0u;
-        if (live && gq < 4 && ((mask >> gq) & 1)) {
-          const int idx = i0 + __popc(mask & ((1 << gq) - 1));
-          const uint16_t* rec = pds + ((t * G + g) * n_sel + idx) * kRec;
-          pb[u][0] = __ldg(reinterpret_cast<const uint32_t*>(rec + 2 * cq));
-          sb[u][0] = __ldg(reinterpret_cast<const uint32_t*>(rec + 12 + 2 * cq));
-          if (cq < 2) {
-            pb[u][1] = __ldg(reinterpret_cast<const uint32_t*>(rec + 8 + 2 * cq));
-            sb[u][1] = __ldg(reinterpret_cast<const uint32_t*>(rec + 20 + 2 * cq));
+        for (int h = 0; h < kHeadsPerGroup; ++h)
+          cp_async16(st + swz512(i0 + h, lane), src + h * kHeadDim, u < n_ent);
+      }
+      // records: thread -> (entry u, key slot, 16-byte part)
+      if (tid < kEnt * 4 * 3) {
+        const int u = tid / 12, slot = (tid / 3) & 3, part = tid % 3;
+        const int64_t e = ent_at(u);
+        const int mask = static_cast<int>(e & 15);
+        const bool live = u < n_ent && ((mask >> slot) & 1);
+        const int64_t t = live ? (e >> 32) : 0;
+        const int i0 = static_cast<int>((e >> 4) & 0x0fffffff);
+        const int idx = live ? i0 + __popc(mask & ((1 << slot) - 1)) : 0;
+        const uint16_t* src = pds + ((t * G + g) * n_sel + idx) * kRec + part * 8;
+        cp_async16(st + kKvRecOff + (u * 4 + slot) * (kRec * 2) + part * 16, src, live);
+      }
+      if (tid == 0) {
+        const int fl = (cur.item.w & 3) | (cur.ch == 0 ? kChFirst : 0) | (cur.ch == cur.nch - 1 ? kChLast : 0);
+        desc[stage] = make_int4(cur.item.x, g, n_ent, fl);
+      }
+    } else if (tid == 0) {
+      desc[stage] = make_int4(0, 0, -1, 0);
+    }
+    cp_async_commit();
+    // advance
+    if (cur.w < n_work && ++cur.ch == cur.nch) {
+      cur.w += gridDim.x;
+      cur.item = cur.item_next;
+      cur.item_next = kv_item(wl, cur.w + gridDim.x, n_work, G);
+      cur.ch = 0;
+      cur.nch = (cur.item.z - cur.item.y + kEnt - 1) / kEnt;
+    }
+    load_ents();
+  };
+  issue(0);
+  issue(1);
+  issue(2);
+
+  float ak[2][4], av[2][4];
+  for (int c = 0;; ++c) {
+    const int stage = c % kKvStages;
+    const uint32_t st = sbase + stage * kKvStageBytes;
+    cp_async_wait<2>();
+    __syncthreads();  // chunk c has landed; every warp is done with chunk c - 1
+    const int4 d = desc[stage];
+    issue((c + 3) % kKvStages);
+    if (d.z < 0) break;
+    const int64_t b = d.x;
+    const int g = d.y;
+    const int fl = d.w;
+    float* part = partial + ((b * G + g) * 128 + warp * 16 + gq * 2 + (cq & 1)) * 16;
+    if (fl & kChFirst) {
+      if ((fl & kItemFirst) || cq >= 2) {
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) ak[mt][i] = av[mt][i] = 0.f;
+      } else {
+        const float4* src = reinterpret_cast<const float4*>(part);
+        const float4 x0 = src[0], x1 = src[1], x2 = src[2], x3 = src[3];
+        ak[0][0] = x0.x; ak[0][1] = x0.y; ak[0][2] = x0.z; ak[0][3] = x0.w;
+        ak[1][0] = x1.x; ak[1][1] = x1.y; ak[1][2] = x1.z; ak[1][3] = x1.w;
+        av[0][0] = x2.x; av[0][1] = x2.y; av[0][2] = x2.z; av[0][3] = x2.w;
+        av[1][0] = x3.x; av[1][1] = x3.y; av[1][2] = x3.z; av[1][3] = x3.w;
+      }
+    }
+#pragma unroll
+    for (int ks = 0; ks < 3; ++ks) {
+      // B fragments: P (dV) and dS (dK) of key slot gq for the k-step's head slots
+      uint32_t pb0 = 0, pb1 = 0, sb0 = 0, sb1 = 0;
+      if (gq < 4) {
+        int u0, u1, wp;
+        if (ks < 2) {
+          u0 = 2 * ks;
+          u1 = 2 * ks + 1;
+          wp = cq;
+        } else {
+          u0 = cq >> 1;
+          u1 = 2 + (cq >> 1);
+          wp = 4 + (cq & 1);
+        }
+        const uint32_t r0 = st + kKvRecOff + (u0 * 4 + gq) * (kRec * 2);
+        const uint32_t r1 = st + kKvRecOff + (u1 * 4 + gq) * (kRec * 2);
+        asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(pb0) : "r"(r0 + wp * 4));
+        asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(pb1) : "r"(r1 + wp * 4));
+        asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(sb0) : "r"(r0 + (6 + wp) * 4));
+        asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(sb1) : "r"(r1 + (6 + wp) * 4));
+      }
+      // A fragments: this lane addresses row (entry, head) of matrix `mat`
+      int u, h;
+      if (ks < 2) {
+        u = 2 * ks + (mat >> 1);
+        h = rr;
+      } else {
+        u = 2 * (mat >> 1) + (rr >> 2);
+        h = 8 + (rr & 3);
+      }
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const int dch = warp * 4 + mt * 2 + (mat & 1);
+        uint32_t aq[4], ad[4];
+        ldsm_x4_t(aq, st + swz512(u * 24 + h, dch));
+        ldsm_x4_t(ad, st + swz512(u * 24 + kHeadsPerGroup + h, dch));
+        mma_16816(ak[mt], aq, sb0, sb1);
+        mma_16816(av[mt], ad, pb0, pb1);
+      }
+    }
+    if ((fl & kChLast) && cq < 2) {
+      if (fl & kItemLast) {
+        // C fragment of m-tile mt: (dim 32w+16mt+g | +8, key 2c | 2c+1)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int64_t key = 4 * b + 2 * cq + j;
+          if (key < T_kv) {
+            __nv_bfloat16* rk = dk + (key * G + g) * kHeadDim + warp * 32 + gq;
+            __nv_bfloat16* rv = dv + (key * G + g) * kHeadDim + warp * 32 + gq;
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+              rk[16 * mt] = __float2bfloat16_rn(ak[mt][j] * scale);
+              rk[16 * mt + 8] = __float2bfloat16_rn(ak[mt][2 + j] * scale);
+              rv[16 * mt] = __float2bfloat16_rn(av[mt][j]);
+              rv[16 * mt + 8] = __float2bfloat16_rn(av[mt][2 + j]);
+            }
           }
         }
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
-          uint32_t a[4];
-          slice_frag(a, sq[u], mt);
-          mma_16816(ak[mt], a, sb[u][0], sb[u][1]);
-          slice_frag(a, sd[u], mt);
-          mma_16816(av[mt], a, pb[u][0], pb[u][1]);
-        }
+      } else {
+        float4* dst = reinterpret_cast<float4*>(part);
+        dst[0] = make_float4(ak[0][0], ak[0][1], ak[0][2], ak[0][3]);
+        dst[1] = make_float4(ak[1][0], ak[1][1], ak[1][2], ak[1][3]);
+        dst[2] = make_float4(av[0][0], av[0][1], av[0][2], av[0][3]);
+        dst[3] = make_float4(av[1][0], av[1][1], av[1][2], av[1][3]);
       }
     }
   }
-
-  // C fragment: (dim 4g+mt | 32+4g+mt, key 2c | 2c+1) of the warp's slice; keys 0..3 valid.
-  if (cq < 2) {
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int64_t key = 4 * b + 2 * cq + j;
-      if (key >= T_kv) continue;
-      const int64_t off = (key * G + g) * kHeadDim + warp * 64 + 4 * gq;
-      uint2 wk, wv;
-      wk.x = pack_bf16(ak[0][j] * scale, ak[1][j] * scale);
-      wk.y = pack_bf16(ak[2][j] * scale, ak[3][j] * scale);
-      wv.x = pack_bf16(av[0][j], av[1][j]);
-      wv.y = pack_bf16(av[2][j], av[3][j]);
-      *reinterpret_cast<uint2*>(dk + off) = wk;
-      *reinterpret_cast<uint2*>(dv + off) = wv;
-      wk.x = pack_bf16(ak[0][2 + j] * scale, ak[1][2 + j] * scale);
-      wk.y = pack_bf16(ak[2][2 + j] * scale, ak[3][2 + j] * scale);
-      wv.x = pack_bf16(av[0][2 + j], av[1][2 + j]);
-      wv.y = pack_bf16(av[2][2 + j], av[3][2 + j]);
-      *reinterpret_cast<uint2*>(dk + off + 32) = wk;
-      *reinterpret_cast<uint2*>(dv + off + 32) = wv;
-    }
-  }
+  cp_async_wait<0>();
 }
 
 }  // namespace
 
 cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* k, const void* v,
-                               const void* out, const float* lse, const int32_t* row_cnt,
+                               const float* lse, const float* delta, const int32_t* row_cnt,
                                const int32_t* row_cols, int64_t T, int G, int n_sel, float scale, void* dq,
-                               float* delta, uint16_t* pds, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(kOffCols) + static_cast<size_t>(n_sel) * 4;
-  cudaError_t e = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+                               uint16_t* pds, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDq);
   if (e != cudaSuccess) return e;
-  dq_kernel<<<static_cast<unsigned>(T * G), kDqThreads, smem, s>>>(
+  const int64_t n_items = T * G;
+  const int64_t grid = n_items < sm_count() ? n_items : sm_count();
+  dq_kernel<<<static_cast<unsigned>(grid), kDqThreads, kSmemDq, s>>>(
       static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q),
-      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
-      static_cast<const __nv_bfloat16*>(out), lse, row_cnt, row_cols, G, n_sel, scale, scale * kLog2e,
-      static_cast<__nv_bfloat16*>(dq), delta, pds);
+      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), lse, delta, row_cnt, row_cols,
+      n_items, G, n_sel, scale, scale * kLog2e, static_cast<__nv_bfloat16*>(dq), pds);
   return cudaGetLastError();
 }
 
-cudaError_t launch_backward_dkdv(const void* grad_out, const void* q, const uint16_t* pds,
-                                 const int32_t* quad_ptr, const int64_t* quad_ent, int64_t T, int64_t T_kv,
-                                 int G, int n_sel, float scale, void* dk, void* dv, cudaStream_t s) {
-  (void)T;
-  const int64_t n_quads = (T_kv + 3) / 4;
-  dkdv_kernel<<<static_cast<unsigned>(n_quads * G), kKvThreads, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q), pds, quad_ptr,
-      quad_ent, T_kv, G, n_sel, scale, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+cudaError_t launch_backward_dkdv(const void* grad_out, const void* q, const uint16_t* pds, const int64_t* quad_ent,
+                                 const int32_t* wl_cnt, const int4* wl, int p, int64_t n_quads, int64_t T_kv,
+                                 int G, int n_sel, float scale, float* partial, void* dk, void* dv,
+                                 cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
+  if (e != cudaSuccess) return e;
+  dkdv_kernel<<<static_cast<unsigned>(sm_count()), kKvThreads, kKvSmem, s>>>(
+      static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q), pds, quad_ent, wl_cnt + p,
+      wl + static_cast<int64_t>(p) * n_quads, T_kv, G, n_sel, scale, partial, static_cast<__nv_bfloat16*>(dk),
+      static_cast<__nv_bfloat16*>(dv));
   return cudaGetLastError();
 }
 

@@ -1,123 +1,133 @@
-// QSA forward: one CTA per (query token t, KV group g).
+// QSA forward: persistent, one CTA (8 warps) per SM.
 //
-// Computes, for the 12 query heads of group g, the softmax attention of
-// "Query Sparse Attention (QSA)" (cuDNN-Frontend page, "Selection and
-// components": scaled QK over the selected keys, online softmax, PV, FP32
-// output cast to BF16, natural-log LSE; empty rows give zero output and -inf
-// LSE) over the row's de-duplicated route set R_t.
+// Computes, for the 12 query heads of every (query token t, KV group g), the
+// softmax attention of the cuDNN-Frontend "Query Sparse Attention (QSA)" page
+// ("Selection and components": scaled QK over the selected keys, online softmax,
+// PV, FP32 output cast to BF16, natural-log LSE; empty rows give zero output and
+// -inf LSE) over the row's de-duplicated route set R_t.
 //
-// Data flow per CTA (4 warps):
-//   * R_t (ascending) is staged in shared memory; Q's 12 rows (padded to the
-//     16-row MMA tile with zeros) are loaded once into A fragments.
-//   * K and V rows of R_t are gathered in chunks of 32 keys with 16-byte
-//     cp.async copies into a double-buffered, XOR-swizzled shared tile; rows past
-//     the end of R_t are zero-filled, so unselected K/V values are never read.
-//   * Per chunk: warp w forms S = Q K^T for keys 8w..8w+7 (mma.sync bf16,
-//     fp32 accumulate), the chunk row maximum is combined across warps through
-//     shared memory, P = exp2(S*scale*log2e - m) is written as BF16, and warp w
-//     accumulates O[:, 64w:64w+64] += P V with running-max rescaling.
-#include "qsa_device.cuh"
+// Pipeline (qsa_pipe.cuh): the CTA's items are cut into 64-key chunks that flow
+// through a 3-stage ring of swizzled K / V tiles (plus the item's 12 Q rows on
+// its first chunk), gathered with 16-byte cp.async copies two chunks ahead of
+// the compute.  Rows past the end of R_t are zero-filled, so unselected K/V
+// values never reach an output.  Per chunk, warp w forms S = Q K^T for keys
+// 8w..8w+7 (mma.sync m16n8k16 BF16, FP32 accumulate, Q fragments held in
+// registers for the whole item), the chunk's row maxima are combined across the
+// warps in shared memory, P = exp2(S*scale*log2e - m) is written as BF16, and
+// warp w accumulates O[:, 32w:32w+32] += P V with running-max rescaling.
 #include "qsa_internal.h"
+#include "qsa_pipe.cuh"
 
 namespace qsa {
 namespace {
 
-constexpr int kThreads = 128;
-constexpr int kChunk = 32;       // keys per pipeline stage
-constexpr int kPStride = 40;     // bf16 per row of the P tile (80 B: conflict-free ldmatrix)
-constexpr int kTileBytes = kChunk * 512;
-constexpr int kOffK = 16 * 512;                 // after the Q tile
-constexpr int kOffV = kOffK + 2 * kTileBytes;
-constexpr int kOffP = kOffV + 2 * kTileBytes;
+constexpr int kThreads = kPipeThreads;
+constexpr int kWarps = kThreads / 32;
+constexpr int kStages = 3;
+constexpr int kTile = kPipeKeys * 512;                  // one swizzled [64][256] BF16 tile
+constexpr int kStageBytes = 2 * kTile + kHeadsPerGroup * 512;  // K | V | Q rows
+constexpr int kPStride = 72;                            // bf16 per P row (144 B)
+constexpr int kOffZero = kStages * kStageBytes;         // 512 zero bytes: Q rows 12..15
+constexpr int kOffP = kOffZero + 512;
 constexpr int kOffMax = kOffP + kRowTile * kPStride * 2;
-constexpr int kOffSum = kOffMax + 4 * kRowTile * 4;
-constexpr int kOffCols = kOffSum + 4 * kRowTile * 4;
+constexpr int kOffSum = kOffMax + kWarps * kRowTile * 4;
+constexpr int kOffDesc = kOffSum + kWarps * kRowTile * 4;
+constexpr int kSmemBytes = kOffDesc + kStages * 16;
+static_assert(kSmemBytes <= 232448, "shared memory per block");
+constexpr int kFirst = 1, kLast = 2;
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
 fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
            const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ row_cnt,
-           const int32_t* __restrict__ row_cols, int G, int n_sel, float scale_log2,
+           const int32_t* __restrict__ row_cols, int64_t n_items, int G, int n_sel, float scale_log2,
            __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, cq = lane & 3, mi = lane >> 3;
+  const int H = G * kHeadsPerGroup;
+  int4* desc = reinterpret_cast<int4*>(smem + kOffDesc);
   __nv_bfloat16* sP = reinterpret_cast<__nv_bfloat16*>(smem + kOffP);
   float* sMax = reinterpret_cast<float*>(smem + kOffMax);
   float* sSum = reinterpret_cast<float*>(smem + kOffSum);
-  int32_t* sCols = reinterpret_cast<int32_t*>(smem + kOffCols);
+  if (tid < 32) reinterpret_cast<uint4*>(smem + kOffZero)[tid] = make_uint4(0, 0, 0, 0);
 
-  const int H = G * kHeadsPerGroup;
-  const int64_t t = blockIdx.x / G;
-  const int g = static_cast<int>(blockIdx.x - t * G);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gq = lane >> 2, cq = lane & 3;
-  const int cnt = row_cnt[t];
-  const int64_t qrow0 = t * H + g * kHeadsPerGroup;  // first of the group's 12 query-head rows
-
-  if (cnt == 0) {  // padding query: zero output, -inf LSE
-    uint4* o = reinterpret_cast<uint4*>(out + qrow0 * kHeadDim);
-    for (int i = tid; i < kHeadsPerGroup * 32; i += kThreads) o[i] = make_uint4(0, 0, 0, 0);
-    if (tid < kHeadsPerGroup) lse[qrow0 + tid] = -INFINITY;
-    return;
-  }
-
-  for (int i = tid; i < cnt; i += kThreads) sCols[i] = row_cols[t * n_sel + i];
-  const uint32_t sQa = smem_u32(smem), sKa = smem_u32(smem + kOffK), sVa = smem_u32(smem + kOffV);
-  for (int i = tid; i < kRowTile * 32; i += kThreads) {
-    const int r = i >> 5, c = i & 31;
-    const bool ok = r < kHeadsPerGroup;
-    cp_async16(sQa + swz512(r, c), q + (qrow0 + (ok ? r : 0)) * kHeadDim + c * 8, ok);
-  }
-  cp_async_commit();
-  __syncthreads();  // sCols visible to every issuing thread
-
-  const int n_chunks = (cnt + kChunk - 1) / kChunk;
-  auto issue = [&](int ch) {
-    const int stage = ch & 1, base = ch * kChunk;
-    const int nk = min(kChunk, cnt - base);
-#pragma unroll 4
-    for (int i = tid; i < 2 * kChunk * 32; i += kThreads) {
-      const int tensor = i / (kChunk * 32);
-      const int r = (i >> 5) & (kChunk - 1), c = i & 31;
-      const bool ok = r < nk;
-      const int64_t key = ok ? sCols[base + r] : 0;
-      const __nv_bfloat16* src = (tensor ? v : k) + (key * G + g) * kHeadDim + c * 8;
-      cp_async16((tensor ? sVa : sKa) + stage * kTileBytes + swz512(r, c), src, ok);
+  Cursor cur;
+  cursor_init(cur, row_cnt, n_items, G);
+  int32_t key[8];
+  cursor_keys(key, cur, n_items, G, row_cols, n_sel);
+  // Issues the cursor's chunk into `stage`, records its descriptor, advances.
+  auto issue = [&](int stage) {
+    const uint32_t st = sbase + stage * kStageBytes;
+    if (cur.it < n_items) {
+      const int64_t t = cur.it / G;
+      const int g = static_cast<int>(cur.it - t * G);
+      const int nk = cursor_nk(cur, n_items);
+      if (nk > 0) {
+        gather_rows(st, st + kTile, k, v, key, g, G, nk);
+        if (cur.ch == 0) gather_heads(st + 2 * kTile, q + (t * H + g * kHeadsPerGroup) * kHeadDim);
+      }
+      if (tid == 0)
+        desc[stage] = make_int4(static_cast<int>(t), g, nk,
+                                (cur.ch == 0 ? kFirst : 0) | (cur.ch == cur.nch - 1 ? kLast : 0));
+    } else if (tid == 0) {
+      desc[stage] = make_int4(0, 0, -1, 0);  // end of the CTA's sequence
     }
+    cp_async_commit();
+    cursor_next(cur, row_cnt, n_items, G);
+    cursor_keys(key, cur, n_items, G, row_cols, n_sel);
   };
   issue(0);
-  cp_async_commit();
-  if (n_chunks > 1) issue(1);
-  cp_async_commit();
-  cp_async_wait<2>();  // the Q tile has landed
-  __syncthreads();
+  issue(1);
 
   uint32_t qa[16][4];
-#pragma unroll
-  for (int ks = 0; ks < 16; ++ks) {
-    const int mi = lane >> 3;
-    ldsm_x4(qa[ks], sQa + swz512(((mi & 1) << 3) + (lane & 7), 2 * ks + (mi >> 1)));
-  }
+  float o[4][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  const uint32_t spa = smem_u32(sP);
 
-  float o[8][4];
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY;  // running max, rows gq and gq+8 (log2 domain)
-  float l0 = 0.f, l1 = 0.f;              // running sum of exp2(s - m)
-  const uint32_t sPa = smem_u32(sP);
-
-  for (int ch = 0; ch < n_chunks; ++ch) {
-    const int stage = ch & 1;
-    const int nk = min(kChunk, cnt - ch * kChunk);
+  for (int c = 0;; ++c) {
+    const int stage = c % kStages;
+    const uint32_t st = sbase + stage * kStageBytes;
     cp_async_wait<1>();
-    __syncthreads();
-
-    // S = Q K^T for this warp's 8 keys.
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t kb = sKa + stage * kTileBytes;
+    __syncthreads();  // chunk c has landed; every warp is done with chunk c - 1
+    const int4 d = desc[stage];
+    issue((c + 2) % kStages);
+    const int nk = d.z;
+    if (nk < 0) break;
+    const int64_t qrow0 = static_cast<int64_t>(d.x) * H + d.y * kHeadsPerGroup;
+    if (nk == 0) {  // padding query: zero output, -inf LSE
+      uint4* orow = reinterpret_cast<uint4*>(out + qrow0 * kHeadDim);
+      for (int i = tid; i < kHeadsPerGroup * 32; i += kThreads) orow[i] = make_uint4(0, 0, 0, 0);
+      if (tid < kHeadsPerGroup) lse[qrow0 + tid] = -INFINITY;
+      continue;
+    }
+    if (d.w & kFirst) {
 #pragma unroll
-    for (int ks = 0; ks < 16; ks += 2) {
-      uint32_t b[4];
-      ldsm_x4(b, kb + swz512(warp * 8 + (lane & 7), 2 * ks + (lane >> 3)));
-      mma_16816(s, qa[ks], b[0], b[1]);
-      mma_16816(s, qa[ks + 1], b[2], b[3]);
+      for (int ks = 0; ks < 16; ++ks) {
+        const int r = ((mi & 1) << 3) + (lane & 7);
+        const int cc = 2 * ks + (mi >> 1);
+        ldsm_x4(qa[ks], r < kHeadsPerGroup ? st + 2 * kTile + swz512(r, cc) : sbase + kOffZero + (cc << 4));
+      }
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
+    }
+    // S = Q K^T for this warp's 8 keys, as four independent accumulation chains
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    {
+      float sp[4][4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sp[j][0] = sp[j][1] = sp[j][2] = sp[j][3] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < 16; ks += 2) {
+        uint32_t b[4];
+        ldsm_x4(b, st + swz512(warp * 8 + (lane & 7), 2 * ks + mi));
+        mma_16816(sp[(ks >> 1) & 3], qa[ks], b[0], b[1]);
+        mma_16816(sp[(ks >> 1) & 3], qa[ks + 1], b[2], b[3]);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s[i] = (sp[0][i] + sp[1][i]) + (sp[2][i] + sp[3][i]);
     }
     const int key0 = warp * 8 + 2 * cq;
     const bool v0 = key0 < nk, v1 = key0 + 1 < nk;
@@ -125,19 +135,19 @@ fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict_
     s[1] = v1 ? s[1] * scale_log2 : -INFINITY;
     s[2] = v0 ? s[2] * scale_log2 : -INFINITY;
     s[3] = v1 ? s[3] * scale_log2 : -INFINITY;
-    float mx0 = fmaxf(s[0], s[1]), mx1 = fmaxf(s[2], s[3]);
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    float x0 = fmaxf(s[0], s[1]), x1 = fmaxf(s[2], s[3]);
+    x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 1));
+    x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 2));
+    x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 1));
+    x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 2));
     if (cq == 0) {
-      sMax[warp * kRowTile + gq] = mx0;
-      sMax[warp * kRowTile + gq + 8] = mx1;
+      sMax[warp * kRowTile + gq] = x0;
+      sMax[warp * kRowTile + gq + 8] = x1;
     }
     __syncthreads();
     float n0 = m0, n1 = m1;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < kWarps; ++w) {
       n0 = fmaxf(n0, sMax[w * kRowTile + gq]);
       n1 = fmaxf(n1, sMax[w * kRowTile + gq + 8]);
     }
@@ -158,70 +168,78 @@ fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict_
     m0 = n0;
     m1 = n1;
     __syncthreads();
-    float cs0 = 0.f, cs1 = 0.f;
+    float c0 = 0.f, c1 = 0.f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      cs0 += sSum[w * kRowTile + gq];
-      cs1 += sSum[w * kRowTile + gq + 8];
+    for (int w = 0; w < kWarps; ++w) {
+      c0 += sSum[w * kRowTile + gq];
+      c1 += sSum[w * kRowTile + gq + 8];
     }
-    l0 = l0 * a0 + cs0;
-    l1 = l1 * a1 + cs1;
+    l0 = l0 * a0 + c0;
+    l1 = l1 * a1 + c1;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
+    for (int nt = 0; nt < 4; ++nt) {
       o[nt][0] *= a0;
       o[nt][1] *= a0;
       o[nt][2] *= a1;
       o[nt][3] *= a1;
     }
-
-    // O[:, 64w:64w+64] += P V
-    const uint32_t vb = sVa + stage * kTileBytes;
+    // O[:, 32w:32w+32] += P V over the chunk's 64 keys
 #pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
+    for (int ks = 0; ks < 4; ++ks) {
       uint32_t pa[4];
-      const int mi = lane >> 3;
-      ldsm_x4(pa, sPa + (((((mi & 1) << 3) + (lane & 7)) * kPStride + 16 * ks + ((mi >> 1) << 3)) << 1));
+      ldsm_x4(pa, spa + (((((mi & 1) << 3) + (lane & 7)) * kPStride + 16 * ks + ((mi >> 1) << 3)) << 1));
 #pragma unroll
-      for (int nt = 0; nt < 8; nt += 2) {
+      for (int nt = 0; nt < 4; nt += 2) {
         uint32_t b[4];
-        ldsm_x4_t(b, vb + swz512(16 * ks + ((mi & 1) << 3) + (lane & 7), warp * 8 + nt + (mi >> 1)));
+        ldsm_x4_t(b, st + kTile + swz512(16 * ks + ((mi & 1) << 3) + (lane & 7), warp * 4 + nt + (mi >> 1)));
         mma_16816(o[nt], pa, b[0], b[1]);
         mma_16816(o[nt + 1], pa, b[2], b[3]);
       }
     }
-    __syncthreads();  // every warp is done with this stage
-    if (ch + 2 < n_chunks) issue(ch + 2);
-    cp_async_commit();
+    if (d.w & kLast) {
+      const float i0 = 1.f / l0, i1 = 1.f / l1;
+      __nv_bfloat16* orow = out + qrow0 * kHeadDim;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const int dim = warp * 32 + nt * 8 + 2 * cq;
+        *reinterpret_cast<uint32_t*>(orow + gq * kHeadDim + dim) = pack_bf16(o[nt][0] * i0, o[nt][1] * i0);
+        if (gq + 8 < kHeadsPerGroup)
+          *reinterpret_cast<uint32_t*>(orow + (gq + 8) * kHeadDim + dim) = pack_bf16(o[nt][2] * i1, o[nt][3] * i1);
+      }
+      if (warp == 0 && cq == 0) {
+        lse[qrow0 + gq] = (m0 + log2f(l0)) * kLn2;
+        if (gq + 8 < kHeadsPerGroup) lse[qrow0 + gq + 8] = (m1 + log2f(l1)) * kLn2;
+      }
+    }
   }
   cp_async_wait<0>();
-
-  const float i0 = 1.f / l0, i1 = 1.f / l1;
-  __nv_bfloat16* orow = out + qrow0 * kHeadDim;
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    const int dim = warp * 64 + nt * 8 + 2 * cq;
-    *reinterpret_cast<uint32_t*>(orow + gq * kHeadDim + dim) = pack_bf16(o[nt][0] * i0, o[nt][1] * i0);
-    if (gq + 8 < kHeadsPerGroup)
-      *reinterpret_cast<uint32_t*>(orow + (gq + 8) * kHeadDim + dim) = pack_bf16(o[nt][2] * i1, o[nt][3] * i1);
-  }
-  if (warp == 0 && cq == 0) {
-    lse[qrow0 + gq] = (m0 + log2f(l0)) * kLn2;
-    if (gq + 8 < kHeadsPerGroup) lse[qrow0 + gq + 8] = (m1 + log2f(l1)) * kLn2;
-  }
 }
 
 }  // namespace
 
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
 cudaError_t launch_forward(const void* q, const void* k, const void* v, const int32_t* row_cnt,
                            const int32_t* row_cols, int64_t T, int G, int n_sel, float scale, void* out,
-                           float* lse, cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(kOffCols) + static_cast<size_t>(n_sel) * 4;
-  cudaError_t e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+                           float* lse, int* status, cudaStream_t s) {
+  (void)status;  // the forward has no wait that can expire: nothing to report
+  cudaError_t e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  fwd_kernel<<<static_cast<unsigned>(T * G), kThreads, smem, s>>>(
+  const int64_t n_items = T * G;
+  const int64_t grid = n_items < sm_count() ? n_items : sm_count();
+  fwd_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), row_cnt, row_cols, G, n_sel, scale * kLog2e,
+      static_cast<const __nv_bfloat16*>(v), row_cnt, row_cols, n_items, G, n_sel, scale * kLog2e,
       static_cast<__nv_bfloat16*>(out), lse);
   return cudaGetLastError();
 }

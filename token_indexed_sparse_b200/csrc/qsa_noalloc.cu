@@ -49,7 +49,7 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 // Status for sizes outside the supported envelope, in the order qsa_forward checks them.
 qsa_status_t size_status(int64_t T, int64_t T_kv, int H, int G, int n_sel) {
   if (T < 1 || T_kv < 1 || n_sel < 1 || n_sel > 16384 || G < 1 || H < 1) return QSA_ERR_INVALID_ARGUMENT;
-  if (T_kv > INT32_MAX || T > INT32_MAX / n_sel) return QSA_ERR_INVALID_ARGUMENT;
+  if (T_kv > INT32_MAX || T > INT32_MAX / n_sel || T > (int64_t{1} << 30)) return QSA_ERR_INVALID_ARGUMENT;
   if (H % G != 0 || H / G != qsa::kHeadsPerGroup) return QSA_ERR_UNSUPPORTED;
   return QSA_ERR_INVALID_ARGUMENT;
 }
@@ -70,16 +70,19 @@ extern "C" qsa_status_t qsa_forward_noalloc(const void* q, const void* k, const 
     return QSA_ERR_MISALIGNED;
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return QSA_ERR_CUDA;
-  // Scratch layout: row counts [T] int32, then the sorted route lists [T, n_sel]
-  // int32.  The route kernel overwrites every value the forward kernel reads, so
-  // nothing needs clearing between calls.
-  int32_t* row_cnt = static_cast<int32_t*>(scratch);
-  int32_t* row_cols =
-      reinterpret_cast<int32_t*>(static_cast<unsigned char*>(scratch) + align256(static_cast<size_t>(T) * 4));
+  // Scratch layout (the same as qsa_forward's workspace): a status word, row
+  // counts [T] int32, then the sorted route lists [T, n_sel] int32.  The route
+  // kernel overwrites every value the forward kernel reads (and zeroes the status
+  // word), so nothing needs clearing between calls.
+  unsigned char* base = static_cast<unsigned char*>(scratch);
+  int* status = reinterpret_cast<int*>(base);
+  int32_t* row_cnt = reinterpret_cast<int32_t*>(base + 256);
+  int32_t* row_cols = reinterpret_cast<int32_t*>(base + 256 + align256(static_cast<size_t>(T) * 4));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, s) != cudaSuccess)
+  if (qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, status, nullptr, nullptr, nullptr,
+                             H, s) != cudaSuccess)
     return QSA_ERR_CUDA;
-  if (qsa::launch_forward(q, k, v, row_cnt, row_cols, T, G, n_sel, scale, out, lse, s) != cudaSuccess)
+  if (qsa::launch_forward(q, k, v, row_cnt, row_cols, T, G, n_sel, scale, out, lse, status, s) != cudaSuccess)
     return QSA_ERR_CUDA;
   return QSA_OK;
 }

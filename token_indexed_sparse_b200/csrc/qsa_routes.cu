@@ -27,24 +27,26 @@ constexpr int kSortCap = 4096;  // int64 entries sorted in shared memory (32 KB)
 // bitonic merge), so the virtual padding at the end never has to move.  All
 // threads of the block must call it.  `T` is int32_t or int64_t; `s` may point
 // to shared or global memory (global memory writes are ordered by the
-// __syncthreads between steps).
+// __syncthreads between steps).  Index arithmetic is 32-bit shifts and masks:
+// n2 <= 2^30.
 template <typename T>
-__device__ void block_sort(T* s, int64_t len, int64_t n2) {
-  const int64_t half_n = n2 >> 1;
-  for (int64_t k = 2; k <= n2; k <<= 1) {
-    const int64_t half = k >> 1;
-    for (int64_t p = threadIdx.x; p < half_n; p += blockDim.x) {
-      const int64_t blk = p / half, off = p - blk * half;
-      const int64_t i = blk * k + off, j = blk * k + (k - 1 - off);
+__device__ void block_sort(T* s, int len, int n2) {
+  const int half_n = n2 >> 1;
+  for (int lk = 1; (1 << lk) <= n2; ++lk) {
+    const int k = 1 << lk, lh = lk - 1;
+    for (int p = threadIdx.x; p < half_n; p += blockDim.x) {
+      const int off = p & ((1 << lh) - 1);
+      const int base = (p >> lh) << lk;
+      const int i = base + off, j = base + (k - 1 - off);
       if (j < len) {
         const T a = s[i], b = s[j];
         if (b < a) { s[i] = b; s[j] = a; }
       }
     }
     __syncthreads();
-    for (int64_t h = half >> 1; h >= 1; h >>= 1) {
-      for (int64_t p = threadIdx.x; p < half_n; p += blockDim.x) {
-        const int64_t i = (p / h) * 2 * h + (p % h), j = i + h;
+    for (int lg = lh - 1; lg >= 0; --lg) {
+      for (int p = threadIdx.x; p < half_n; p += blockDim.x) {
+        const int i = ((p >> lg) << (lg + 1)) | (p & ((1 << lg) - 1)), j = i + (1 << lg);
         if (j < len) {
           const T a = s[i], b = s[j];
           if (b < a) { s[i] = b; s[j] = a; }
@@ -83,13 +85,143 @@ __device__ int block_exclusive_scan(int x, int* scratch /* >= 32 ints */, int* t
   return base + incl - x;
 }
 
+// Ascending bitonic sort of the 32*NPL values a warp holds in registers
+// (element e = lane * NPL + r lives in v[r] of lane e / NPL).  Same "flip" network
+// as block_sort: comparators whose partner is in another lane exchange values
+// with shfl.xor, the others compare registers of one lane.  Fully unrolled.
+template <int NPL>
+__device__ __forceinline__ void warp_sort(int32_t (&v)[NPL], int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32 * NPL; k <<= 1) {
+    // flip step: e <-> e ^ (k - 1)
+    if (k <= NPL) {
+#pragma unroll
+      for (int r = 0; r < NPL; ++r) {
+        const int p = r ^ (k - 1);
+        if (p > r) {
+          const int32_t a = v[r], b = v[p];
+          v[r] = min(a, b);
+          v[p] = max(a, b);
+        }
+      }
+    } else {
+      // partner of (lane, r) is (lane ^ m, r ^ (NPL - 1)); the lower half of the
+      // k-block (bit k/2 of the element index clear) keeps the minimum
+      const int m = k / NPL - 1;
+      const bool lower = (lane & (k / (2 * NPL))) == 0;
+#pragma unroll
+      for (int r = 0; r < NPL / 2; ++r) {
+        const int r2 = NPL - 1 - r;
+        const int32_t x = v[r], y = v[r2];
+        const int32_t tx = __shfl_xor_sync(0xffffffffu, y, m);  // partner of register r
+        const int32_t ty = __shfl_xor_sync(0xffffffffu, x, m);  // partner of register r2
+        v[r] = lower ? min(x, tx) : max(x, tx);
+        v[r2] = lower ? min(y, ty) : max(y, ty);
+      }
+    }
+    // half-cleaners: e <-> e ^ h
+#pragma unroll
+    for (int h = k / 4; h >= 1; h >>= 1) {
+      if (h < NPL) {
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) {
+          if ((r & h) == 0) {
+            const int32_t a = v[r], b = v[r | h];
+            v[r] = min(a, b);
+            v[r | h] = max(a, b);
+          }
+        }
+      } else {
+        const int m = h / NPL;
+        const bool lower = (lane & m) == 0;
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) {
+          const int32_t t = __shfl_xor_sync(0xffffffffu, v[r], m);
+          v[r] = lower ? min(v[r], t) : max(v[r], t);
+        }
+      }
+    }
+  }
+}
+
+// One warp per query row (rows of up to 32*NPL route slots): filter, sort in
+// registers, de-duplicate, compact; optional key-quad counts and delta.
+template <int NPL>
+__global__ void __launch_bounds__(256) route_rows_warp_kernel(
+    const int32_t* __restrict__ routes, int64_t T, int32_t T_kv, int n_sel, int32_t* __restrict__ row_cnt,
+    int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt, int* __restrict__ status,
+    const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out, float* __restrict__ delta,
+    int H) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+  if (t >= T) return;
+  const int32_t* row = routes + t * n_sel;
+  int32_t v[NPL];
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) {
+    const int i = lane * NPL + r;
+    int32_t x = INT_MAX;
+    if (i < n_sel) {
+      const int32_t y = __ldg(row + i);
+      if (y >= 0 && y < T_kv) x = y;
+    }
+    v[r] = x;
+  }
+  warp_sort<NPL>(v, lane);
+  // previous element of v[0] lives in the previous lane's v[NPL - 1]
+  int32_t prev = __shfl_up_sync(0xffffffffu, v[NPL - 1], 1);
+  if (lane == 0) prev = INT_MIN;
+  int mine = 0;
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) {
+    const int32_t p = r == 0 ? prev : v[r - 1];
+    const int32_t x = v[r];
+    if (x != INT_MAX && x != p) {
+      ++mine;
+      if (quad_cnt != nullptr && (p == INT_MIN || (p >> 2) != (x >> 2))) atomicAdd(quad_cnt + (x >> 2), 1);
+    }
+  }
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int pos = incl - mine;
+  int32_t* dst = row_cols + t * n_sel;
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) {
+    const int32_t p = r == 0 ? prev : v[r - 1];
+    const int32_t x = v[r];
+    if (x != INT_MAX && x != p) dst[pos++] = x;
+  }
+  if (lane == 31) row_cnt[t] = incl;
+
+  if (delta != nullptr) {  // delta[t, h] = rowsum(dO * out)
+    for (int h = 0; h < H; ++h) {
+      const int64_t off = (t * H + h) * kHeadDim + lane * 8;
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(dout + off));
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(out + off));
+      float x = bf16_lo(a.x) * bf16_lo(b.x) + bf16_hi(a.x) * bf16_hi(b.x) + bf16_lo(a.y) * bf16_lo(b.y) +
+                bf16_hi(a.y) * bf16_hi(b.y) + bf16_lo(a.z) * bf16_lo(b.z) + bf16_hi(a.z) * bf16_hi(b.z) +
+                bf16_lo(a.w) * bf16_lo(b.w) + bf16_hi(a.w) * bf16_hi(b.w);
+      x = warp_sum(x);
+      if (lane == 0) delta[t * H + h] = x;
+    }
+  }
+}
+
 // One block per query row: filter invalid IDs, sort, de-duplicate, compact.
 __global__ void __launch_bounds__(kRowThreads) route_rows_kernel(
     const int32_t* __restrict__ routes, int32_t T_kv, int n_sel, int n2,
-    int32_t* __restrict__ row_cnt, int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt) {
+    int32_t* __restrict__ row_cnt, int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt,
+    int* __restrict__ status, const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out,
+    float* __restrict__ delta, int H) {
   extern __shared__ int32_t sv[];  // n2 values, then 32 ints of scan scratch
   int* scratch = sv + n2;
   const int64_t t = blockIdx.x;
+  if (status != nullptr && t == 0 && threadIdx.x == 0) *status = 0;
   const int32_t* row = routes + t * n_sel;
   for (int i = threadIdx.x; i < n2; i += blockDim.x) {
     int32_t x = INT_MAX;
@@ -115,12 +247,26 @@ __global__ void __launch_bounds__(kRowThreads) route_rows_kernel(
   }
   int total;
   int pos = block_exclusive_scan(mine, scratch, &total);
-  int32_t* out = row_cols + t * n_sel;
+  int32_t* dst = row_cols + t * n_sel;
   for (int i = lo; i < hi; ++i) {
     const int32_t x = sv[i];
-    if (x != INT_MAX && (i == 0 || sv[i - 1] != x)) out[pos++] = x;
+    if (x != INT_MAX && (i == 0 || sv[i - 1] != x)) dst[pos++] = x;
   }
   if (threadIdx.x == 0) row_cnt[t] = total;
+
+  if (delta != nullptr) {  // delta[t, h] = rowsum(dO * out), one warp per head row
+    const int lane = threadIdx.x & 31;
+    for (int h = threadIdx.x >> 5; h < H; h += blockDim.x >> 5) {
+      const int64_t off = (t * H + h) * kHeadDim + lane * 8;
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(dout + off));
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(out + off));
+      float x = bf16_lo(a.x) * bf16_lo(b.x) + bf16_hi(a.x) * bf16_hi(b.x) + bf16_lo(a.y) * bf16_lo(b.y) +
+                bf16_hi(a.y) * bf16_hi(b.y) + bf16_lo(a.z) * bf16_lo(b.z) + bf16_hi(a.z) * bf16_hi(b.z) +
+                bf16_lo(a.w) * bf16_lo(b.w) + bf16_hi(a.w) * bf16_hi(b.w);
+      x = warp_sum(x);
+      if (lane == 0) delta[t * H + h] = x;
+    }
+  }
 }
 
 // Single block: exclusive scan of quad counts (n_quads + 1 offsets).
@@ -169,37 +315,109 @@ __global__ void __launch_bounds__(256) quad_fill_kernel(const int32_t* __restric
   }
 }
 
-// One block per quad: sort its list ascending (by query, the high word).
+// First index in sorted entries s[0, len) whose query (high word) is >= q.
+template <typename P>
+__device__ int lower_bound_query(const P* s, int len, int64_t q) {
+  int lo = 0, hi = len;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if ((s[mid] >> 32) < q) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// One block per quad: sort its list ascending (by query, the high word), then
+// record where each query phase [p*C, (p+1)*C) starts in the sorted list:
+// phase_ptr[b*(P+1) + p], p = 0..P (phase P ends the list).
 __global__ void __launch_bounds__(kSortThreads) quad_sort_kernel(const int32_t* __restrict__ ptr,
-                                                                 int64_t* __restrict__ ent) {
+                                                                 int64_t* __restrict__ ent, int P, int C,
+                                                                 int32_t* __restrict__ phase_ptr) {
   __shared__ int64_t sv[kSortCap];
   const int64_t b = blockIdx.x;
-  const int64_t lo = ptr[b], len = ptr[b + 1] - lo;
-  if (len <= 1) return;
-  int64_t n2 = 1;
-  while (n2 < len) n2 <<= 1;
+  const int lo = ptr[b], len = ptr[b + 1] - lo;
+  int32_t* pp = phase_ptr + b * (P + 1);
   int64_t* seg = ent + lo;
+  if (len <= 1) {
+    for (int p = threadIdx.x; p <= P; p += blockDim.x)
+      pp[p] = lo + ((len == 1 && (seg[0] >> 32) < static_cast<int64_t>(p) * C) ? 1 : 0);
+    return;
+  }
+  int n2 = 1;
+  while (n2 < len) n2 <<= 1;
   if (n2 <= kSortCap) {
-    for (int64_t i = threadIdx.x; i < n2; i += blockDim.x) sv[i] = i < len ? seg[i] : LLONG_MAX;
+    for (int i = threadIdx.x; i < n2; i += blockDim.x) sv[i] = i < len ? seg[i] : LLONG_MAX;
     __syncthreads();
     block_sort<int64_t>(sv, n2, n2);
-    for (int64_t i = threadIdx.x; i < len; i += blockDim.x) seg[i] = sv[i];
+    for (int i = threadIdx.x; i < len; i += blockDim.x) seg[i] = sv[i];
+    for (int p = threadIdx.x; p <= P; p += blockDim.x)
+      pp[p] = lo + lower_bound_query(sv, len, static_cast<int64_t>(p) * C);
   } else {
     block_sort<int64_t>(seg, len, n2);  // in place, in global memory
+    for (int p = threadIdx.x; p <= P; p += blockDim.x)
+      pp[p] = lo + lower_bound_query(seg, len, static_cast<int64_t>(p) * C);
   }
 }
 
-int next_pow2(int x) {
+// Thread per quad: append the quad's non-empty phase ranges to the per-phase
+// work lists, wl[p][*] = (quad, first entry, end entry, flags), flags bit 0:
+// no entries before this range, bit 1: no entries after it.  Quads that no query
+// routes to get their dK/dV rows zeroed here.  The order inside a work list
+// does not matter: each item accumulates its own quad, in list order.
+__global__ void __launch_bounds__(256) quad_worklist_kernel(
+    const int32_t* __restrict__ ptr, const int32_t* __restrict__ phase_ptr, int64_t n_quads, int64_t T_kv, int G,
+    int P, int32_t* __restrict__ wl_cnt, int4* __restrict__ wl, __nv_bfloat16* __restrict__ dk,
+    __nv_bfloat16* __restrict__ dv) {
+  const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (b >= n_quads) return;
+  const int q0 = ptr[b], q1 = ptr[b + 1];
+  if (q0 == q1) {
+    const int64_t k_end = min(T_kv, 4 * b + 4);
+    for (int64_t key = 4 * b; key < k_end; ++key) {
+      uint4* rk = reinterpret_cast<uint4*>(dk + key * G * kHeadDim);
+      uint4* rv = reinterpret_cast<uint4*>(dv + key * G * kHeadDim);
+      for (int i = 0; i < G * kHeadDim / 8; ++i) rk[i] = rv[i] = make_uint4(0, 0, 0, 0);
+    }
+    return;
+  }
+  const int32_t* pp = phase_ptr + b * (P + 1);
+  for (int p = 0; p < P; ++p) {
+    const int lo = pp[p], hi = pp[p + 1];
+    if (hi > lo) {
+      const int slot = atomicAdd(wl_cnt + p, 1);
+      wl[static_cast<int64_t>(p) * n_quads + slot] =
+          make_int4(static_cast<int>(b), lo, hi, (lo == q0 ? 1 : 0) | (hi == q1 ? 2 : 0));
+    }
+  }
+}
+
+}  // namespace
+
+static int next_pow2(int x) {
   int n = 1;
   while (n < x) n <<= 1;
   return n;
 }
 
-}  // namespace
-
 cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel, int32_t* row_cnt,
-                              int32_t* row_cols, int32_t* quad_cnt, cudaStream_t s) {
-  const int n2 = next_pow2(n_sel < 2 ? 2 : n_sel);
+                              int32_t* row_cols, int32_t* quad_cnt, int* status, const void* dout,
+                              const void* out, float* delta, int H, cudaStream_t s) {
+  const auto* dq = static_cast<const __nv_bfloat16*>(dout);
+  const auto* o = static_cast<const __nv_bfloat16*>(out);
+  const unsigned wblocks = static_cast<unsigned>((T + 7) / 8);
+  const int32_t tkv = static_cast<int32_t>(T_kv);
+#define QSA_ROWS_WARP(NPL)                                                                                       \
+  route_rows_warp_kernel<NPL><<<wblocks, 256, 0, s>>>(routes, T, tkv, n_sel, row_cnt, row_cols, quad_cnt, status, \
+                                                      dq, o, delta, H);                                          \
+  return cudaGetLastError()
+  if (n_sel <= 64) { QSA_ROWS_WARP(2); }
+  if (n_sel <= 128) { QSA_ROWS_WARP(4); }
+  if (n_sel <= 256) { QSA_ROWS_WARP(8); }
+  if (n_sel <= 512) { QSA_ROWS_WARP(16); }
+  if (n_sel <= 1024) { QSA_ROWS_WARP(32); }
+  if (n_sel <= 2048) { QSA_ROWS_WARP(64); }
+#undef QSA_ROWS_WARP
+  const int n2 = next_pow2(n_sel);
   const size_t smem = static_cast<size_t>(n2 + 32) * sizeof(int32_t);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(route_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -207,7 +425,7 @@ cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, in
     if (e != cudaSuccess) return e;
   }
   route_rows_kernel<<<static_cast<unsigned>(T), kRowThreads, smem, s>>>(
-      routes, static_cast<int32_t>(T_kv), n_sel, n2, row_cnt, row_cols, quad_cnt);
+      routes, tkv, n_sel, n2, row_cnt, row_cols, quad_cnt, status, dq, o, delta, H);
   return cudaGetLastError();
 }
 
@@ -224,8 +442,17 @@ cudaError_t launch_quad_fill(const int32_t* row_cnt, const int32_t* row_cols, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_quad_sort(const int32_t* quad_ptr, int64_t n_quads, int64_t* quad_ent, cudaStream_t s) {
-  quad_sort_kernel<<<static_cast<unsigned>(n_quads), kSortThreads, 0, s>>>(quad_ptr, quad_ent);
+cudaError_t launch_quad_sort(const int32_t* quad_ptr, int64_t n_quads, int64_t* quad_ent, int P, int C,
+                             int32_t* phase_ptr, cudaStream_t s) {
+  quad_sort_kernel<<<static_cast<unsigned>(n_quads), kSortThreads, 0, s>>>(quad_ptr, quad_ent, P, C, phase_ptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quad_worklist(const int32_t* quad_ptr, const int32_t* phase_ptr, int64_t n_quads, int64_t T_kv,
+                                 int G, int P, int32_t* wl_cnt, int4* wl, void* dk, void* dv, cudaStream_t s) {
+  quad_worklist_kernel<<<static_cast<unsigned>((n_quads + 255) / 256), 256, 0, s>>>(
+      quad_ptr, phase_ptr, n_quads, T_kv, G, P, wl_cnt, wl, static_cast<__nv_bfloat16*>(dk),
+      static_cast<__nv_bfloat16*>(dv));
   return cudaGetLastError();
 }
 
