@@ -253,7 +253,8 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
 // a partial or, on its last range, the BF16 result: the summation order is the
 // fixed list order, so dK/dV are bitwise reproducible.
 constexpr int kKvThreads = 256;
-constexpr int kKvStages = 4;
+constexpr int kKvStages = 2;
+constexpr int kKvCtasPerSm = 2;
 constexpr int kEnt = 4;                                   // entries per chunk
 constexpr int kKvRows = kEnt * 2 * kHeadsPerGroup;        // 96 staged rows per chunk
 constexpr int kKvRecOff = kKvRows * 512;                  // records after the rows
@@ -276,7 +277,7 @@ __device__ __forceinline__ int4 kv_item(const int4* wl, int64_t w, int64_t n_wor
   return w < n_work ? __ldg(wl + w / G) : make_int4(0, 0, 0, 0);
 }
 
-__global__ void __launch_bounds__(kKvThreads, 1)
+__global__ void __launch_bounds__(kKvThreads, kKvCtasPerSm)
 dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ q,
             const uint16_t* __restrict__ pds, const int64_t* __restrict__ quad_ent,
             const int32_t* __restrict__ wl_cnt, const int4* __restrict__ wl, int64_t T_kv, int G, int n_sel,
@@ -353,18 +354,16 @@ dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restr
     }
     load_ents();
   };
-  issue(0);
-  issue(1);
-  issue(2);
+  for (int s0 = 0; s0 < kKvStages - 1; ++s0) issue(s0);
 
   float ak[2][4], av[2][4];
   for (int c = 0;; ++c) {
     const int stage = c % kKvStages;
     const uint32_t st = sbase + stage * kKvStageBytes;
-    cp_async_wait<2>();
+    cp_async_wait<kKvStages - 2>();
     __syncthreads();  // chunk c has landed; every warp is done with chunk c - 1
     const int4 d = desc[stage];
-    issue((c + 3) % kKvStages);
+    issue((c + kKvStages - 1) % kKvStages);
     if (d.z < 0) break;
     const int64_t b = d.x;
     const int g = d.y;
@@ -479,7 +478,7 @@ cudaError_t launch_backward_dkdv(const void* grad_out, const void* q, const uint
                                  cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
   if (e != cudaSuccess) return e;
-  dkdv_kernel<<<static_cast<unsigned>(sm_count()), kKvThreads, kKvSmem, s>>>(
+  dkdv_kernel<<<static_cast<unsigned>(kKvCtasPerSm * sm_count()), kKvThreads, kKvSmem, s>>>(
       static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q), pds, quad_ent, wl_cnt + p,
       wl + static_cast<int64_t>(p) * n_quads, T_kv, G, n_sel, scale, partial, static_cast<__nv_bfloat16*>(dk),
       static_cast<__nv_bfloat16*>(dv));
