@@ -41,6 +41,21 @@ UNIT = "pairs/s"
 FWD_FLOPS_PER_PAIR_HEAD = 4 * 256      # QK^T + PV
 BWD_FLOPS_PER_PAIR_HEAD = 10 * 256     # S recompute, dP, dV, dQ, dK
 DKDV_FLOPS_PER_PAIR_HEAD = 4 * 256     # dK = dS^T Q, dV = P^T dO
+# DRAM bytes (read + write) per step of a stage's kernel, from the ncu capture
+# summarised under profiles/, valid only for the kernel source it was taken on:
+# stage -> (bytes per step, source file, sha256 of that file at capture time).
+TRAFFIC = {}
+
+
+def stage_traffic(stage):
+    import hashlib
+    if stage not in TRAFFIC:
+        return None
+    nbytes, rel, digest = TRAFFIC[stage]
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return nbytes if hashlib.sha256(f.read()).hexdigest() == digest else None
+
+
 FWD_STAGES = ["fwd_route_rows", "fwd_attention"]
 BWD_STAGES = ["bwd_route_rows", "bwd_quad_scan", "bwd_quad_fill", "bwd_quad_sort", "bwd_dq", "bwd_dkdv"]
 
@@ -315,7 +330,7 @@ def run_ours(args):
         achieved = work / (avg[dominant] * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None,
+                    "frac": achieved / peak, "traffic": stage_traffic(dominant),
                     "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)"}
     step_tflops = flops / (ms_per_step * 1e-3) / 1e12
     line = {
@@ -333,7 +348,8 @@ def run_ours(args):
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
-        "gpu_launches": args.steps * (len(FWD_STAGES) + len(BWD_STAGES)),
+        "gpu_launches": args.steps * (qsa.launch_count(wl.T, wl.T_kv, wl.H, wl.G, wl.W, False)
+                                      + qsa.launch_count(wl.T, wl.T_kv, wl.H, wl.G, wl.W, True)),
         "clocks": clk,
     }
     if world > 1:

@@ -143,6 +143,17 @@ qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k,
                              const qsa_event_t* stage_events, int n_stage_events);
 
 /*
+ * Number of kernels one qsa_forward (backward = 0) or qsa_backward (backward = 1)
+ * call enqueues for these sizes, not counting the cudaMemsetAsync nodes of the
+ * backward (two).  The forward launches 2; the backward launches 6 plus one dK/dV
+ * launch per query phase, where a phase spans as many consecutive queries as keep
+ * their Q and dO rows (H KB per query) within 48 MiB of L2 (at most 64 phases).
+ * Returns 0 for sizes the calls reject.  For instrumentation and for sizing CUDA
+ * graphs; the paper has no counterpart.
+ */
+int qsa_launch_count(int64_t T, int64_t T_kv, int H, int G, int n_sel, int backward);
+
+/*
  * Route preprocessing on its own, exposing the index structures the attention
  * kernels consume.  Cites: "fa4_qsa" page, `_preprocess` (duplicates collapse,
  * invalid IDs discarded; forward and reverse lists).

@@ -56,6 +56,16 @@ def test_workspace_sizes(lib):
     assert lib.qsa_backward_workspace_size(2**30, 16, 12, 1, 4) == 0   # T * n_sel > INT32_MAX
 
 
+def test_launch_counts(lib):
+    # forward: route rows + attention; backward: 6 kernels + one dK/dV launch per
+    # query phase of 48 MiB / (H KB) queries (2048 at H = 24, 4096 at H = 12)
+    assert lib.qsa_launch_count(32768, 32768, 24, 2, 564, 0) == 2
+    assert lib.qsa_launch_count(32768, 32768, 24, 2, 564, 1) == 6 + 16
+    assert lib.qsa_launch_count(16384, 16384, 12, 1, 512, 1) == 6 + 4
+    assert lib.qsa_launch_count(256, 256, 12, 1, 64, 1) == 6 + 1
+    assert lib.qsa_launch_count(16, 16, 8, 1, 4, 1) == 0
+
+
 def _fwd(lib, q=256, k=256, v=256, routes=256, T=16, T_kv=16, H=12, G=1, n_sel=4, scale=0.0625,
          out=256, lse=256, ws=256, ws_bytes=1 << 20):
     P = ctypes.c_void_p

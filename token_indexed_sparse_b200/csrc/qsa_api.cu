@@ -221,6 +221,14 @@ qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k,
   return QSA_OK;
 }
 
+int qsa_launch_count(int64_t T, int64_t T_kv, int H, int G, int n_sel, int backward) {
+  if (check_sizes(T, T_kv, H, G, n_sel) != QSA_OK) return 0;
+  if (!backward) return 2;
+  int P = 1, C = 1;
+  dkdv_phases(T, H, &P, &C);
+  return 6 + P;
+}
+
 size_t qsa_route_plan_scratch_size(int64_t T, int64_t T_kv) {
   if (T < 1 || T_kv < 1 || T_kv > INT32_MAX) return 0;
   const size_t nq = static_cast<size_t>((T_kv + 3) / 4);

@@ -11,12 +11,11 @@
 //     from the route kernel, accumulates dQ, and stores the BF16 P / dS of every
 //     routed pair (`pds`, one 48-byte record [P h0..h11 | dS h0..h11] per
 //     (t, g, position in R_t)).
-//   * dkdv_kernel, one CTA per (aligned key quad, group g): walks the quad's
-//     query list in ascending query order and accumulates dK^T = Q^T dS and
-//     dV^T = dO^T P on tensor cores.  Each warp owns 64 of the 256 dims and loads
-//     its Q / dO slices straight from global memory into A fragments, so the
-//     kernel uses no shared memory; the fixed list order makes dK/dV bitwise
-//     reproducible.
+//   * dkdv_kernel, persistent over (aligned key quad, group g, query-phase range)
+//     work items: walks the quad's query list in ascending query order, stages
+//     each entry's Q / dO rows and P / dS records in shared memory and
+//     accumulates dK^T = Q^T dS and dV^T = dO^T P on tensor cores; the fixed list
+//     order makes dK/dV bitwise reproducible.
 #include "qsa_internal.h"
 #include "qsa_pipe.cuh"
 

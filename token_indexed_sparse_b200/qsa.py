@@ -55,6 +55,8 @@ def library() -> ctypes.CDLL:
     lib.qsa_forward_ex.argtypes = lib.qsa_forward.argtypes + [vp, i32]
     lib.qsa_backward_ex.restype = i32
     lib.qsa_backward_ex.argtypes = lib.qsa_backward.argtypes + [vp, i32]
+    lib.qsa_launch_count.restype = i32
+    lib.qsa_launch_count.argtypes = [i64, i64, i32, i32, i32, i32]
     lib.qsa_route_plan_scratch_size.restype = sz
     lib.qsa_route_plan_scratch_size.argtypes = [i64, i64]
     lib.qsa_route_plan.restype = i32
@@ -106,6 +108,11 @@ def forward_workspace_size(T, T_kv, H, G, n_sel) -> int:
 
 def backward_workspace_size(T, T_kv, H, G, n_sel) -> int:
     return int(library().qsa_backward_workspace_size(T, T_kv, H, G, n_sel))
+
+
+def launch_count(T, T_kv, H, G, n_sel, backward: bool) -> int:
+    """Kernels one forward / backward call enqueues (0 for rejected sizes)."""
+    return int(library().qsa_launch_count(T, T_kv, H, G, n_sel, 1 if backward else 0))
 
 
 def _workspace(nbytes: int, device, given: torch.Tensor | None) -> torch.Tensor:
