@@ -78,8 +78,8 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
   auto issue = [&](int stage) {
     const uint32_t st = sbase + stage * kStageBytes;
     if (cur.it < n_items) {
-      const int64_t t = cur.it / G;
-      const int g = static_cast<int>(cur.it - t * G);
+      const int64_t t = cur.t;
+      const int g = cur.g;
       const int nk = cursor_nk(cur, n_items);
       int flags = (cur.ch == 0 ? kFirst : 0) | (cur.ch == cur.nch - 1 ? kLast : 0);
       if (nk > 0) {
@@ -267,13 +267,18 @@ constexpr int kItemFirst = 1, kItemLast = 2, kChFirst = 4, kChLast = 8;
 
 struct KvCursor {
   int64_t w;        // work index (item = w / G, g = w % G); >= n_work when exhausted
+  int64_t wi;       // w / G, kept incrementally (no division in the loop)
+  int wg;           // w % G
+  int dt, dg;       // gridDim.x / G and gridDim.x % G
   int4 item;        // (quad, lo, hi, flags) of the current work index
   int4 item_next;   // of the next one (prefetched)
   int ch, nch;
 };
 
-__device__ __forceinline__ int4 kv_item(const int4* wl, int64_t w, int64_t n_work, int G) {
-  return w < n_work ? __ldg(wl + w / G) : make_int4(0, 0, 0, 0);
+// Work-list item one grid stride after the cursor's, or zeros past the end.
+__device__ __forceinline__ int4 kv_item_next(const KvCursor& c, const int4* wl, int64_t n_work, int G) {
+  const int64_t wi_next = c.wi + c.dt + (c.wg + c.dg >= G ? 1 : 0);
+  return c.w + gridDim.x < n_work ? __ldg(wl + wi_next) : make_int4(0, 0, 0, 0);
 }
 
 __global__ void __launch_bounds__(kKvThreads, kKvCtasPerSm)
@@ -292,8 +297,12 @@ dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restr
 
   KvCursor cur;
   cur.w = blockIdx.x;
-  cur.item = kv_item(wl, cur.w, n_work, G);
-  cur.item_next = kv_item(wl, cur.w + gridDim.x, n_work, G);
+  cur.wi = static_cast<int>(blockIdx.x) / G;
+  cur.wg = static_cast<int>(blockIdx.x) % G;
+  cur.dt = static_cast<int>(gridDim.x) / G;
+  cur.dg = static_cast<int>(gridDim.x) % G;
+  cur.item = cur.w < n_work ? __ldg(wl + cur.wi) : make_int4(0, 0, 0, 0);
+  cur.item_next = kv_item_next(cur, wl, n_work, G);
   cur.ch = 0;
   cur.nch = (cur.item.z - cur.item.y + kEnt - 1) / kEnt;
   int64_t ent[kEnt];
@@ -309,7 +318,7 @@ dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restr
   auto issue = [&](int stage) {
     const uint32_t st = sbase + stage * kKvStageBytes;
     if (cur.w < n_work) {
-      const int g = static_cast<int>(cur.w % G);
+      const int g = cur.wg;
       const int n_ent = min(kEnt, cur.item.z - (cur.item.y + cur.ch * kEnt));
       // rows: index i = u * 24 + tensor * 12 + head; warp w copies the 12 rows
       // (one contiguous 6 KB block) of entry w / 2, tensor w % 2
@@ -346,8 +355,14 @@ dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restr
     // advance
     if (cur.w < n_work && ++cur.ch == cur.nch) {
       cur.w += gridDim.x;
+      cur.wi += cur.dt;
+      cur.wg += cur.dg;
+      if (cur.wg >= G) {
+        cur.wg -= G;
+        ++cur.wi;
+      }
       cur.item = cur.item_next;
-      cur.item_next = kv_item(wl, cur.w + gridDim.x, n_work, G);
+      cur.item_next = kv_item_next(cur, wl, n_work, G);
       cur.ch = 0;
       cur.nch = (cur.item.z - cur.item.y + kEnt - 1) / kEnt;
     }

@@ -21,51 +21,64 @@
 namespace qsa {
 namespace {
 
-constexpr int kThreads = kPipeThreads;
-constexpr int kWarps = kThreads / 32;
-constexpr int kStages = 3;
-constexpr int kTile = kPipeKeys * 512;                  // one swizzled [64][256] BF16 tile
-constexpr int kStageBytes = 2 * kTile + kHeadsPerGroup * 512;  // K | V | Q rows
-constexpr int kPStride = 72;                            // bf16 per P row (144 B)
-constexpr int kOffZero = kStages * kStageBytes;         // 512 zero bytes: Q rows 12..15
-constexpr int kOffP = kOffZero + 512;
-constexpr int kOffMax = kOffP + kRowTile * kPStride * 2;
-constexpr int kOffSum = kOffMax + kWarps * kRowTile * 4;
-constexpr int kOffDesc = kOffSum + kWarps * kRowTile * 4;
-constexpr int kSmemBytes = kOffDesc + kStages * 16;
-static_assert(kSmemBytes <= 232448, "shared memory per block");
+// Kernel shape: NW warps per CTA (chunks of KEYS = 8 * NW keys, warp w owns keys
+// 8w..8w+7 of S and dims [DPW * w, DPW * (w + 1)) of O), STAGES-deep gather ring
+// (gathers run STAGES - 1 chunks ahead), CPS CTAs resident per SM.
+template <int NW, int STAGES, int CPS>
+struct FwdShape {
+  static constexpr int kThreads = NW * 32;
+  static constexpr int kKeys = 8 * NW;
+  static constexpr int kDpw = kHeadDim / NW;                   // output dims per warp
+  static constexpr int kNt = kDpw / 8;                         // n8 tiles of P V per warp
+  static constexpr int kKs = kKeys / 16;                       // k16 steps of P V
+  static constexpr int kTile = kKeys * 512;                    // one swizzled [KEYS][256] BF16 tile
+  static constexpr int kStageBytes = 2 * kTile + kHeadsPerGroup * 512;  // K | V | Q rows
+  static constexpr int kPStride = kKeys + 8;                   // bf16 per P row (conflict-free ldmatrix)
+  static constexpr int kOffZero = STAGES * kStageBytes;        // 512 zero bytes: Q rows 12..15
+  static constexpr int kOffP = kOffZero + 512;
+  static constexpr int kOffMax = kOffP + kRowTile * kPStride * 2;
+  static constexpr int kOffSum = kOffMax + NW * kRowTile * 4;
+  static constexpr int kOffDesc = kOffSum + NW * kRowTile * 4;
+  static constexpr int kSmemBytes = kOffDesc + STAGES * 16;
+  static_assert(kSmemBytes * CPS + 1024 * CPS <= 233472, "shared memory per SM");
+  static_assert(kKs >= 1 && kNt % 2 == 0, "shape");
+};
 constexpr int kFirst = 1, kLast = 2;
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int NW, int STAGES, int CPS>
+__global__ void __launch_bounds__(NW * 32, CPS)
 fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
            const __nv_bfloat16* __restrict__ v, const int32_t* __restrict__ row_cnt,
            const int32_t* __restrict__ row_cols, int64_t n_items, int G, int n_sel, float scale_log2,
            __nv_bfloat16* __restrict__ out, float* __restrict__ lse) {
+  using S_ = FwdShape<NW, STAGES, CPS>;
+  constexpr int KEYS = S_::kKeys, kTile = S_::kTile, kStageBytes = S_::kStageBytes, kPStride = S_::kPStride;
+  constexpr int kNt = S_::kNt, kKs = S_::kKs;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, cq = lane & 3, mi = lane >> 3;
   const int H = G * kHeadsPerGroup;
-  int4* desc = reinterpret_cast<int4*>(smem + kOffDesc);
-  __nv_bfloat16* sP = reinterpret_cast<__nv_bfloat16*>(smem + kOffP);
-  float* sMax = reinterpret_cast<float*>(smem + kOffMax);
-  float* sSum = reinterpret_cast<float*>(smem + kOffSum);
-  if (tid < 32) reinterpret_cast<uint4*>(smem + kOffZero)[tid] = make_uint4(0, 0, 0, 0);
+  int4* desc = reinterpret_cast<int4*>(smem + S_::kOffDesc);
+  __nv_bfloat16* sP = reinterpret_cast<__nv_bfloat16*>(smem + S_::kOffP);
+  float* sMax = reinterpret_cast<float*>(smem + S_::kOffMax);
+  float* sSum = reinterpret_cast<float*>(smem + S_::kOffSum);
+  if (tid < 32) reinterpret_cast<uint4*>(smem + S_::kOffZero)[tid] = make_uint4(0, 0, 0, 0);
 
   Cursor cur;
-  cursor_init(cur, row_cnt, n_items, G);
+  cursor_init<KEYS>(cur, row_cnt, n_items, G);
   int32_t key[8];
-  cursor_keys(key, cur, n_items, G, row_cols, n_sel);
+  cursor_keys<KEYS>(key, cur, n_items, G, row_cols, n_sel);
   // Issues the cursor's chunk into `stage`, records its descriptor, advances.
   auto issue = [&](int stage) {
     const uint32_t st = sbase + stage * kStageBytes;
     if (cur.it < n_items) {
-      const int64_t t = cur.it / G;
-      const int g = static_cast<int>(cur.it - t * G);
-      const int nk = cursor_nk(cur, n_items);
+      const int64_t t = cur.t;
+      const int g = cur.g;
+      const int nk = cursor_nk<KEYS>(cur, n_items);
       if (nk > 0) {
         gather_rows(st, st + kTile, k, v, key, g, G, nk);
-        if (cur.ch == 0) gather_heads(st + 2 * kTile, q + (t * H + g * kHeadsPerGroup) * kHeadDim);
+        if (cur.ch == 0) gather_heads<NW>(st + 2 * kTile, q + (t * H + g * kHeadsPerGroup) * kHeadDim);
       }
       if (tid == 0)
         desc[stage] = make_int4(static_cast<int>(t), g, nk,
@@ -74,30 +87,30 @@ fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict_
       desc[stage] = make_int4(0, 0, -1, 0);  // end of the CTA's sequence
     }
     cp_async_commit();
-    cursor_next(cur, row_cnt, n_items, G);
-    cursor_keys(key, cur, n_items, G, row_cols, n_sel);
+    cursor_next<KEYS>(cur, row_cnt, n_items, G);
+    cursor_keys<KEYS>(key, cur, n_items, G, row_cols, n_sel);
   };
-  issue(0);
-  issue(1);
+#pragma unroll
+  for (int s0 = 0; s0 < STAGES - 1; ++s0) issue(s0);
 
   uint32_t qa[16][4];
-  float o[4][4];
+  float o[kNt][4];
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   const uint32_t spa = smem_u32(sP);
 
   for (int c = 0;; ++c) {
-    const int stage = c % kStages;
+    const int stage = c % STAGES;
     const uint32_t st = sbase + stage * kStageBytes;
-    cp_async_wait<1>();
+    cp_async_wait<STAGES - 2>();
     __syncthreads();  // chunk c has landed; every warp is done with chunk c - 1
     const int4 d = desc[stage];
-    issue((c + 2) % kStages);
+    issue((c + STAGES - 1) % STAGES);
     const int nk = d.z;
     if (nk < 0) break;
     const int64_t qrow0 = static_cast<int64_t>(d.x) * H + d.y * kHeadsPerGroup;
     if (nk == 0) {  // padding query: zero output, -inf LSE
       uint4* orow = reinterpret_cast<uint4*>(out + qrow0 * kHeadDim);
-      for (int i = tid; i < kHeadsPerGroup * 32; i += kThreads) orow[i] = make_uint4(0, 0, 0, 0);
+      for (int i = tid; i < kHeadsPerGroup * 32; i += S_::kThreads) orow[i] = make_uint4(0, 0, 0, 0);
       if (tid < kHeadsPerGroup) lse[qrow0 + tid] = -INFINITY;
       continue;
     }
@@ -106,10 +119,10 @@ fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict_
       for (int ks = 0; ks < 16; ++ks) {
         const int r = ((mi & 1) << 3) + (lane & 7);
         const int cc = 2 * ks + (mi >> 1);
-        ldsm_x4(qa[ks], r < kHeadsPerGroup ? st + 2 * kTile + swz512(r, cc) : sbase + kOffZero + (cc << 4));
+        ldsm_x4(qa[ks], r < kHeadsPerGroup ? st + 2 * kTile + swz512(r, cc) : sbase + S_::kOffZero + (cc << 4));
       }
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+      for (int nt = 0; nt < kNt; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
       m0 = m1 = -INFINITY;
       l0 = l1 = 0.f;
     }
@@ -147,7 +160,7 @@ fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict_
     __syncthreads();
     float n0 = m0, n1 = m1;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
+    for (int w = 0; w < NW; ++w) {
       n0 = fmaxf(n0, sMax[w * kRowTile + gq]);
       n1 = fmaxf(n1, sMax[w * kRowTile + gq + 8]);
     }
@@ -170,28 +183,28 @@ fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict_
     __syncthreads();
     float c0 = 0.f, c1 = 0.f;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
+    for (int w = 0; w < NW; ++w) {
       c0 += sSum[w * kRowTile + gq];
       c1 += sSum[w * kRowTile + gq + 8];
     }
     l0 = l0 * a0 + c0;
     l1 = l1 * a1 + c1;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
+    for (int nt = 0; nt < kNt; ++nt) {
       o[nt][0] *= a0;
       o[nt][1] *= a0;
       o[nt][2] *= a1;
       o[nt][3] *= a1;
     }
-    // O[:, 32w:32w+32] += P V over the chunk's 64 keys
+    // O[:, DPW*w : DPW*(w+1)] += P V over the chunk's keys
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
+    for (int ks = 0; ks < kKs; ++ks) {
       uint32_t pa[4];
       ldsm_x4(pa, spa + (((((mi & 1) << 3) + (lane & 7)) * kPStride + 16 * ks + ((mi >> 1) << 3)) << 1));
 #pragma unroll
-      for (int nt = 0; nt < 4; nt += 2) {
+      for (int nt = 0; nt < kNt; nt += 2) {
         uint32_t b[4];
-        ldsm_x4_t(b, st + kTile + swz512(16 * ks + ((mi & 1) << 3) + (lane & 7), warp * 4 + nt + (mi >> 1)));
+        ldsm_x4_t(b, st + kTile + swz512(16 * ks + ((mi & 1) << 3) + (lane & 7), warp * kNt + nt + (mi >> 1)));
         mma_16816(o[nt], pa, b[0], b[1]);
         mma_16816(o[nt + 1], pa, b[2], b[3]);
       }
@@ -200,8 +213,8 @@ fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict_
       const float i0 = 1.f / l0, i1 = 1.f / l1;
       __nv_bfloat16* orow = out + qrow0 * kHeadDim;
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        const int dim = warp * 32 + nt * 8 + 2 * cq;
+      for (int nt = 0; nt < kNt; ++nt) {
+        const int dim = warp * S_::kDpw + nt * 8 + 2 * cq;
         *reinterpret_cast<uint32_t*>(orow + gq * kHeadDim + dim) = pack_bf16(o[nt][0] * i0, o[nt][1] * i0);
         if (gq + 8 < kHeadsPerGroup)
           *reinterpret_cast<uint32_t*>(orow + (gq + 8) * kHeadDim + dim) = pack_bf16(o[nt][2] * i1, o[nt][3] * i1);
@@ -229,15 +242,23 @@ int sm_count() {
   return cached[dev];
 }
 
+// Forward kernel shape used by launch_forward: 4 CTAs of 2 warps per SM, 16-key
+// chunks, 2-stage ring (more independent items per SM beat wider CTAs: at 8 warps
+// per SM, 4 x 2 ran the seq32k forward in 4.7 ms, 2 x 4 in 4.9 ms, 1 x 8 in 6.5 ms).
+constexpr int kFwdWarps = 2, kFwdStages = 2, kFwdCtasPerSm = 4;
+
 cudaError_t launch_forward(const void* q, const void* k, const void* v, const int32_t* row_cnt,
                            const int32_t* row_cols, int64_t T, int G, int n_sel, float scale, void* out,
                            float* lse, int* status, cudaStream_t s) {
   (void)status;  // the forward has no wait that can expire: nothing to report
-  cudaError_t e = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  using S_ = FwdShape<kFwdWarps, kFwdStages, kFwdCtasPerSm>;
+  auto kern = fwd_kernel<kFwdWarps, kFwdStages, kFwdCtasPerSm>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S_::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int64_t n_items = T * G;
-  const int64_t grid = n_items < sm_count() ? n_items : sm_count();
-  fwd_kernel<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, s>>>(
+  const int64_t slots = static_cast<int64_t>(kFwdCtasPerSm) * sm_count();
+  const int64_t grid = n_items < slots ? n_items : slots;
+  kern<<<static_cast<unsigned>(grid), S_::kThreads, S_::kSmemBytes, s>>>(
       static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
       static_cast<const __nv_bfloat16*>(v), row_cnt, row_cols, n_items, G, n_sel, scale * kLog2e,
       static_cast<__nv_bfloat16*>(out), lse);
