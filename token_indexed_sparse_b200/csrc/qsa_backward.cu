@@ -23,79 +23,96 @@ namespace qsa {
 namespace {
 
 // ---------------------------------------------------------------------------
-// dQ (+ P/dS records): persistent, one CTA (8 warps) per SM
+// dQ (+ P/dS records): persistent, CPS CTAs of NW warps per SM
 // ---------------------------------------------------------------------------
-// Same pipeline as the forward kernel (qsa_pipe.cuh): 64-key chunks of K and V
-// rows gathered two chunks ahead into a 3-stage ring of swizzled tiles (rows
-// past the end of R_t zero-filled: dQ multiplies their zero dS by their K rows).
-// Once per item the 12 Q and dO rows, the 12 LSE values and the 12 delta values
-// (delta = rowsum(dO * out), computed by the route kernel) go to one of two item
-// buffers.  Per chunk, warp w computes S = Q K^T and dP = dO V^T for keys
+// Same pipeline as the forward kernel (qsa_pipe.cuh): chunks of KEYS = 8 NW keys
+// of K and V rows gathered STAGES - 1 chunks ahead into a ring of swizzled tiles
+// (rows past the end of R_t zero-filled: dQ multiplies their zero dS by their K
+// rows).  Once per item the 12 Q and dO rows, the 12 LSE values and the 12 delta
+// values (delta = rowsum(dO * out), computed by the route kernel) go to an item
+// buffer.  Per chunk, warp w computes S = Q K^T and dP = dO V^T for keys
 // 8w..8w+7, P = exp2(S*scale*log2e - lse*log2e), dS = P (dP - delta), stores the
-// BF16 P / dS records and accumulates dQ[:, 32w:32w+32] += dS K.
-constexpr int kDqThreads = kPipeThreads;
-constexpr int kStages = 3;
-constexpr int kTile = kPipeKeys * 512;
-constexpr int kStageBytes = 2 * kTile;
+// BF16 P / dS records and accumulates dQ[:, DPW*w : DPW*(w+1)] += dS K.
 constexpr int kRec = 24;  // bf16 per (t, g, key) record: 12 P + 12 dS
-constexpr int kItemQ = 0, kItemDO = kHeadsPerGroup * 512, kItemLse = 2 * kHeadsPerGroup * 512;
-constexpr int kItemDelta = kItemLse + 64, kItemBytes = kItemDelta + 64;
-constexpr int kOffItem = kStages * kStageBytes;
-constexpr int kOffZero = kOffItem + 2 * kItemBytes;
-constexpr int kDsStride = 72;  // bf16 per dS row (144 B)
-constexpr int kOffDS = kOffZero + 512;
-constexpr int kOffRec = kOffDS + kRowTile * kDsStride * 2;
-constexpr int kOffDesc = kOffRec + kPipeKeys * kRec * 2;
-constexpr int kSmemDq = kOffDesc + kStages * 16;
-static_assert(kSmemDq <= 232448, "shared memory per block");
-static_assert(kOffItem % 16 == 0 && kItemBytes % 16 == 0 && kOffZero % 16 == 0 && kOffDS % 16 == 0 &&
-                  kOffRec % 16 == 0 && kOffDesc % 16 == 0,
-              "alignment");
 constexpr int kFirst = 1, kLast = 2, kSlot = 4;
 
-__global__ void __launch_bounds__(kDqThreads, 1)
+template <int NW, int STAGES, int CPS>
+struct DqShape {
+  static constexpr int kThreads = NW * 32;
+  static constexpr int kKeys = 8 * NW;
+  static constexpr int kDpw = kHeadDim / NW;  // dQ dims per warp
+  static constexpr int kNt = kDpw / 8;
+  static constexpr int kKs = kKeys / 16;
+  static constexpr int kTile = kKeys * 512;
+  static constexpr int kStageBytes = 2 * kTile;
+  // Item buffers: with a 2-stage ring the next item's buffer is issued after
+  // every warp has read the current one, so one buffer suffices; deeper rings
+  // keep an item pending and alternate two.
+  static constexpr int kSlots = STAGES == 2 ? 1 : 2;
+  static constexpr int kItemQ = 0, kItemDO = kHeadsPerGroup * 512, kItemLse = 2 * kHeadsPerGroup * 512;
+  static constexpr int kItemDelta = kItemLse + 64, kItemBytes = kItemDelta + 64;
+  static constexpr int kOffItem = STAGES * kStageBytes;
+  static constexpr int kOffZero = kOffItem + kSlots * kItemBytes;
+  static constexpr int kDsStride = kKeys + 8;  // bf16 per dS row (conflict-free ldmatrix)
+  static constexpr int kOffDS = kOffZero + 512;
+  static constexpr int kOffRec = kOffDS + ((kRowTile * kDsStride * 2 + 15) / 16) * 16;
+  static constexpr int kOffDesc = kOffRec + kKeys * kRec * 2;
+  static constexpr int kSmemBytes = kOffDesc + STAGES * 16;
+  static_assert(kSmemBytes * CPS + 1024 * CPS <= 233472, "shared memory per SM");
+  static_assert(kOffItem % 16 == 0 && kItemBytes % 16 == 0 && kOffZero % 16 == 0 && kOffDS % 16 == 0 &&
+                    kOffRec % 16 == 0 && kOffDesc % 16 == 0,
+                "alignment");
+  static_assert(kKs >= 1 && kNt % 2 == 0 && kThreads >= 24, "shape");
+};
+
+template <int NW, int STAGES, int CPS>
+__global__ void __launch_bounds__(NW * 32, CPS)
 dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ q,
           const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
           const float* __restrict__ lse, const float* __restrict__ delta, const int32_t* __restrict__ row_cnt,
           const int32_t* __restrict__ row_cols, int64_t n_items, int G, int n_sel, float scale, float scale_log2,
           __nv_bfloat16* __restrict__ dq, uint16_t* __restrict__ pds) {
+  using S_ = DqShape<NW, STAGES, CPS>;
+  constexpr int KEYS = S_::kKeys, kTile = S_::kTile, kStageBytes = S_::kStageBytes, kDsStride = S_::kDsStride;
+  constexpr int kNt = S_::kNt, kKs = S_::kKs, kItemBytes = S_::kItemBytes, kThreads = S_::kThreads;
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, cq = lane & 3, mi = lane >> 3;
   const int H = G * kHeadsPerGroup;
-  int4* desc = reinterpret_cast<int4*>(smem + kOffDesc);
-  __nv_bfloat16* sDS = reinterpret_cast<__nv_bfloat16*>(smem + kOffDS);
-  uint16_t* sRec = reinterpret_cast<uint16_t*>(smem + kOffRec);
+  int4* desc = reinterpret_cast<int4*>(smem + S_::kOffDesc);
+  __nv_bfloat16* sDS = reinterpret_cast<__nv_bfloat16*>(smem + S_::kOffDS);
+  uint16_t* sRec = reinterpret_cast<uint16_t*>(smem + S_::kOffRec);
   const uint32_t sDSa = smem_u32(sDS);
-  if (tid < 32) reinterpret_cast<uint4*>(smem + kOffZero)[tid] = make_uint4(0, 0, 0, 0);
+  if (tid < 32) reinterpret_cast<uint4*>(smem + S_::kOffZero)[tid] = make_uint4(0, 0, 0, 0);
 
   Cursor cur;
-  cursor_init(cur, row_cnt, n_items, G);
+  cursor_init<KEYS>(cur, row_cnt, n_items, G);
   int32_t key[8];
-  cursor_keys(key, cur, n_items, G, row_cols, n_sel);
+  cursor_keys<KEYS>(key, cur, n_items, G, row_cols, n_sel);
   int islot = 0;  // item buffer of the next non-empty item
   auto issue = [&](int stage) {
     const uint32_t st = sbase + stage * kStageBytes;
     if (cur.it < n_items) {
       const int64_t t = cur.t;
       const int g = cur.g;
-      const int nk = cursor_nk(cur, n_items);
+      const int nk = cursor_nk<KEYS>(cur, n_items);
       int flags = (cur.ch == 0 ? kFirst : 0) | (cur.ch == cur.nch - 1 ? kLast : 0);
       if (nk > 0) {
         gather_rows(st, st + kTile, k, v, key, g, G, nk);
         if (cur.ch == 0) {
           const int64_t qrow0 = t * H + g * kHeadsPerGroup;
-          const uint32_t ib = sbase + kOffItem + islot * kItemBytes;
-          gather_heads(ib + kItemQ, q + qrow0 * kHeadDim);
-          gather_heads(ib + kItemDO, dout + qrow0 * kHeadDim);
-          const int j = tid - kHeadsPerGroup * 16;  // threads 192..197
-          if (j >= 0 && j < 3) cp_async16(ib + kItemLse + 16 * j, lse + qrow0 + 4 * j, true);
-          if (j >= 3 && j < 6) cp_async16(ib + kItemDelta + 16 * (j - 3), delta + qrow0 + 4 * (j - 3), true);
+          const uint32_t ib = sbase + S_::kOffItem + islot * kItemBytes;
+          gather_heads<NW>(ib + S_::kItemQ, q + qrow0 * kHeadDim);
+          gather_heads<NW>(ib + S_::kItemDO, dout + qrow0 * kHeadDim);
+          const int j = tid - (kThreads - 24);  // the last 24 threads: 12 LSE + 12 delta values
+          if (j >= 0 && j < kHeadsPerGroup) cp_async4(ib + S_::kItemLse + 4 * j, lse + qrow0 + j);
+          if (j >= kHeadsPerGroup) cp_async4(ib + S_::kItemDelta + 4 * (j - 12), delta + qrow0 + (j - 12));
           flags |= islot ? kSlot : 0;
-          islot ^= 1;
+          if (S_::kSlots > 1) islot ^= 1;
         } else {
-          flags |= islot ? 0 : kSlot;  // the item's slot was flipped at its first chunk
+          // the item's slot was flipped at its first chunk
+          flags |= (S_::kSlots > 1 ? (islot ? 0 : kSlot) : 0);
         }
       }
       if (tid == 0) desc[stage] = make_int4(static_cast<int>(t), g, nk, flags | ((cur.ch) << 3));
@@ -103,20 +120,20 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
       desc[stage] = make_int4(0, 0, -1, 0);
     }
     cp_async_commit();
-    cursor_next(cur, row_cnt, n_items, G);
-    cursor_keys(key, cur, n_items, G, row_cols, n_sel);
+    cursor_next<KEYS>(cur, row_cnt, n_items, G);
+    cursor_keys<KEYS>(key, cur, n_items, G, row_cols, n_sel);
   };
-  issue(0);
-  issue(1);
+#pragma unroll
+  for (int s0 = 0; s0 < STAGES - 1; ++s0) issue(s0);
 
   uint32_t qa[16][4], da[16][4];
-  float acc[4][4];
+  float acc[kNt][4];
   float ls0 = INFINITY, ls1 = INFINITY, dl0 = 0.f, dl1 = 0.f;
 
   for (int c = 0;; ++c) {
-    const int stage = c % kStages;
+    const int stage = c % STAGES;
     const uint32_t st = sbase + stage * kStageBytes;
-    cp_async_wait<1>();
+    cp_async_wait<STAGES - 2>();
     __syncthreads();  // chunk c has landed; every warp is done with chunk c - 1
     const int4 d = desc[stage];
     const int nk = d.z;
@@ -125,29 +142,29 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
     const int g = d.y;
     const int64_t qrow0 = t * H + g * kHeadsPerGroup;
     if (nk == 0) {  // padding query: dQ = 0 (no item buffer is used)
-      issue((c + 2) % kStages);
+      issue((c + STAGES - 1) % STAGES);
       uint4* orow = reinterpret_cast<uint4*>(dq + qrow0 * kHeadDim);
-      for (int i = tid; i < kHeadsPerGroup * 32; i += kDqThreads) orow[i] = make_uint4(0, 0, 0, 0);
+      for (int i = tid; i < kHeadsPerGroup * 32; i += kThreads) orow[i] = make_uint4(0, 0, 0, 0);
       continue;
     }
     if (d.w & kFirst) {
-      const uint32_t ib = sbase + kOffItem + ((d.w & kSlot) ? kItemBytes : 0);
+      const uint32_t ib = sbase + S_::kOffItem + ((d.w & kSlot) ? kItemBytes : 0);
 #pragma unroll
       for (int ks = 0; ks < 16; ++ks) {
         const int r = ((mi & 1) << 3) + (lane & 7);
         const int cc = 2 * ks + (mi >> 1);
         const bool real = r < kHeadsPerGroup;
-        ldsm_x4(qa[ks], real ? ib + kItemQ + swz512(r, cc) : sbase + kOffZero + (cc << 4));
-        ldsm_x4(da[ks], real ? ib + kItemDO + swz512(r, cc) : sbase + kOffZero + (cc << 4));
+        ldsm_x4(qa[ks], real ? ib + S_::kItemQ + swz512(r, cc) : sbase + S_::kOffZero + (cc << 4));
+        ldsm_x4(da[ks], real ? ib + S_::kItemDO + swz512(r, cc) : sbase + S_::kOffZero + (cc << 4));
       }
-      const float* il = reinterpret_cast<const float*>(smem + (ib - sbase) + kItemLse);
-      const float* idl = reinterpret_cast<const float*>(smem + (ib - sbase) + kItemDelta);
+      const float* il = reinterpret_cast<const float*>(smem + (ib - sbase) + S_::kItemLse);
+      const float* idl = reinterpret_cast<const float*>(smem + (ib - sbase) + S_::kItemDelta);
       ls0 = il[gq] * kLog2e;
       dl0 = idl[gq];
       ls1 = gq + 8 < kHeadsPerGroup ? il[gq + 8] * kLog2e : INFINITY;
       dl1 = gq + 8 < kHeadsPerGroup ? idl[gq + 8] : 0.f;
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+      for (int nt = 0; nt < kNt; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
     }
     // S = Q K^T and dP = dO V^T for this warp's 8 keys, two chains each
     float s[4], dp[4];
@@ -175,7 +192,7 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
       }
     }
     __syncthreads();  // every warp has read this item's buffer: its slot may be refilled
-    issue((c + 2) % kStages);
+    issue((c + STAGES - 1) % STAGES);
 
     const int key0 = warp * 8 + 2 * cq;
     const bool v0 = key0 < nk, v1 = key0 + 1 < nk;
@@ -201,20 +218,20 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
     }
     __syncthreads();
     {
-      const int base = (d.w >> 3) * kPipeKeys;
+      const int base = (d.w >> 3) * KEYS;
       const uint4* src = reinterpret_cast<const uint4*>(sRec);
       uint4* dst = reinterpret_cast<uint4*>(pds + ((t * G + g) * n_sel + base) * kRec);
-      for (int i = tid; i < nk * 3; i += kDqThreads) dst[i] = src[i];
+      for (int i = tid; i < nk * 3; i += kThreads) dst[i] = src[i];
     }
-    // dQ[:, 32w:32w+32] += dS K over the chunk's 64 keys
+    // dQ[:, DPW*w : DPW*(w+1)] += dS K over the chunk's keys
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
+    for (int ks = 0; ks < kKs; ++ks) {
       uint32_t a[4];
       ldsm_x4(a, sDSa + (((((mi & 1) << 3) + (lane & 7)) * kDsStride + 16 * ks + ((mi >> 1) << 3)) << 1));
 #pragma unroll
-      for (int nt = 0; nt < 4; nt += 2) {
+      for (int nt = 0; nt < kNt; nt += 2) {
         uint32_t b[4];
-        ldsm_x4_t(b, st + swz512(16 * ks + ((mi & 1) << 3) + (lane & 7), warp * 4 + nt + (mi >> 1)));
+        ldsm_x4_t(b, st + swz512(16 * ks + ((mi & 1) << 3) + (lane & 7), warp * kNt + nt + (mi >> 1)));
         mma_16816(acc[nt], a, b[0], b[1]);
         mma_16816(acc[nt + 1], a, b[2], b[3]);
       }
@@ -222,8 +239,8 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
     if (d.w & kLast) {
       __nv_bfloat16* drow = dq + qrow0 * kHeadDim;
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        const int dim = warp * 32 + nt * 8 + 2 * cq;
+      for (int nt = 0; nt < kNt; ++nt) {
+        const int dim = warp * S_::kDpw + nt * 8 + 2 * cq;
         *reinterpret_cast<uint32_t*>(drow + gq * kHeadDim + dim) = pack_bf16(acc[nt][0] * scale, acc[nt][1] * scale);
         if (gq + 8 < kHeadsPerGroup)
           *reinterpret_cast<uint32_t*>(drow + (gq + 8) * kHeadDim + dim) =
@@ -471,15 +488,22 @@ dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restr
 
 }  // namespace
 
+// dQ kernel shape used by launch_backward_dq: 2 CTAs of 4 warps per SM, 32-key
+// chunks, 2-stage ring.
+constexpr int kDqWarps = 4, kDqStages = 2, kDqCtasPerSm = 2;
+
 cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* k, const void* v,
                                const float* lse, const float* delta, const int32_t* row_cnt,
                                const int32_t* row_cols, int64_t T, int G, int n_sel, float scale, void* dq,
                                uint16_t* pds, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemDq);
+  using S_ = DqShape<kDqWarps, kDqStages, kDqCtasPerSm>;
+  auto kern = dq_kernel<kDqWarps, kDqStages, kDqCtasPerSm>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S_::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int64_t n_items = T * G;
-  const int64_t grid = n_items < sm_count() ? n_items : sm_count();
-  dq_kernel<<<static_cast<unsigned>(grid), kDqThreads, kSmemDq, s>>>(
+  const int64_t slots = static_cast<int64_t>(kDqCtasPerSm) * sm_count();
+  const int64_t grid = n_items < slots ? n_items : slots;
+  kern<<<static_cast<unsigned>(grid), S_::kThreads, S_::kSmemBytes, s>>>(
       static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q),
       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), lse, delta, row_cnt, row_cols,
       n_items, G, n_sel, scale, scale * kLog2e, static_cast<__nv_bfloat16*>(dq), pds);
