@@ -322,44 +322,43 @@ dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restr
   cur.item_next = kv_item_next(cur, wl, n_work, G);
   cur.ch = 0;
   cur.nch = (cur.item.z - cur.item.y + kEnt - 1) / kEnt;
-  int64_t ent[kEnt];
-  auto load_ents = [&]() {
-    const int e0 = cur.item.y + cur.ch * kEnt;
-#pragma unroll
-    for (int u = 0; u < kEnt; ++u) ent[u] = (cur.w < n_work && e0 + u < cur.item.z) ? __ldg(quad_ent + e0 + u) : -1;
+  // Warp w copies the 12 rows (one contiguous 6 KB block) of entry w / 2,
+  // tensor w % 2, to rows u * 24 + tn * 12 + h of the stage; warps 0, 2, 4, 6
+  // also copy their entry's P/dS records.  Each warp loads only its own entry.
+  const int u_w = warp >> 1, tn_w = warp & 1;
+  const uint32_t row_off = static_cast<uint32_t>(u_w * 24 + tn_w * kHeadsPerGroup) * 512;
+  // swizzle of row u*24 + tn*12 + h: (u*24 + tn*12 + h) & 7 == (h & 7) ^ (4 tn)
+  const uint32_t xl4 = static_cast<uint32_t>(lane ^ (tn_w << 2)) << 4;
+  int64_t ent = -1;
+  auto load_ent = [&]() {
+    const int e = cur.item.y + cur.ch * kEnt + u_w;
+    ent = (cur.w < n_work && e < cur.item.z) ? __ldg(quad_ent + e) : -1;
   };
-  load_ents();
-  // ent[u] for a runtime u without dynamic register indexing
-  auto ent_at = [&](int u) { return u == 0 ? ent[0] : u == 1 ? ent[1] : u == 2 ? ent[2] : ent[3]; };
+  load_ent();
 
   auto issue = [&](int stage) {
     const uint32_t st = sbase + stage * kKvStageBytes;
     if (cur.w < n_work) {
       const int g = cur.wg;
       const int n_ent = min(kEnt, cur.item.z - (cur.item.y + cur.ch * kEnt));
-      // rows: index i = u * 24 + tensor * 12 + head; warp w copies the 12 rows
-      // (one contiguous 6 KB block) of entry w / 2, tensor w % 2
+      const bool live_u = u_w < n_ent;
+      const int64_t t = live_u ? (ent >> 32) : 0;
       {
-        const int u = warp >> 1, tn = warp & 1;
-        const int64_t eu = ent_at(u);
-        const int64_t t = eu >= 0 ? (eu >> 32) : 0;
-        const __nv_bfloat16* src = (tn ? dout : q) + ((t * H + g * kHeadsPerGroup) * kHeadDim + lane * 8);
-        const int i0 = u * 24 + tn * kHeadsPerGroup;
+        const __nv_bfloat16* src = (tn_w ? dout : q) + ((t * H + g * kHeadsPerGroup) * kHeadDim + lane * 8);
+        const uint32_t dst = st + row_off;
 #pragma unroll
         for (int h = 0; h < kHeadsPerGroup; ++h)
-          cp_async16(st + swz512(i0 + h, lane), src + h * kHeadDim, u < n_ent);
+          cp_async16(dst + h * 512 + (xl4 ^ ((h & 7) << 4)), src + h * kHeadDim, live_u);
       }
-      // records: thread -> (entry u, key slot, 16-byte part)
-      if (tid < kEnt * 4 * 3) {
-        const int u = tid / 12, slot = (tid / 3) & 3, part = tid % 3;
-        const int64_t e = ent_at(u);
-        const int mask = static_cast<int>(e & 15);
-        const bool live = u < n_ent && ((mask >> slot) & 1);
-        const int64_t t = live ? (e >> 32) : 0;
-        const int i0 = static_cast<int>((e >> 4) & 0x0fffffff);
+      // records: lanes 0..11 of the tensor-0 warp of entry u copy (key slot, 16-byte part)
+      if (tn_w == 0 && lane < 12) {
+        const int slot = lane / 3, part = lane - 3 * slot;
+        const int mask = static_cast<int>(ent & 15);
+        const bool live = live_u && ((mask >> slot) & 1);
+        const int i0 = static_cast<int>((ent >> 4) & 0x0fffffff);
         const int idx = live ? i0 + __popc(mask & ((1 << slot) - 1)) : 0;
-        const uint16_t* src = pds + ((t * G + g) * n_sel + idx) * kRec + part * 8;
-        cp_async16(st + kKvRecOff + (u * 4 + slot) * (kRec * 2) + part * 16, src, live);
+        const uint16_t* src = pds + (((live ? t : 0) * G + g) * n_sel + idx) * kRec + part * 8;
+        cp_async16(st + kKvRecOff + (u_w * 4 + slot) * (kRec * 2) + part * 16, src, live);
       }
       if (tid == 0) {
         const int fl = (cur.item.w & 3) | (cur.ch == 0 ? kChFirst : 0) | (cur.ch == cur.nch - 1 ? kChLast : 0);
@@ -383,7 +382,7 @@ dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restr
       cur.ch = 0;
       cur.nch = (cur.item.z - cur.item.y + kEnt - 1) / kEnt;
     }
-    load_ents();
+    load_ent();
   };
   for (int s0 = 0; s0 < kKvStages - 1; ++s0) issue(s0);
 
