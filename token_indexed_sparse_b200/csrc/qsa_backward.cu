@@ -282,6 +282,12 @@ static_assert(kKvSmem <= 232448, "shared memory per block");
 static_assert(kKvStageBytes % 128 == 0, "alignment");
 constexpr int kItemFirst = 1, kItemLast = 2, kChFirst = 4, kChLast = 8;
 
+// Byte offset of 16-byte column c of stage row r, which belongs to entry u: the
+// 512-byte-row XOR swizzle with the phase of odd entries shifted by 4.
+__device__ __forceinline__ uint32_t swz_ent(int u, int r, int c) {
+  return static_cast<uint32_t>(r) * 512u + (static_cast<uint32_t>(c ^ ((r & 7) ^ ((u & 1) << 2))) << 4);
+}
+
 struct KvCursor {
   int64_t w;        // work index (item = w / G, g = w % G); >= n_work when exhausted
   int64_t wi;       // w / G, kept incrementally (no division in the loop)
@@ -327,8 +333,11 @@ dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restr
   // also copy their entry's P/dS records.  Each warp loads only its own entry.
   const int u_w = warp >> 1, tn_w = warp & 1;
   const uint32_t row_off = static_cast<uint32_t>(u_w * 24 + tn_w * kHeadsPerGroup) * 512;
-  // swizzle of row u*24 + tn*12 + h: (u*24 + tn*12 + h) & 7 == (h & 7) ^ (4 tn)
-  const uint32_t xl4 = static_cast<uint32_t>(lane ^ (tn_w << 2)) << 4;
+  // Stage rows use the 512-byte-row swizzle with the phase of odd entries
+  // shifted by 4 (swz_ent): the k-step that packs heads 8..11 of entries 2j and
+  // 2j + 1 then reads eight distinct 16-byte bank groups.  For row
+  // u*24 + tn*12 + h the phase is (h & 7) ^ 4 (tn ^ (u & 1)).
+  const uint32_t xl4 = static_cast<uint32_t>(lane ^ ((tn_w ^ (u_w & 1)) << 2)) << 4;
   int64_t ent = -1;
   auto load_ent = [&]() {
     const int e = cur.item.y + cur.ch * kEnt + u_w;
@@ -449,8 +458,8 @@ dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restr
       for (int mt = 0; mt < 2; ++mt) {
         const int dch = warp * 4 + mt * 2 + (mat & 1);
         uint32_t aq[4], ad[4];
-        ldsm_x4_t(aq, st + swz512(u * 24 + h, dch));
-        ldsm_x4_t(ad, st + swz512(u * 24 + kHeadsPerGroup + h, dch));
+        ldsm_x4_t(aq, st + swz_ent(u, u * 24 + h, dch));
+        ldsm_x4_t(ad, st + swz_ent(u, u * 24 + kHeadsPerGroup + h, dch));
         mma_16816(ak[mt], aq, sb0, sb1);
         mma_16816(av[mt], ad, pb0, pb1);
       }
