@@ -194,6 +194,41 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def bitmap_adapter_aux(qsa, torch, routes, wl, dev, flush, peaks, reps=10):
+    """Times the bitmap -> route IDs adapter on this workload's routes rendered as
+    a single-sequence block bitmap (an auxiliary line: not part of the step)."""
+    T, T_kv = wl.T, wl.T_kv
+    NB = (T_kv + 3) // 4
+    if T * NB > (1 << 32):
+        return None
+    sel = torch.zeros((T, NB), dtype=torch.uint8, device=dev)
+    valid = (routes >= 0) & (routes < T_kv)
+    rows = torch.arange(T, device=dev).unsqueeze(1).expand_as(routes)[valid]
+    sel[rows, (routes[valid] // 4).long()] = 1
+    zero = torch.zeros(T, dtype=torch.int32, device=dev)
+    hi = torch.arange(T, dtype=torch.int32, device=dev) + wl.q_offset
+    for _ in range(2):
+        qsa.bitmap_routes(sel, zero, hi, zero, zero, T_kv, wl.W)
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(reps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        qsa.bitmap_routes(sel, zero, hi, zero, zero, T_kv, wl.W)
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    t = np.arange(T, dtype=np.int64) + wl.q_offset
+    scanned = int(np.minimum(t // 4, NB - 1).sum() + T)      # bitmap bytes in each row's reachable range
+    nbytes = scanned + 16 * T + 4 * T * wl.W + 4 * T
+    avg = float(np.mean(ms))
+    del sel
+    return {"kernel": "bitmap_routes", "workload": f"{wl.name} routes as a [{T}, {NB}] uint8 block bitmap",
+            "ms": avg, "bytes": nbytes, "bound": "hbm", "achieved": nbytes / (avg * 1e-3) / 1e9,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": nbytes / (avg * 1e-3) / 1e9 / peaks["hbm_gbs"]}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -332,6 +367,7 @@ def run_ours(args):
         roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": stage_traffic(dominant),
                     "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)"}
+    aux = {"bitmap_routes": bitmap_adapter_aux(qsa, torch, routes, wl, dev, flush, peaks)}
     step_tflops = flops / (ms_per_step * 1e-3) / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -351,6 +387,7 @@ def run_ours(args):
         "gpu_launches": args.steps * (qsa.launch_count(wl.T, wl.T_kv, wl.H, wl.G, wl.W, False)
                                       + qsa.launch_count(wl.T, wl.T_kv, wl.H, wl.G, wl.W, True)),
         "clocks": clk,
+        "aux": aux,
     }
     if world > 1:
         dist.barrier()

@@ -176,6 +176,38 @@ qsa_status_t qsa_route_plan(const int32_t* routes, int64_t T, int64_t T_kv, int 
                             qsa_stream_t stream);
 
 /*
+ * Block-selection bitmap -> route IDs, so that callers of the bitmap API can use
+ * the route-set calls above.  Cites: "Query Sparse Attention (QSA)" page,
+ * "Tensors" (sel_blocks, lo, hi, blk_base, tok_base) and "Selection and
+ * components" (the block lookup): key token j is allowed for query t iff
+ * lo[t] <= j <= hi[t], 0 <= b < NB and sel_blocks[t, b] != 0, where
+ * b = blk_base[t] + floor((j - tok_base[t]) / block_size).  The allowed set is a
+ * route set: qsa_forward / qsa_backward on the returned routes compute the
+ * bitmap API's attention.
+ *   in : sel_blocks [T, NB] uint8 (row-major; nonzero selects global block b);
+ *        lo, hi, blk_base, tok_base [T] int32; T_kv key tokens (keys outside
+ *        [0, T_kv) are never allowed); block_size >= 1; n_sel route width.
+ *        block_first / block_last are not taken: the lookup does not read them
+ *        (their agreement with the bases is a caller contract the page leaves
+ *        unchecked).
+ *   out: routes [T, n_sel] int32, each row the allowed keys ascending, then -1;
+ *        a row with more than n_sel allowed keys keeps its n_sel smallest.
+ *        row_cnt [T] int32 (may be NULL): the true size of each allowed set.
+ *        max_cnt (may be NULL; one int32): set to the largest row_cnt, so a
+ *        caller can size n_sel (the call zeroes it first, on the stream).
+ *   Errors: NULL sel_blocks / lo / hi / blk_base / tok_base / routes, T, NB,
+ *   T_kv, n_sel or block_size < 1, T_kv > INT32_MAX or T * n_sel > 2^31 - 1:
+ *   QSA_ERR_INVALID_ARGUMENT; int32 pointers not 4-byte aligned:
+ *   QSA_ERR_MISALIGNED; a failed launch: QSA_ERR_CUDA.  Asynchronous on
+ *   `stream`; reads no device value on the host.
+ */
+qsa_status_t qsa_bitmap_routes(const uint8_t* sel_blocks, const int32_t* lo, const int32_t* hi,
+                               const int32_t* blk_base, const int32_t* tok_base,
+                               int64_t T, int64_t NB, int64_t T_kv, int block_size, int n_sel,
+                               int32_t* routes, int32_t* row_cnt, int32_t* max_cnt,
+                               qsa_stream_t stream);
+
+/*
  * Allocation-free forward, for callers that cannot allocate device memory: for
  * example an extension running inside a host application that owns the device
  * allocator and offers it no allocation hook, or a latency-critical path that

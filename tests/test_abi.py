@@ -99,6 +99,22 @@ def test_host_validation_before_any_launch(lib):
     assert st == 3                                   # int64 entries need 8-byte alignment
 
 
+def test_bitmap_routes_host_validation(lib):
+    P = ctypes.c_void_p
+
+    def call(sel=256, lo=256, hi=256, bb=256, tb=256, T=8, NB=4, T_kv=16, bs=4, n_sel=16, routes=256,
+             cnt=0, mx=0):
+        return lib.qsa_bitmap_routes(P(sel), P(lo), P(hi), P(bb), P(tb), T, NB, T_kv, bs, n_sel, P(routes),
+                                     P(cnt), P(mx), None)
+    assert call(sel=0) == 1
+    assert call(routes=0) == 1
+    assert call(T=0) == 1 and call(NB=0) == 1 and call(T_kv=0) == 1 and call(n_sel=0) == 1
+    assert call(bs=0) == 1
+    assert call(T_kv=2**31) == 1
+    assert call(T=2**30, n_sel=4) == 1                 # T * n_sel > INT32_MAX
+    assert call(lo=258) == 3 and call(routes=258) == 3 and call(cnt=258) == 3
+
+
 def test_no_cpu_fallback_without_library(monkeypatch, tmp_path):
     from token_indexed_sparse_b200 import qsa
     monkeypatch.setattr(qsa, "_lib", None)

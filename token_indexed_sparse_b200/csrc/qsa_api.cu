@@ -229,6 +229,21 @@ int qsa_launch_count(int64_t T, int64_t T_kv, int H, int G, int n_sel, int backw
   return 6 + P;
 }
 
+qsa_status_t qsa_bitmap_routes(const uint8_t* sel_blocks, const int32_t* lo, const int32_t* hi,
+                               const int32_t* blk_base, const int32_t* tok_base, int64_t T, int64_t NB,
+                               int64_t T_kv, int block_size, int n_sel, int32_t* routes, int32_t* row_cnt,
+                               int32_t* max_cnt, qsa_stream_t stream) {
+  if (!sel_blocks || !lo || !hi || !blk_base || !tok_base || !routes) return QSA_ERR_INVALID_ARGUMENT;
+  if (T < 1 || NB < 1 || T_kv < 1 || n_sel < 1 || block_size < 1) return QSA_ERR_INVALID_ARGUMENT;
+  if (T_kv > INT32_MAX || T > INT32_MAX / n_sel) return QSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(lo, 4) || !aligned(hi, 4) || !aligned(blk_base, 4) || !aligned(tok_base, 4) ||
+      !aligned(routes, 4) || (row_cnt && !aligned(row_cnt, 4)) || (max_cnt && !aligned(max_cnt, 4)))
+    return QSA_ERR_MISALIGNED;
+  QSA_TRY(qsa::launch_bitmap_routes(sel_blocks, lo, hi, blk_base, tok_base, T, NB, T_kv, block_size, n_sel, routes,
+                                    row_cnt, max_cnt, reinterpret_cast<cudaStream_t>(stream)));
+  return QSA_OK;
+}
+
 size_t qsa_route_plan_scratch_size(int64_t T, int64_t T_kv) {
   if (T < 1 || T_kv < 1 || T_kv > INT32_MAX) return 0;
   const size_t nq = static_cast<size_t>((T_kv + 3) / 4);

@@ -51,4 +51,9 @@ cudaError_t launch_backward_dkdv(const void* grad_out, const void* q, const uint
                                  int G, int n_sel, float scale, float* partial, void* dk, void* dv,
                                  cudaStream_t s);
 
+// Bitmap selection -> route IDs (qsa_bitmap.cu); zeroes *max_cnt first when given.
+cudaError_t launch_bitmap_routes(const uint8_t* sel, const int32_t* lo, const int32_t* hi, const int32_t* blk_base,
+                                 const int32_t* tok_base, int64_t T, int64_t NB, int64_t T_kv, int block_size,
+                                 int n_sel, int32_t* routes, int32_t* row_cnt, int32_t* max_cnt, cudaStream_t s);
+
 }  // namespace qsa

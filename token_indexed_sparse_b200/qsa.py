@@ -57,6 +57,8 @@ def library() -> ctypes.CDLL:
     lib.qsa_backward_ex.argtypes = lib.qsa_backward.argtypes + [vp, i32]
     lib.qsa_launch_count.restype = i32
     lib.qsa_launch_count.argtypes = [i64, i64, i32, i32, i32, i32]
+    lib.qsa_bitmap_routes.restype = i32
+    lib.qsa_bitmap_routes.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp]
     lib.qsa_route_plan_scratch_size.restype = sz
     lib.qsa_route_plan_scratch_size.argtypes = [i64, i64]
     lib.qsa_route_plan.restype = i32
@@ -202,3 +204,25 @@ def route_plan(routes, T_kv: int):
                             _ptr(quad_ent), _ptr(scratch), scratch.numel(), _stream(dev))
     _check(st, "qsa_route_plan")
     return row_cnt, row_cols, quad_ptr, quad_ent
+
+
+def bitmap_routes(sel_blocks, lo, hi, blk_base, tok_base, T_kv: int, n_sel: int, block_size: int = 4):
+    """Bitmap selection -> route IDs on the GPU (``qsa_bitmap_routes``).
+
+    Returns ``(routes [T, n_sel] int32, row_cnt [T] int32, max_cnt [1] int32)``,
+    all on the device and produced asynchronously on the current stream.
+    """
+    lib = library()
+    sel = _prep(sel_blocks, torch.uint8, "sel_blocks")
+    dev = sel.device
+    T, NB = sel.shape
+    lo, hi, blk_base, tok_base = (_prep(x, torch.int32, n) for x, n in
+                                  ((lo, "lo"), (hi, "hi"), (blk_base, "blk_base"), (tok_base, "tok_base")))
+    routes = torch.empty((T, n_sel), dtype=torch.int32, device=dev)
+    row_cnt = torch.empty((T,), dtype=torch.int32, device=dev)
+    max_cnt = torch.empty((1,), dtype=torch.int32, device=dev)
+    st = lib.qsa_bitmap_routes(_ptr(sel), _ptr(lo), _ptr(hi), _ptr(blk_base), _ptr(tok_base), T, NB, T_kv,
+                               block_size, n_sel, _ptr(routes), _ptr(row_cnt), _ptr(max_cnt), _stream(dev))
+    _check(st, "qsa_bitmap_routes")
+    return routes, row_cnt, max_cnt
+

@@ -196,3 +196,52 @@ def pair_count(routes: np.ndarray, T_kv: int) -> int:
     key = np.sort(key, axis=1)
     distinct = (key[:, 1:] != key[:, :-1]) & (key[:, 1:] >= 0)
     return int(distinct.sum() + (key[:, 0] >= 0).sum())
+
+
+def make_bitmap_case(T: int, n_docs: int, blocks_per_row: int, seed: int, block_size: int = 4,
+                     perturb_frac: float = 0.05) -> dict:
+    """A seeded packed-sequence input in the bitmap selection format.
+
+    ``T`` tokens are cut into ``n_docs`` documents at sorted distinct cut points
+    (document origins need not be multiples of ``block_size``).  Each document
+    numbers its own blocks from its origin; the last block of a document may be
+    short.  Query t gets ``lo`` = its document's origin, ``hi`` = t, the
+    document's ``blk_base`` / ``tok_base``, and ``blocks_per_row`` selected
+    blocks drawn uniformly from all NB global blocks (so some fall outside its
+    bounds or document).  A seeded ``perturb_frac`` of rows gets bounds that
+    stray outside the document or are empty (lo > hi).  Returns numpy arrays
+    ``sel_blocks [T, NB] uint8, lo, hi, blk_base, tok_base [T] int32,
+    block_first, block_last [NB] int32`` and ``T_kv = T``.
+    """
+    rng = np.random.default_rng(seed)
+    cuts = np.sort(rng.choice(np.arange(1, T), size=n_docs - 1, replace=False)) if n_docs > 1 else np.array([], int)
+    starts = np.concatenate([[0], cuts]).astype(np.int64)
+    ends = np.concatenate([cuts, [T]]).astype(np.int64)
+    block_first, block_last, doc_blk = [], [], []
+    for s, e in zip(starts, ends):
+        doc_blk.append(len(block_first))
+        for b0 in range(s, e, block_size):
+            block_first.append(b0)
+            block_last.append(min(b0 + block_size, e) - 1)
+    NB = len(block_first)
+    doc_of = np.searchsorted(ends, np.arange(T), side="right")
+    lo = starts[doc_of].astype(np.int32)
+    hi = np.arange(T, dtype=np.int32)
+    blk_base = np.array(doc_blk, dtype=np.int32)[doc_of]
+    tok_base = starts[doc_of].astype(np.int32)
+    sel = np.zeros((T, NB), dtype=np.uint8)
+    k = min(blocks_per_row, NB)
+    for t in range(T):
+        sel[t, rng.choice(NB, size=k, replace=False)] = 1
+    n_pert = int(perturb_frac * T)
+    rows = rng.choice(T, size=n_pert, replace=False)
+    for i, t in enumerate(rows):
+        if i % 3 == 0:
+            lo[t] = max(0, int(lo[t]) - int(rng.integers(1, 9)))   # reaches into the previous document
+        elif i % 3 == 1:
+            lo[t] = hi[t] + 1                                        # empty bounds
+        else:
+            hi[t] = min(T - 1, int(hi[t]) + int(rng.integers(1, 9)))  # beyond the query
+    return {"sel_blocks": sel, "lo": lo, "hi": hi, "blk_base": blk_base, "tok_base": tok_base,
+            "block_first": np.array(block_first, np.int32), "block_last": np.array(block_last, np.int32),
+            "T_kv": T, "NB": NB}
