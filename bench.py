@@ -229,6 +229,41 @@ def bitmap_adapter_aux(qsa, torch, routes, wl, dev, flush, peaks, reps=10):
             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": nbytes / (avg * 1e-3) / 1e9 / peaks["hbm_gbs"]}
 
 
+def selector_aux(qsa, torch, dev, flush, peaks, T=32768, Hi=64, NB=8192, k=127, reps=5):
+    """Times the block selector on the seq32k shape (an auxiliary line: not part of
+    the step): tcgen05 scores of every candidate block, then top-k + expansion."""
+    g = torch.Generator(device=dev).manual_seed(4321)
+    qi = torch.randn(T, Hi, 128, device=dev, generator=g).to(torch.bfloat16)
+    kbar = torch.randn(NB, 128, device=dev, generator=g).to(torch.bfloat16)
+    scores = torch.empty(T, NB, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(2):
+        qsa.selector_scores(qi, kbar, 1 / 64, scores=scores, status=status)
+        qsa.selector_topk(scores, k, NB)
+    torch.cuda.synchronize()
+    ms_s, ms_k = [], []
+    for _ in range(reps):
+        flush.zero_()
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record()
+        qsa.selector_scores(qi, kbar, 1 / 64, scores=scores, status=status)
+        e[1].record()
+        qsa.selector_topk(scores, k, NB)
+        e[2].record()
+        torch.cuda.synchronize()
+        ms_s.append(e[0].elapsed_time(e[1]))
+        ms_k.append(e[1].elapsed_time(e[2]))
+    n = np.minimum(np.arange(T, dtype=np.int64) // 4, NB)
+    flops = 2.0 * Hi * 128 * float(n.sum())
+    avg_s, avg_k = float(np.mean(ms_s)), float(np.mean(ms_k))
+    ok = int(status.item()) == 0
+    del qi, kbar, scores
+    return {"kernel": "selector_scores (tcgen05)", "workload": f"T={T}, {Hi} indexer heads x 128 dims, NB={NB} "
+            f"compressed blocks, top-{k} + tail", "ms": avg_s, "bound": "tensor", "flops": flops,
+            "achieved": flops / (avg_s * 1e-3) / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": flops / (avg_s * 1e-3) / 1e12 / peaks["bf16_tflops"], "topk_ms": avg_k, "status_ok": ok}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -367,7 +402,8 @@ def run_ours(args):
         roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": stage_traffic(dominant),
                     "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)"}
-    aux = {"bitmap_routes": bitmap_adapter_aux(qsa, torch, routes, wl, dev, flush, peaks)}
+    aux = {"bitmap_routes": bitmap_adapter_aux(qsa, torch, routes, wl, dev, flush, peaks),
+           "selector": selector_aux(qsa, torch, dev, flush, peaks)}
     step_tflops = flops / (ms_per_step * 1e-3) / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -208,6 +208,45 @@ qsa_status_t qsa_bitmap_routes(const uint8_t* sel_blocks, const int32_t* lo, con
                                qsa_stream_t stream);
 
 /*
+ * QSA block selector, in two calls.  Cites: "Query Sparse Attention (QSA)" page,
+ * "Finding QSA attention and its indexer" (each complete compressed block is
+ * scored as scale * sum_h relu(qi[t, h] . kbar[block]); ratio-causal top-k;
+ * local block IDs expanded with the incomplete causal tail and the packed
+ * sequence's token origin) and the "cudnn_qsa" page, _pack_indices (four-slot
+ * route groups: one complete block or the tail, -1 padded).
+ *
+ * Query t sits at key position pos[t] of a sequence whose first token is
+ * tok_base[t] and whose first compressed block is blk_base[t] (pos, blk_base,
+ * tok_base [T] int32; NULL means pos[t] = t and zero bases).  Its own block is
+ * o = (pos - tok_base) / 4; its candidates are the local blocks c in
+ * [0, min(o, NB - blk_base)), local block c being global block blk_base + c of
+ * kbar and covering tokens tok_base + 4c .. + 3.
+ *
+ * qsa_selector_scores: qi [T, Hi, Di] BF16, kbar [NB, Di] BF16 (both 16-byte
+ * aligned, contiguous), Di == 128, Hi in {32, 64, 128, 256}, scale > 0 finite.
+ * Writes scores[t * score_stride + c] (FP32) for every candidate c and leaves
+ * the other entries untouched; score_stride >= NB.  Runs on the tensor cores
+ * (tcgen05, operands staged by TMA).  `status` (nullable device int) is set to
+ * 2 if an internal bounded wait gave up (then some scores are missing).
+ * qsa_selector_topk: from those scores, blocks [T, k] int32 = the k best
+ * candidates (larger score first, equal scores by the lower local ID), written
+ * ascending and -1 padded (all candidates when there are fewer than k);
+ * routes [T, 4 (k + 1)] int32 = their tokens as four-slot groups, then the
+ * causal tail (tokens tok_base + 4o .. pos, -1 padded), then -1.
+ * Errors: NULL required pointers, T, NB or k < 1, score_stride < NB, sizes
+ * whose products exceed 2^31 - 1: QSA_ERR_INVALID_ARGUMENT; other Di or Hi:
+ * QSA_ERR_UNSUPPORTED; misaligned pointers: QSA_ERR_MISALIGNED; a failed
+ * launch (or no tensor-map encoder in the driver): QSA_ERR_CUDA.
+ */
+qsa_status_t qsa_selector_scores(const void* qi, const void* kbar, int64_t T, int64_t NB, int Hi, int Di,
+                                 float scale, const int32_t* pos, const int32_t* blk_base,
+                                 const int32_t* tok_base, float* scores, int64_t score_stride,
+                                 int* status, qsa_stream_t stream);
+qsa_status_t qsa_selector_topk(const float* scores, int64_t score_stride, int64_t T, int64_t NB, int k,
+                               const int32_t* pos, const int32_t* blk_base, const int32_t* tok_base,
+                               int32_t* blocks, int32_t* routes, qsa_stream_t stream);
+
+/*
  * Allocation-free forward, for callers that cannot allocate device memory: for
  * example an extension running inside a host application that owns the device
  * allocator and offers it no allocation hook, or a latency-critical path that

@@ -21,6 +21,8 @@ Readings where the pages leave a step open (also listed in the design doc):
   blocks ``c`` in ``[0, o)`` (complete blocks strictly before the own block);
   local block c is global block ``blk_base[t] + c`` and covers key tokens
   ``tok_base[t] + 4c .. + 3``.
+* Candidates must exist: local blocks whose global index ``blk_base + c`` is
+  ``>= NB`` are not candidates (the count is ``min(o, NB - blk_base)``).
 * Top-k: the k largest scores; equal scores are ordered by the lower local
   block ID.  With fewer than k candidates, all are taken.
 * Outputs: the selected local block IDs ascending, -1 padded to k; the routes
@@ -43,9 +45,15 @@ def _meta(T, pos, blk_base, tok_base):
 
 
 def own_blocks(T, pos=None, tok_base=None) -> np.ndarray:
-    """Local index of each query's own (tail) block: the number of candidates."""
+    """Local index of each query's own (tail) block."""
     pos, _, tok_base = _meta(T, pos, None, tok_base)
-    return (pos - tok_base) // 4
+    return np.maximum((pos - tok_base) // 4, 0)
+
+
+def n_candidates(T, NB, pos=None, blk_base=None, tok_base=None) -> np.ndarray:
+    """Candidates per query: local blocks [0, n) with n = min(own block, NB - blk_base)."""
+    pos, blk_base, tok_base = _meta(T, pos, blk_base, tok_base)
+    return np.maximum(np.minimum(own_blocks(T, pos, tok_base), NB - blk_base), 0)
 
 
 def selector_scores(qi, kbar, scale: float, pos=None, blk_base=None, tok_base=None) -> np.ndarray:
@@ -57,7 +65,7 @@ def selector_scores(qi, kbar, scale: float, pos=None, blk_base=None, tok_base=No
     kbar = np.asarray(kbar, dtype=np.float64)
     T = qi.shape[0]
     pos, blk_base, tok_base = _meta(T, pos, blk_base, tok_base)
-    o = (pos - tok_base) // 4
+    o = n_candidates(T, kbar.shape[0], pos, blk_base, tok_base)
     width = int(max(o.max(initial=0), 0))
     S = np.full((T, width), np.nan)
     for t in range(T):
@@ -108,6 +116,6 @@ def select(qi, kbar, scale: float, k: int, pos=None, blk_base=None, tok_base=Non
     """Scores, selected local blocks and expanded routes: the whole selector."""
     T = np.asarray(qi).shape[0]
     S = selector_scores(qi, kbar, scale, pos, blk_base, tok_base)
-    n_cand = own_blocks(T, pos, tok_base)
+    n_cand = n_candidates(T, np.asarray(kbar).shape[0], pos, blk_base, tok_base)
     blocks = topk_blocks(S, n_cand, k)
     return S, blocks, expand_routes(blocks, T, pos, tok_base)

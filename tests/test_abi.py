@@ -115,6 +115,23 @@ def test_bitmap_routes_host_validation(lib):
     assert call(lo=258) == 3 and call(routes=258) == 3 and call(cnt=258) == 3
 
 
+def test_selector_host_validation(lib):
+    P = ctypes.c_void_p
+
+    def scores(qi=256, kb=256, T=8, NB=4, Hi=64, Di=128, scale=0.5, sc=256, stride=4):
+        return lib.qsa_selector_scores(P(qi), P(kb), T, NB, Hi, Di, scale, None, None, None, P(sc), stride, None,
+                                       None)
+    assert scores(qi=0) == 1 and scores(sc=0) == 1
+    assert scores(T=0) == 1 and scores(stride=3) == 1 and scores(scale=0.0) == 1
+    assert scores(Di=64) == 2 and scores(Hi=48) == 2 and scores(Hi=16) == 2
+    assert scores(qi=264) == 3 and scores(sc=258) == 3
+
+    def topk(sc=256, stride=4, T=8, NB=4, k=2, b=256, r=256):
+        return lib.qsa_selector_topk(P(sc), stride, T, NB, k, None, None, None, P(b), P(r), None)
+    assert topk(b=0) == 1 and topk(k=0) == 1 and topk(stride=2) == 1
+    assert topk(r=258) == 3
+
+
 def test_no_cpu_fallback_without_library(monkeypatch, tmp_path):
     from token_indexed_sparse_b200 import qsa
     monkeypatch.setattr(qsa, "_lib", None)

@@ -12,7 +12,7 @@ import os
 
 import numpy as np
 
-from oracle.qsa_selector import expand_routes, own_blocks, select, selector_scores, topk_blocks
+from oracle.qsa_selector import n_candidates, own_blocks, select, selector_scores, topk_blocks
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 
@@ -35,7 +35,7 @@ def test_one_head_identity_keys_reduce_to_a_sort():
     T, NB, k = 64, 16, 5
     qi = rng.integers(-3, 4, size=(T, 1, NB)).astype(float)     # many ties
     S = selector_scores(qi, np.eye(NB), 2.0)
-    n = own_blocks(T)
+    n = n_candidates(T, NB)
     blocks = topk_blocks(S, n, k)
     for t in range(T):
         m = int(n[t])
@@ -111,3 +111,14 @@ def test_packed_sequences_and_route_format():
                 assert start // 4 == own and v[-1] == t       # the causal tail
             seen.extend(v.tolist())
         assert seen == sorted(set(seen))                      # distinct, ascending
+
+
+def test_candidates_stop_at_the_last_compressed_block():
+    # 40 queries but only 6 compressed blocks: later queries see blocks 0..5
+    T, NB = 40, 6
+    assert n_candidates(T, NB).tolist() == [min(t // 4, NB) for t in range(T)]
+    assert own_blocks(T).tolist() == [t // 4 for t in range(T)]
+    rng = np.random.default_rng(2)
+    S, blocks, routes = select(rng.standard_normal((T, 2, 4)), rng.standard_normal((NB, 4)), 1.0, 8)
+    assert (blocks[39][blocks[39] >= 0] < NB).all() and (blocks[39] >= 0).sum() == NB
+    assert routes[39].tolist()[4 * NB:4 * NB + 4] == [36, 37, 38, 39]

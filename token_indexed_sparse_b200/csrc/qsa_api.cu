@@ -244,6 +244,36 @@ qsa_status_t qsa_bitmap_routes(const uint8_t* sel_blocks, const int32_t* lo, con
   return QSA_OK;
 }
 
+qsa_status_t qsa_selector_scores(const void* qi, const void* kbar, int64_t T, int64_t NB, int Hi, int Di,
+                                 float scale, const int32_t* pos, const int32_t* blk_base, const int32_t* tok_base,
+                                 float* scores, int64_t score_stride, int* status, qsa_stream_t stream) {
+  if (!qi || !kbar || !scores) return QSA_ERR_INVALID_ARGUMENT;
+  if (T < 1 || NB < 1 || score_stride < NB || !(scale > 0.f) || !std::isfinite(scale))
+    return QSA_ERR_INVALID_ARGUMENT;
+  if (Di != 128 || (Hi != 32 && Hi != 64 && Hi != 128 && Hi != 256)) return QSA_ERR_UNSUPPORTED;
+  if (T > INT32_MAX / Hi || NB > INT32_MAX || T > INT64_MAX / score_stride) return QSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(qi, 16) || !aligned(kbar, 16) || !aligned(scores, 4) || (pos && !aligned(pos, 4)) ||
+      (blk_base && !aligned(blk_base, 4)) || (tok_base && !aligned(tok_base, 4)) || (status && !aligned(status, 4)))
+    return QSA_ERR_MISALIGNED;
+  QSA_TRY(qsa::launch_selector_scores(qi, kbar, T, NB, Hi, scale, pos, blk_base, tok_base, scores, score_stride,
+                                      status, reinterpret_cast<cudaStream_t>(stream)));
+  return QSA_OK;
+}
+
+qsa_status_t qsa_selector_topk(const float* scores, int64_t score_stride, int64_t T, int64_t NB, int k,
+                               const int32_t* pos, const int32_t* blk_base, const int32_t* tok_base, int32_t* blocks,
+                               int32_t* routes, qsa_stream_t stream) {
+  if (!scores || !blocks || !routes) return QSA_ERR_INVALID_ARGUMENT;
+  if (T < 1 || NB < 1 || k < 1 || score_stride < NB) return QSA_ERR_INVALID_ARGUMENT;
+  if (T > INT32_MAX || k > (INT32_MAX / 4) - 1 || T > INT32_MAX / (4 * (k + 1))) return QSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(scores, 4) || !aligned(blocks, 4) || !aligned(routes, 4) || (pos && !aligned(pos, 4)) ||
+      (blk_base && !aligned(blk_base, 4)) || (tok_base && !aligned(tok_base, 4)))
+    return QSA_ERR_MISALIGNED;
+  QSA_TRY(qsa::launch_selector_topk(scores, score_stride, T, NB, k, pos, blk_base, tok_base, blocks, routes,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+  return QSA_OK;
+}
+
 size_t qsa_route_plan_scratch_size(int64_t T, int64_t T_kv) {
   if (T < 1 || T_kv < 1 || T_kv > INT32_MAX) return 0;
   const size_t nq = static_cast<size_t>((T_kv + 3) / 4);

@@ -56,4 +56,12 @@ cudaError_t launch_bitmap_routes(const uint8_t* sel, const int32_t* lo, const in
                                  const int32_t* tok_base, int64_t T, int64_t NB, int64_t T_kv, int block_size,
                                  int n_sel, int32_t* routes, int32_t* row_cnt, int32_t* max_cnt, cudaStream_t s);
 
+// Selector (qsa_selector.cu): scores of the candidate blocks, then top-k and route expansion.
+cudaError_t launch_selector_scores(const void* qi, const void* kbar, int64_t T, int64_t NB, int Hi, float scale,
+                                   const int32_t* pos, const int32_t* blk_base, const int32_t* tok_base,
+                                   float* scores, int64_t stride, int* status, cudaStream_t s);
+cudaError_t launch_selector_topk(const float* scores, int64_t stride, int64_t T, int64_t NB, int k,
+                                 const int32_t* pos, const int32_t* blk_base, const int32_t* tok_base,
+                                 int32_t* blocks, int32_t* routes, cudaStream_t s);
+
 }  // namespace qsa

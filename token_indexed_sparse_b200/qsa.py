@@ -59,6 +59,10 @@ def library() -> ctypes.CDLL:
     lib.qsa_launch_count.argtypes = [i64, i64, i32, i32, i32, i32]
     lib.qsa_bitmap_routes.restype = i32
     lib.qsa_bitmap_routes.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, vp, vp, vp, vp]
+    lib.qsa_selector_scores.restype = i32
+    lib.qsa_selector_scores.argtypes = [vp, vp, i64, i64, i32, i32, f32, vp, vp, vp, vp, i64, vp, vp]
+    lib.qsa_selector_topk.restype = i32
+    lib.qsa_selector_topk.argtypes = [vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp]
     lib.qsa_route_plan_scratch_size.restype = sz
     lib.qsa_route_plan_scratch_size.argtypes = [i64, i64]
     lib.qsa_route_plan.restype = i32
@@ -225,4 +229,56 @@ def bitmap_routes(sel_blocks, lo, hi, blk_base, tok_base, T_kv: int, n_sel: int,
                                block_size, n_sel, _ptr(routes), _ptr(row_cnt), _ptr(max_cnt), _stream(dev))
     _check(st, "qsa_bitmap_routes")
     return routes, row_cnt, max_cnt
+
+
+def _opt_i32(x, name):
+    return None if x is None else _prep(x, torch.int32, name)
+
+
+def selector_scores(qi, kbar, scale: float, pos=None, blk_base=None, tok_base=None, scores=None, status=None):
+    """Candidate block scores on the tensor cores (``qsa_selector_scores``).
+
+    ``qi`` [T, Hi, 128] and ``kbar`` [NB, 128] BF16 on the GPU.  Returns
+    ``scores`` [T, NB] FP32 (entries that are not candidates are left as they
+    were: NaN in a fresh tensor) and a one-element device status tensor.
+    """
+    lib = library()
+    qi = _prep(qi, torch.bfloat16, "qi")
+    kbar = _prep(kbar, torch.bfloat16, "kbar")
+    T, Hi, Di = qi.shape
+    NB = kbar.shape[0]
+    dev = qi.device
+    pos, blk_base, tok_base = (_opt_i32(x, n) for x, n in ((pos, "pos"), (blk_base, "blk_base"),
+                                                           (tok_base, "tok_base")))
+    if scores is None:
+        scores = torch.full((T, NB), float("nan"), dtype=torch.float32, device=dev)
+    if status is None:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+    st = lib.qsa_selector_scores(_ptr(qi), _ptr(kbar), T, NB, Hi, Di, scale, _ptr(pos), _ptr(blk_base),
+                                 _ptr(tok_base), _ptr(scores), scores.stride(0), _ptr(status), _stream(dev))
+    _check(st, "qsa_selector_scores")
+    return scores, status
+
+
+def selector_topk(scores, k: int, NB: int, pos=None, blk_base=None, tok_base=None):
+    """Top-k local blocks and expanded token routes (``qsa_selector_topk``)."""
+    lib = library()
+    scores = _prep(scores, torch.float32, "scores")
+    T = scores.shape[0]
+    dev = scores.device
+    pos, blk_base, tok_base = (_opt_i32(x, n) for x, n in ((pos, "pos"), (blk_base, "blk_base"),
+                                                           (tok_base, "tok_base")))
+    blocks = torch.empty((T, k), dtype=torch.int32, device=dev)
+    routes = torch.empty((T, 4 * (k + 1)), dtype=torch.int32, device=dev)
+    st = lib.qsa_selector_topk(_ptr(scores), scores.stride(0), T, NB, k, _ptr(pos), _ptr(blk_base), _ptr(tok_base),
+                               _ptr(blocks), _ptr(routes), _stream(dev))
+    _check(st, "qsa_selector_topk")
+    return blocks, routes
+
+
+def select(qi, kbar, scale: float, k: int, pos=None, blk_base=None, tok_base=None):
+    """The whole selector: (scores, blocks, routes, status)."""
+    scores, status = selector_scores(qi, kbar, scale, pos, blk_base, tok_base)
+    blocks, routes = selector_topk(scores, k, kbar.shape[0], pos, blk_base, tok_base)
+    return scores, blocks, routes, status
 
