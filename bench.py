@@ -44,7 +44,12 @@ DKDV_FLOPS_PER_PAIR_HEAD = 4 * 256     # dK = dS^T Q, dV = P^T dO
 # DRAM bytes (read + write) per step of a stage's kernel, from the ncu capture
 # summarised under profiles/, valid only for the kernel source it was taken on:
 # stage -> (bytes per step, source file, sha256 of that file at capture time).
-TRAFFIC = {}
+TRAFFIC = {
+    # one step's 16 dK/dV launches on seq32k: ncu dram__bytes_read.sum + dram__bytes_write.sum
+    # (profiles/dkdv_seq32k.md)
+    "bwd_dkdv": (5471966464, "token_indexed_sparse_b200/csrc/qsa_backward.cu",
+                 "0b663f1ac9daea7b9d38f0222f562e8088daeba11d9a02d65a9a74334b68f9a5"),
+}
 
 
 def stage_traffic(stage):
