@@ -197,8 +197,9 @@ qsa_status_t qsa_route_plan(const int32_t* routes, int64_t T, int64_t T_kv, int 
  *        caller can size n_sel (the call zeroes it first, on the stream).
  *   Errors: NULL sel_blocks / lo / hi / blk_base / tok_base / routes, T, NB,
  *   T_kv, n_sel or block_size < 1, T_kv > INT32_MAX or T * n_sel > 2^31 - 1:
- *   QSA_ERR_INVALID_ARGUMENT; int32 pointers not 4-byte aligned:
- *   QSA_ERR_MISALIGNED; a failed launch: QSA_ERR_CUDA.  Asynchronous on
+ *   QSA_ERR_INVALID_ARGUMENT; sel_blocks not 16-byte aligned (it is read with
+ *   16-byte loads) or int32 pointers not 4-byte aligned: QSA_ERR_MISALIGNED;
+ *   a failed launch: QSA_ERR_CUDA.  Asynchronous on
  *   `stream`; reads no device value on the host.
  */
 qsa_status_t qsa_bitmap_routes(const uint8_t* sel_blocks, const int32_t* lo, const int32_t* hi,

@@ -113,6 +113,7 @@ def test_bitmap_routes_host_validation(lib):
     assert call(T_kv=2**31) == 1
     assert call(T=2**30, n_sel=4) == 1                 # T * n_sel > INT32_MAX
     assert call(lo=258) == 3 and call(routes=258) == 3 and call(cnt=258) == 3
+    assert call(sel=264) == 3                          # the bitmap is read with 16-byte loads
 
 
 def test_selector_host_validation(lib):

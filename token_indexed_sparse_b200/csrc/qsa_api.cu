@@ -236,7 +236,7 @@ qsa_status_t qsa_bitmap_routes(const uint8_t* sel_blocks, const int32_t* lo, con
   if (!sel_blocks || !lo || !hi || !blk_base || !tok_base || !routes) return QSA_ERR_INVALID_ARGUMENT;
   if (T < 1 || NB < 1 || T_kv < 1 || n_sel < 1 || block_size < 1) return QSA_ERR_INVALID_ARGUMENT;
   if (T_kv > INT32_MAX || T > INT32_MAX / n_sel) return QSA_ERR_INVALID_ARGUMENT;
-  if (!aligned(lo, 4) || !aligned(hi, 4) || !aligned(blk_base, 4) || !aligned(tok_base, 4) ||
+  if (!aligned(sel_blocks, 16) || !aligned(lo, 4) || !aligned(hi, 4) || !aligned(blk_base, 4) || !aligned(tok_base, 4) ||
       !aligned(routes, 4) || (row_cnt && !aligned(row_cnt, 4)) || (max_cnt && !aligned(max_cnt, 4)))
     return QSA_ERR_MISALIGNED;
   QSA_TRY(qsa::launch_bitmap_routes(sel_blocks, lo, hi, blk_base, tok_base, T, NB, T_kv, block_size, n_sel, routes,
