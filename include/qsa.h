@@ -115,6 +115,22 @@ qsa_status_t qsa_backward(const void* grad_out, const void* q, const void* k, co
                           void* workspace, size_t workspace_bytes, qsa_stream_t stream);
 
 /*
+ * Backward with FP32 dK / dV, for callers that add dK / dV contributions of
+ * several calls before the one rounding to BF16 (context parallelism: each
+ * rank's queries contribute to the global keys, and the partials are summed by
+ * a reduce-scatter).  Cites: "Query Sparse Attention (QSA)" page, "Selection
+ * and components" (FP32 accumulation; dK/dV summed over query heads).
+ * Same arguments and checks as qsa_backward, except that dk and dv are FP32
+ * [T_kv, G, 256] (16-byte aligned): the FP32 values that qsa_backward rounds to
+ * BF16 (keys no query routes to get exact zeros).
+ */
+qsa_status_t qsa_backward_fp32kv(const void* grad_out, const void* q, const void* k, const void* v,
+                                 const void* out, const float* lse, const int32_t* routes,
+                                 int64_t T, int64_t T_kv, int H, int G, int n_sel, float scale,
+                                 void* dq, float* dk, float* dv,
+                                 void* workspace, size_t workspace_bytes, qsa_stream_t stream);
+
+/*
  * Same as qsa_forward / qsa_backward, and in addition records caller-created
  * CUDA events (cudaEvent_t, passed as qsa_event_t) on `stream` after each stage,
  * for per-kernel timing.  Stage i's event is recorded right after stage i is

@@ -1,0 +1,67 @@
+"""GPU checks of the FP32 dK/dV backward and of the context-parallel path.
+
+With one GPU the process group has one rank: the all-gather and the
+reduce-scatter are identities, so the CP path must reproduce the plain calls
+bit for bit.  The FP32 dK/dV backward ("Query Sparse Attention (QSA)" page,
+"Selection and components": FP32 accumulation) must round to exactly the BF16
+backward's dK/dV and match the oracle.  The collective plumbing over several
+ranks is covered on CPU processes (tests/test_cp.py).
+"""
+
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+
+from oracle import backward_dense
+from token_indexed_sparse_b200 import cp, qsa
+from token_indexed_sparse_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+def _inputs(num, T):
+    wl = W.CONFIGS[num].scaled(T)
+    routes = torch.from_numpy(np.array(W.make_routes(wl))).to(DEV)
+    q, k, v, do = (x.to(DEV) for x in W.make_tensors(wl))
+    return wl, routes, q, k, v, do
+
+
+@pytest.mark.parametrize("num,T", [(3, 1024), (5, 256)])
+def test_fp32_kv_backward(num, T):
+    wl, routes, q, k, v, do = _inputs(num, T)
+    out, lse = qsa.forward(q, k, v, routes, wl.scale)
+    dq, dk, dv = qsa.backward(do, q, k, v, out, lse, routes, wl.scale)
+    dq32, dk32, dv32 = qsa.backward(do, q, k, v, out, lse, routes, wl.scale, kv_fp32=True)
+    torch.cuda.synchronize()
+    assert dk32.dtype == torch.float32 and dv32.dtype == torch.float32
+    assert torch.equal(dq32, dq)
+    assert torch.equal(dk32.to(torch.bfloat16), dk) and torch.equal(dv32.to(torch.bfloat16), dv)
+    r = routes.cpu().numpy()
+    _, o_dk, o_dv = backward_dense(do.double().cpu().numpy(), q.double().cpu().numpy(), k.double().cpu().numpy(),
+                                   v.double().cpu().numpy(), r, wl.scale)
+    for a, b in ((dk32, o_dk), (dv32, o_dv)):
+        a = a.double().cpu().numpy()
+        assert np.abs(a - b).max() / max(np.abs(b).max(), 1e-3) <= 1e-2
+
+
+def test_cp_single_rank_reproduces_plain_calls():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            device_id=torch.device(DEV))
+    try:
+        wl, routes, q, k, v, do = _inputs(5, 512)
+        out, lse = qsa.forward(q, k, v, routes, wl.scale)
+        dq, dk, dv = qsa.backward(do, q, k, v, out, lse, routes, wl.scale)
+        c_out, c_lse = cp.cp_forward(q, k, v, routes, wl.scale)
+        c_dq, c_dk, c_dv = cp.cp_backward(do, q, k, v, c_out, c_lse, routes, wl.scale)
+        torch.cuda.synchronize()
+        assert torch.equal(c_out, out) and torch.equal(c_lse, lse)
+        assert torch.equal(c_dq, dq) and torch.equal(c_dk, dk) and torch.equal(c_dv, dv)
+    finally:
+        dist.destroy_process_group()

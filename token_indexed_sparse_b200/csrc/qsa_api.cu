@@ -100,6 +100,61 @@ struct StageEvents {
 
 }  // namespace
 
+// The backward sequence; dk / dv are BF16, or FP32 when kv_f32.
+static qsa_status_t backward_impl(const void* grad_out, const void* q, const void* k, const void* v, const void* out,
+                           const float* lse, const int32_t* routes, int64_t T, int64_t T_kv, int H, int G, int n_sel,
+                           float scale, void* dq, void* dk, void* dv, bool kv_f32, void* workspace,
+                           size_t workspace_bytes, qsa_stream_t stream, const qsa_event_t* stage_events,
+                           int n_stage_events) {
+  if (!grad_out || !q || !k || !v || !out || !lse || !routes || !dq || !dk || !dv || !workspace)
+    return QSA_ERR_INVALID_ARGUMENT;
+  const qsa_status_t st = check_sizes(T, T_kv, H, G, n_sel);
+  if (st != QSA_OK) return st;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return QSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(grad_out, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(routes, 4) ||
+      !aligned(workspace, 256))
+    return QSA_ERR_MISALIGNED;
+  const Layout L = make_layout(T, T_kv, H, G, n_sel, true);
+  if (workspace_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t nq = (T_kv + 3) / 4;
+  int* status = at<int>(workspace, L.status);
+  int32_t* row_cnt = at<int32_t>(workspace, L.row_cnt);
+  int32_t* row_cols = at<int32_t>(workspace, L.row_cols);
+  int32_t* quad_cnt = at<int32_t>(workspace, L.quad_cnt);
+  int32_t* quad_ptr = at<int32_t>(workspace, L.quad_ptr);
+  int32_t* quad_fill = at<int32_t>(workspace, L.quad_fill);
+  int64_t* quad_ent = at<int64_t>(workspace, L.quad_ent);
+  float* delta = at<float>(workspace, L.delta);
+  uint16_t* pds = at<uint16_t>(workspace, L.pds);
+  int32_t* phase_ptr = at<int32_t>(workspace, L.phase_ptr);
+  int32_t* wl_cnt = at<int32_t>(workspace, L.wl_cnt);
+  int4* wl = at<int4>(workspace, L.wl);
+  float* partial = at<float>(workspace, L.partial);
+  const StageEvents ev{stage_events, n_stage_events, s};
+  QSA_TRY(cudaMemsetAsync(quad_cnt, 0, static_cast<size_t>(nq) * 4, s));
+  QSA_TRY(cudaMemsetAsync(wl_cnt, 0, static_cast<size_t>(L.P) * 4, s));
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, quad_cnt, status, grad_out, out, delta,
+                                 H, s));
+  QSA_TRY(ev.mark(0));
+  QSA_TRY(qsa::launch_quad_scan(quad_cnt, nq, quad_ptr, quad_fill, s));
+  QSA_TRY(ev.mark(1));
+  QSA_TRY(qsa::launch_quad_fill(row_cnt, row_cols, T, n_sel, quad_fill, quad_ent, s));
+  QSA_TRY(ev.mark(2));
+  QSA_TRY(qsa::launch_quad_sort(quad_ptr, nq, quad_ent, L.P, L.C, phase_ptr, s));
+  QSA_TRY(qsa::launch_quad_worklist(quad_ptr, phase_ptr, nq, T_kv, G, L.P, wl_cnt, wl, dk, dv, kv_f32, s));
+  QSA_TRY(ev.mark(3));
+  QSA_TRY(qsa::launch_backward_dq(grad_out, q, k, v, lse, delta, row_cnt, row_cols, T, G, n_sel, scale, dq, pds,
+                                  s));
+  QSA_TRY(ev.mark(4));
+  for (int p = 0; p < L.P; ++p)
+    QSA_TRY(qsa::launch_backward_dkdv(grad_out, q, pds, quad_ent, wl_cnt, wl, p, nq, T_kv, G, n_sel, scale, partial,
+                                      dk, dv, kv_f32, s));
+  QSA_TRY(ev.mark(5));
+  return QSA_OK;
+}
+
 extern "C" {
 
 const char* qsa_status_string(qsa_status_t status) {
@@ -172,53 +227,16 @@ qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k,
                              int n_sel, float scale, void* dq, void* dk, void* dv, void* workspace,
                              size_t workspace_bytes, qsa_stream_t stream, const qsa_event_t* stage_events,
                              int n_stage_events) {
-  if (!grad_out || !q || !k || !v || !out || !lse || !routes || !dq || !dk || !dv || !workspace)
-    return QSA_ERR_INVALID_ARGUMENT;
-  const qsa_status_t st = check_sizes(T, T_kv, H, G, n_sel);
-  if (st != QSA_OK) return st;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return QSA_ERR_INVALID_ARGUMENT;
-  if (!aligned(grad_out, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
-      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(routes, 4) ||
-      !aligned(workspace, 256))
-    return QSA_ERR_MISALIGNED;
-  const Layout L = make_layout(T, T_kv, H, G, n_sel, true);
-  if (workspace_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t nq = (T_kv + 3) / 4;
-  int* status = at<int>(workspace, L.status);
-  int32_t* row_cnt = at<int32_t>(workspace, L.row_cnt);
-  int32_t* row_cols = at<int32_t>(workspace, L.row_cols);
-  int32_t* quad_cnt = at<int32_t>(workspace, L.quad_cnt);
-  int32_t* quad_ptr = at<int32_t>(workspace, L.quad_ptr);
-  int32_t* quad_fill = at<int32_t>(workspace, L.quad_fill);
-  int64_t* quad_ent = at<int64_t>(workspace, L.quad_ent);
-  float* delta = at<float>(workspace, L.delta);
-  uint16_t* pds = at<uint16_t>(workspace, L.pds);
-  int32_t* phase_ptr = at<int32_t>(workspace, L.phase_ptr);
-  int32_t* wl_cnt = at<int32_t>(workspace, L.wl_cnt);
-  int4* wl = at<int4>(workspace, L.wl);
-  float* partial = at<float>(workspace, L.partial);
-  const StageEvents ev{stage_events, n_stage_events, s};
-  QSA_TRY(cudaMemsetAsync(quad_cnt, 0, static_cast<size_t>(nq) * 4, s));
-  QSA_TRY(cudaMemsetAsync(wl_cnt, 0, static_cast<size_t>(L.P) * 4, s));
-  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, quad_cnt, status, grad_out, out, delta,
-                                 H, s));
-  QSA_TRY(ev.mark(0));
-  QSA_TRY(qsa::launch_quad_scan(quad_cnt, nq, quad_ptr, quad_fill, s));
-  QSA_TRY(ev.mark(1));
-  QSA_TRY(qsa::launch_quad_fill(row_cnt, row_cols, T, n_sel, quad_fill, quad_ent, s));
-  QSA_TRY(ev.mark(2));
-  QSA_TRY(qsa::launch_quad_sort(quad_ptr, nq, quad_ent, L.P, L.C, phase_ptr, s));
-  QSA_TRY(qsa::launch_quad_worklist(quad_ptr, phase_ptr, nq, T_kv, G, L.P, wl_cnt, wl, dk, dv, s));
-  QSA_TRY(ev.mark(3));
-  QSA_TRY(qsa::launch_backward_dq(grad_out, q, k, v, lse, delta, row_cnt, row_cols, T, G, n_sel, scale, dq, pds,
-                                  s));
-  QSA_TRY(ev.mark(4));
-  for (int p = 0; p < L.P; ++p)
-    QSA_TRY(qsa::launch_backward_dkdv(grad_out, q, pds, quad_ent, wl_cnt, wl, p, nq, T_kv, G, n_sel, scale, partial,
-                                      dk, dv, s));
-  QSA_TRY(ev.mark(5));
-  return QSA_OK;
+  return backward_impl(grad_out, q, k, v, out, lse, routes, T, T_kv, H, G, n_sel, scale, dq, dk, dv, false, workspace,
+                       workspace_bytes, stream, stage_events, n_stage_events);
+}
+
+qsa_status_t qsa_backward_fp32kv(const void* grad_out, const void* q, const void* k, const void* v, const void* out,
+                                 const float* lse, const int32_t* routes, int64_t T, int64_t T_kv, int H, int G,
+                                 int n_sel, float scale, void* dq, float* dk, float* dv, void* workspace,
+                                 size_t workspace_bytes, qsa_stream_t stream) {
+  return backward_impl(grad_out, q, k, v, out, lse, routes, T, T_kv, H, G, n_sel, scale, dq, dk, dv, true, workspace,
+                       workspace_bytes, stream, nullptr, 0);
 }
 
 int qsa_launch_count(int64_t T, int64_t T_kv, int H, int G, int n_sel, int backward) {

@@ -308,8 +308,8 @@ __global__ void __launch_bounds__(kKvThreads, kKvCtasPerSm)
 dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ q,
             const uint16_t* __restrict__ pds, const int64_t* __restrict__ quad_ent,
             const int32_t* __restrict__ wl_cnt, const int4* __restrict__ wl, int64_t T_kv, int G, int n_sel,
-            float scale, float* __restrict__ partial, __nv_bfloat16* __restrict__ dk,
-            __nv_bfloat16* __restrict__ dv) {
+            float scale, float* __restrict__ partial, void* __restrict__ dk_out, void* __restrict__ dv_out,
+            bool f32_out) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -471,14 +471,27 @@ dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restr
         for (int j = 0; j < 2; ++j) {
           const int64_t key = 4 * b + 2 * cq + j;
           if (key < T_kv) {
-            __nv_bfloat16* rk = dk + (key * G + g) * kHeadDim + warp * 32 + gq;
-            __nv_bfloat16* rv = dv + (key * G + g) * kHeadDim + warp * 32 + gq;
+            const int64_t o = (key * G + g) * kHeadDim + warp * 32 + gq;
+            if (f32_out) {  // FP32 sums for callers that add partials before rounding
+              float* rk = static_cast<float*>(dk_out) + o;
+              float* rv = static_cast<float*>(dv_out) + o;
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-              rk[16 * mt] = __float2bfloat16_rn(ak[mt][j] * scale);
-              rk[16 * mt + 8] = __float2bfloat16_rn(ak[mt][2 + j] * scale);
-              rv[16 * mt] = __float2bfloat16_rn(av[mt][j]);
-              rv[16 * mt + 8] = __float2bfloat16_rn(av[mt][2 + j]);
+              for (int mt = 0; mt < 2; ++mt) {
+                rk[16 * mt] = ak[mt][j] * scale;
+                rk[16 * mt + 8] = ak[mt][2 + j] * scale;
+                rv[16 * mt] = av[mt][j];
+                rv[16 * mt + 8] = av[mt][2 + j];
+              }
+            } else {
+              __nv_bfloat16* rk = static_cast<__nv_bfloat16*>(dk_out) + o;
+              __nv_bfloat16* rv = static_cast<__nv_bfloat16*>(dv_out) + o;
+#pragma unroll
+              for (int mt = 0; mt < 2; ++mt) {
+                rk[16 * mt] = __float2bfloat16_rn(ak[mt][j] * scale);
+                rk[16 * mt + 8] = __float2bfloat16_rn(ak[mt][2 + j] * scale);
+                rv[16 * mt] = __float2bfloat16_rn(av[mt][j]);
+                rv[16 * mt + 8] = __float2bfloat16_rn(av[mt][2 + j]);
+              }
             }
           }
         }
@@ -521,13 +534,12 @@ cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* 
 cudaError_t launch_backward_dkdv(const void* grad_out, const void* q, const uint16_t* pds, const int64_t* quad_ent,
                                  const int32_t* wl_cnt, const int4* wl, int p, int64_t n_quads, int64_t T_kv,
                                  int G, int n_sel, float scale, float* partial, void* dk, void* dv,
-                                 cudaStream_t s) {
+                                 bool f32_out, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
   if (e != cudaSuccess) return e;
   dkdv_kernel<<<static_cast<unsigned>(kKvCtasPerSm * sm_count()), kKvThreads, kKvSmem, s>>>(
       static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q), pds, quad_ent, wl_cnt + p,
-      wl + static_cast<int64_t>(p) * n_quads, T_kv, G, n_sel, scale, partial, static_cast<__nv_bfloat16*>(dk),
-      static_cast<__nv_bfloat16*>(dv));
+      wl + static_cast<int64_t>(p) * n_quads, T_kv, G, n_sel, scale, partial, dk, dv, f32_out);
   return cudaGetLastError();
 }
 

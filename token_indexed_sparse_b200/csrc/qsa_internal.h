@@ -28,9 +28,11 @@ cudaError_t launch_quad_fill(const int32_t* row_cnt, const int32_t* row_cols, in
 cudaError_t launch_quad_sort(const int32_t* quad_ptr, int64_t n_quads, int64_t* quad_ent, int P, int C,
                              int32_t* phase_ptr, cudaStream_t s);
 // Per-phase work lists of non-empty (quad, entry range) items (wl_cnt zeroed by
-// the caller); zeroes dK/dV of quads that no query routes to.
+// the caller); zeroes dK/dV (BF16, or FP32 when f32_out) of quads that no query
+// routes to.
 cudaError_t launch_quad_worklist(const int32_t* quad_ptr, const int32_t* phase_ptr, int64_t n_quads, int64_t T_kv,
-                                 int G, int P, int32_t* wl_cnt, int4* wl, void* dk, void* dv, cudaStream_t s);
+                                 int G, int P, int32_t* wl_cnt, int4* wl, void* dk, void* dv, bool f32_out,
+                                 cudaStream_t s);
 
 // Attention kernels (qsa_forward.cu, qsa_backward.cu).
 cudaError_t launch_forward(const void* q, const void* k, const void* v, const int32_t* row_cnt,
@@ -45,11 +47,12 @@ cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* 
 // SM count of the current device (cached).
 int sm_count();
 // dK/dV over the work list of query phase p: accumulates each item's entries
-// onto its quad, reading / writing FP32 partials between phases.
+// onto its quad, reading / writing FP32 partials between phases; the final
+// dK/dV are BF16, or FP32 when f32_out.
 cudaError_t launch_backward_dkdv(const void* grad_out, const void* q, const uint16_t* pds, const int64_t* quad_ent,
                                  const int32_t* wl_cnt, const int4* wl, int p, int64_t n_quads, int64_t T_kv,
                                  int G, int n_sel, float scale, float* partial, void* dk, void* dv,
-                                 cudaStream_t s);
+                                 bool f32_out, cudaStream_t s);
 
 // Bitmap selection -> route IDs (qsa_bitmap.cu); zeroes *max_cnt first when given.
 cudaError_t launch_bitmap_routes(const uint8_t* sel, const int32_t* lo, const int32_t* hi, const int32_t* blk_base,

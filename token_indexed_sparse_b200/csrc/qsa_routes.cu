@@ -366,17 +366,18 @@ __global__ void __launch_bounds__(kSortThreads) quad_sort_kernel(const int32_t* 
 // does not matter: each item accumulates its own quad, in list order.
 __global__ void __launch_bounds__(256) quad_worklist_kernel(
     const int32_t* __restrict__ ptr, const int32_t* __restrict__ phase_ptr, int64_t n_quads, int64_t T_kv, int G,
-    int P, int32_t* __restrict__ wl_cnt, int4* __restrict__ wl, __nv_bfloat16* __restrict__ dk,
-    __nv_bfloat16* __restrict__ dv) {
+    int P, int32_t* __restrict__ wl_cnt, int4* __restrict__ wl, uint8_t* __restrict__ dk,
+    uint8_t* __restrict__ dv, int out_bytes) {
   const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (b >= n_quads) return;
   const int q0 = ptr[b], q1 = ptr[b + 1];
   if (q0 == q1) {
     const int64_t k_end = min(T_kv, 4 * b + 4);
+    const int64_t row = static_cast<int64_t>(G) * kHeadDim * out_bytes;  // bytes per key
     for (int64_t key = 4 * b; key < k_end; ++key) {
-      uint4* rk = reinterpret_cast<uint4*>(dk + key * G * kHeadDim);
-      uint4* rv = reinterpret_cast<uint4*>(dv + key * G * kHeadDim);
-      for (int i = 0; i < G * kHeadDim / 8; ++i) rk[i] = rv[i] = make_uint4(0, 0, 0, 0);
+      uint4* rk = reinterpret_cast<uint4*>(dk + key * row);
+      uint4* rv = reinterpret_cast<uint4*>(dv + key * row);
+      for (int64_t i = 0; i < row / 16; ++i) rk[i] = rv[i] = make_uint4(0, 0, 0, 0);
     }
     return;
   }
@@ -449,10 +450,11 @@ cudaError_t launch_quad_sort(const int32_t* quad_ptr, int64_t n_quads, int64_t* 
 }
 
 cudaError_t launch_quad_worklist(const int32_t* quad_ptr, const int32_t* phase_ptr, int64_t n_quads, int64_t T_kv,
-                                 int G, int P, int32_t* wl_cnt, int4* wl, void* dk, void* dv, cudaStream_t s) {
+                                 int G, int P, int32_t* wl_cnt, int4* wl, void* dk, void* dv, bool f32_out,
+                                 cudaStream_t s) {
   quad_worklist_kernel<<<static_cast<unsigned>((n_quads + 255) / 256), 256, 0, s>>>(
-      quad_ptr, phase_ptr, n_quads, T_kv, G, P, wl_cnt, wl, static_cast<__nv_bfloat16*>(dk),
-      static_cast<__nv_bfloat16*>(dv));
+      quad_ptr, phase_ptr, n_quads, T_kv, G, P, wl_cnt, wl, static_cast<uint8_t*>(dk), static_cast<uint8_t*>(dv),
+      f32_out ? 4 : 2);
   return cudaGetLastError();
 }
 

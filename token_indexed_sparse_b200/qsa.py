@@ -63,6 +63,8 @@ def library() -> ctypes.CDLL:
     lib.qsa_selector_scores.argtypes = [vp, vp, i64, i64, i32, i32, f32, vp, vp, vp, vp, i64, vp, vp]
     lib.qsa_selector_topk.restype = i32
     lib.qsa_selector_topk.argtypes = [vp, i64, i64, i64, i32, vp, vp, vp, vp, vp, vp]
+    lib.qsa_backward_fp32kv.restype = i32
+    lib.qsa_backward_fp32kv.argtypes = lib.qsa_backward.argtypes
     lib.qsa_route_plan_scratch_size.restype = sz
     lib.qsa_route_plan_scratch_size.argtypes = [i64, i64]
     lib.qsa_route_plan.restype = i32
@@ -165,11 +167,13 @@ def forward(q, k, v, routes, scale: float = 1.0 / 16.0, *, out=None, lse=None, w
 
 
 def backward(grad_out, q, k, v, out, lse, routes, scale: float = 1.0 / 16.0, *,
-             dq=None, dk=None, dv=None, workspace=None, stage_events=None):
+             dq=None, dk=None, dv=None, workspace=None, stage_events=None, kv_fp32: bool = False):
     """qsa_backward: returns ``(dq, dk, dv)`` (bf16, shapes of q, k, v).
 
     ``stage_events`` (optional, up to 6 torch.cuda.Event) are recorded after
-    each backward stage (qsa_backward_ex)."""
+    each backward stage (qsa_backward_ex).  With ``kv_fp32`` dk and dv are FP32
+    (qsa_backward_fp32kv: the sums before the BF16 rounding, for adding partials
+    from several calls)."""
     lib = library()
     grad_out = _prep(grad_out, torch.bfloat16, "grad_out")
     q = _prep(q, torch.bfloat16, "q")
@@ -179,15 +183,25 @@ def backward(grad_out, q, k, v, out, lse, routes, scale: float = 1.0 / 16.0, *,
     lse = _prep(lse, torch.float32, "lse")
     routes = _prep(routes, torch.int32, "routes")
     T, T_kv, H, G, n_sel = _sizes(q, k, routes)
+    kv_dtype = torch.float32 if kv_fp32 else torch.bfloat16
     dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
+    dk = torch.empty(k.shape, dtype=kv_dtype, device=k.device) if dk is None else dk
+    dv = torch.empty(v.shape, dtype=kv_dtype, device=v.device) if dv is None else dv
+    if dk.dtype != kv_dtype or dv.dtype != kv_dtype:
+        raise TypeError(f"dk / dv must be {kv_dtype}")
     ws_bytes = lib.qsa_backward_workspace_size(T, T_kv, H, G, n_sel)
     ws = _workspace(ws_bytes, q.device, workspace)
-    ev, n_ev = _events(stage_events)
-    st = lib.qsa_backward_ex(_ptr(grad_out), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(routes),
-                             T, T_kv, H, G, n_sel, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
-                             _ptr(ws), ws.numel(), _stream(q.device), ev, n_ev)
+    if kv_fp32:
+        if stage_events:
+            raise ValueError("stage events are not recorded by the FP32 dK/dV backward")
+        st = lib.qsa_backward_fp32kv(_ptr(grad_out), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(routes),
+                                     T, T_kv, H, G, n_sel, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+                                     _ptr(ws), ws.numel(), _stream(q.device))
+    else:
+        ev, n_ev = _events(stage_events)
+        st = lib.qsa_backward_ex(_ptr(grad_out), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(routes),
+                                 T, T_kv, H, G, n_sel, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+                                 _ptr(ws), ws.numel(), _stream(q.device), ev, n_ev)
     _check(st, "qsa_backward")
     return dq, dk, dv
 
