@@ -19,4 +19,5 @@ from .qsa_oracle import (  # noqa: F401
     backward_keys,
     route_rows_csr,
     key_quad_lists,
+    key_tile_lists,
 )

@@ -123,6 +123,34 @@ def key_quad_lists(routes, kv_length: int):
     return ptr, np.asarray(qs, dtype=np.int32), np.asarray(ms, dtype=np.int32)
 
 
+
+def key_tile_lists(routes, kv_length: int, tile: int = 128):
+    """Key -> query transpose of the route sets, grouped by aligned key tiles.
+
+    The reverse lists of [FA4] ``_preprocess`` at a granularity of ``tile``
+    keys: tile ``b`` covers keys ``tile*b .. tile*b + tile - 1``.  For each
+    tile, the queries whose route set meets it are listed in ascending order,
+    each with ``i0`` = the number of keys of R_t below the tile (the position of
+    its first key in the sorted row) and ``n`` = the number of keys of R_t in
+    the tile.
+
+    Returns ``(tile_ptr [n_tiles+1] int64, query [E] int32, i0 [E] int32,
+    n [E] int32)`` with ``n_tiles = ceil(kv_length / tile)``.
+    """
+    n_tiles = (kv_length + tile - 1) // tile
+    per_tile = [[] for _ in range(n_tiles)]
+    for t, s in enumerate(row_route_sets(routes, kv_length)):
+        tiles = s // tile
+        for b in np.unique(tiles):
+            pos = np.nonzero(tiles == b)[0]
+            per_tile[int(b)].append((t, int(pos[0]), int(pos.size)))
+    ptr = np.zeros(n_tiles + 1, dtype=np.int64)
+    for b in range(n_tiles):
+        ptr[b + 1] = ptr[b] + len(per_tile[b])
+    flat = [e for lst in per_tile for e in lst]   # rows were visited in ascending t
+    cols = np.asarray(flat, dtype=np.int32).reshape(-1, 3)
+    return ptr, cols[:, 0].copy(), cols[:, 1].copy(), cols[:, 2].copy()
+
 # ---------------------------------------------------------------------------
 # Dense-table form: the definition, for finite inputs
 # ---------------------------------------------------------------------------

@@ -332,3 +332,35 @@ def test_route_rows_csr_and_quad_lists():
                 entries.append((t, m))
         got = list(zip(qry[ptr[b]:ptr[b + 1]].tolist(), msk[ptr[b]:ptr[b + 1]].tolist()))
         assert got == entries
+
+
+@pytest.mark.parametrize("tile", [4, 8, 128])
+def test_key_tile_lists(tile):
+    # brute force from the membership table: the rows meeting each tile, the
+    # count of their keys below it and inside it
+    rng = np.random.default_rng(29)
+    T, T_kv = 45, 301
+    routes = _random_routes(rng, T, T_kv, 40)
+    routes[7] = -1
+    routes[8] = np.arange(40) % 3                      # duplicates inside one tile
+    M = oracle.routes_to_membership(routes, T_kv)
+    ptr, qry, i0, n = oracle.key_tile_lists(routes, T_kv, tile)
+    n_tiles = (T_kv + tile - 1) // tile
+    assert len(ptr) == n_tiles + 1 and ptr[-1] == len(qry) == len(i0) == len(n)
+    for b in range(n_tiles):
+        lo, hi = tile * b, min(T_kv, tile * (b + 1))
+        rows = [t for t in range(T) if M[t, lo:hi].any()]
+        got = list(zip(qry[ptr[b]:ptr[b + 1]].tolist(), i0[ptr[b]:ptr[b + 1]].tolist(),
+                       n[ptr[b]:ptr[b + 1]].tolist()))
+        assert got == [(t, int(M[t, :lo].sum()), int(M[t, lo:hi].sum())) for t in rows]
+
+
+def test_key_tile_lists_refine_quads():
+    # tiles of 4 keys are the quads: same rows, and n = popcount of the owner mask
+    rng = np.random.default_rng(31)
+    routes = _random_routes(rng, 30, 64, 20)
+    qptr, qq, qm = oracle.key_quad_lists(routes, 64)
+    tptr, tq, _, tn = oracle.key_tile_lists(routes, 64, 4)
+    np.testing.assert_array_equal(qptr, tptr)
+    np.testing.assert_array_equal(qq, tq)
+    np.testing.assert_array_equal([bin(int(m)).count("1") for m in qm], tn)
