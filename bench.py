@@ -62,7 +62,7 @@ def stage_traffic(stage):
 
 
 FWD_STAGES = ["fwd_route_rows", "fwd_attention"]
-BWD_STAGES = ["bwd_route_rows", "bwd_quad_scan", "bwd_quad_fill", "bwd_quad_sort", "bwd_dq", "bwd_dkdv"]
+BWD_STAGES = ["bwd_route_rows", "bwd_tile_scan", "bwd_tile_fill", "bwd_tile_sort", "bwd_dq", "bwd_dkdv"]
 
 
 def load_peaks():

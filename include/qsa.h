@@ -138,8 +138,8 @@ qsa_status_t qsa_backward_fp32kv(const void* grad_out, const void* q, const void
  * `stage_events` may be NULL when n_stage_events is 0.  The paper has no
  * counterpart: this is an instrumentation hook of this library.
  *   forward stages : 0 route rows (sort/dedup), 1 attention forward
- *   backward stages: 0 route rows + quad counts, 1 quad scan, 2 quad fill,
- *                    3 quad sort, 4 dQ (+ delta, P/dS records), 5 dK/dV
+ *   backward stages: 0 route rows (+ delta), 1 tile counts + scan, 2 tile fill,
+ *                    3 tile sort + work lists, 4 dQ (+ P/dS records), 5 dK/dV
  * A failed eventRecord returns QSA_ERR_CUDA.
  */
 typedef struct CUevent_st* qsa_event_t; /* same type as cudaEvent_t */
@@ -160,12 +160,11 @@ qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k,
 
 /*
  * Number of kernels one qsa_forward (backward = 0) or qsa_backward (backward = 1)
- * call enqueues for these sizes, not counting the cudaMemsetAsync nodes of the
- * backward (two).  The forward launches 2; the backward launches 6 plus one dK/dV
- * launch per query phase, where a phase spans as many consecutive queries as keep
- * their Q and dO rows (H KB per query) within 48 MiB of L2 (at most 64 phases).
- * Returns 0 for sizes the calls reject.  For instrumentation and for sizing CUDA
- * graphs; the paper has no counterpart.
+ * call enqueues for these sizes, not counting the cudaMemsetAsync node of the
+ * backward (one).  The forward launches 2 (route rows, attention); the backward
+ * 8 (route rows, tile counts, tile scan, tile fill, tile sort, work lists, dQ,
+ * dK/dV).  Returns 0 for sizes the calls reject.  For instrumentation and for
+ * sizing CUDA graphs; the pages have no counterpart.
  */
 int qsa_launch_count(int64_t T, int64_t T_kv, int H, int G, int n_sel, int backward);
 
@@ -190,6 +189,26 @@ qsa_status_t qsa_route_plan(const int32_t* routes, int64_t T, int64_t T_kv, int 
                             int32_t* row_cnt, int32_t* row_cols, int32_t* quad_ptr,
                             int64_t* quad_ent, void* scratch, size_t scratch_bytes,
                             qsa_stream_t stream);
+
+/*
+ * The key->query transpose the backward's dK/dV pass walks, on its own: the
+ * reverse lists of the "fa4_qsa" page's `_preprocess` grouped by aligned tiles
+ * of 128 keys instead of single keys.
+ *   row_cnt, row_cols : as qsa_route_plan
+ *   tile_ptr [ceil(T_kv/128)+1] int32 : CSR offsets of the tile lists
+ *   tile_ent [T * n_sel] int64 : for tile b (keys 128b..128b+127), entries
+ *       tile_ent[tile_ptr[b] .. tile_ptr[b+1]) in ascending query order, each
+ *       (t << 32) | (i0 << 8) | (n - 1), where t is a query whose R_t meets the
+ *       tile, n (1..128) is the number of keys of R_t in the tile and
+ *       row_cols[t, i0 .. i0 + n) are those keys.  Slots past tile_ptr[last]
+ *       are left unspecified.
+ *   scratch: qsa_tile_plan_scratch_size(T, T_kv) bytes, 256-byte aligned.
+ * Same size limits and errors as qsa_route_plan.
+ */
+size_t qsa_tile_plan_scratch_size(int64_t T, int64_t T_kv);
+qsa_status_t qsa_tile_plan(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel, int32_t* row_cnt,
+                           int32_t* row_cols, int32_t* tile_ptr, int64_t* tile_ent, void* scratch,
+                           size_t scratch_bytes, qsa_stream_t stream);
 
 /*
  * Block-selection bitmap -> route IDs, so that callers of the bitmap API can use

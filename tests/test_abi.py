@@ -60,9 +60,9 @@ def test_launch_counts(lib):
     # forward: route rows + attention; backward: 6 kernels + one dK/dV launch per
     # query phase of 48 MiB / (H KB) queries (2048 at H = 24, 4096 at H = 12)
     assert lib.qsa_launch_count(32768, 32768, 24, 2, 564, 0) == 2
-    assert lib.qsa_launch_count(32768, 32768, 24, 2, 564, 1) == 6 + 16
-    assert lib.qsa_launch_count(16384, 16384, 12, 1, 512, 1) == 6 + 4
-    assert lib.qsa_launch_count(256, 256, 12, 1, 64, 1) == 6 + 1
+    assert lib.qsa_launch_count(32768, 32768, 24, 2, 564, 1) == 8
+    assert lib.qsa_launch_count(16384, 16384, 12, 1, 512, 1) == 8
+    assert lib.qsa_launch_count(256, 256, 12, 1, 64, 1) == 8
     assert lib.qsa_launch_count(16, 16, 8, 1, 4, 1) == 0
 
 
@@ -97,6 +97,13 @@ def test_host_validation_before_any_launch(lib):
     assert st == 4
     st = lib.qsa_route_plan(P(256), 16, 16, 4, P(256), P(256), P(256), P(260), P(256), 1 << 20, None)
     assert st == 3                                   # int64 entries need 8-byte alignment
+    st = lib.qsa_tile_plan(P(256), 16, 16, 4, P(256), P(256), P(256), P(260), P(256), 1 << 20, None)
+    assert st == 3
+    st = lib.qsa_tile_plan(P(256), 16, 16, 4, P(256), P(0), P(256), P(256), P(256), 1 << 20, None)
+    assert st == 1                                   # null row_cols
+    st = lib.qsa_tile_plan(P(256), 16, 16, 4, P(256), P(256), P(256), P(256), P(256), 8, None)
+    assert st == 4                                   # scratch too small
+    assert lib.qsa_tile_plan_scratch_size(16, 300) == 2 * 256 + 256
 
 
 def test_bitmap_routes_host_validation(lib):

@@ -171,6 +171,53 @@ def test_route_plan_long_quad_list():
     _check_plan(routes, T_kv)
 
 
+def _check_tile_plan(routes, T_kv):
+    r = torch.from_numpy(np.array(routes, dtype=np.int32)).to(DEV)
+    row_cnt, row_cols, tile_ptr, tile_ent = (x.cpu().numpy() for x in qsa.tile_plan(r, T_kv))
+    cnt, cols = oracle.route_rows_csr(routes, T_kv)
+    np.testing.assert_array_equal(row_cnt, cnt)
+    ptr, qry, i0, n = oracle.key_tile_lists(routes, T_kv)
+    np.testing.assert_array_equal(tile_ptr, ptr)
+    ent = tile_ent[: ptr[-1]]
+    np.testing.assert_array_equal(ent >> 32, qry)
+    np.testing.assert_array_equal((ent >> 8) & 0x3FFF, i0)
+    np.testing.assert_array_equal((ent & 0x7F) + 1, n)
+
+
+@pytest.mark.parametrize("number,T", [(1, None), (2, 512), (3, 1024), (4, 768), (5, 256)])
+def test_tile_plan_bitexact(number, T):
+    wl = W.CONFIGS[number] if T is None else W.CONFIGS[number].scaled(T)
+    _check_tile_plan(W.make_routes(wl), wl.T_kv)
+
+
+def test_tile_plan_edge_rows():
+    rng = np.random.default_rng(6)
+    T, T_kv = 300, 397                                  # ragged last tile (keys 384..396)
+    routes = rng.integers(-50, T_kv + 50, size=(T, 150)).astype(np.int32)
+    routes[3] = -1
+    routes[4] = 396
+    routes[5, :128] = np.arange(128, 256)               # one full tile: n = 128
+    routes[5, 128:] = -1
+    routes[6] = np.arange(150) % 5                      # duplicates inside one tile
+    _check_tile_plan(routes, T_kv)
+
+
+def test_tile_plan_long_list():
+    # 20000 queries meet tile 0: its list is longer than the in-shared-memory sort
+    T, T_kv = 20000, 300
+    routes = np.tile(np.array([[3, 1, 200, 0, -1]], dtype=np.int32), (T, 1))
+    routes[::7, 0] = 299
+    _check_tile_plan(routes, T_kv)
+
+
+def test_tile_plan_many_tiles():
+    # more tiles than the shared-memory histograms hold (global-atomic path)
+    rng = np.random.default_rng(8)
+    T, T_kv = 64, 128 * 9000
+    routes = rng.integers(0, T_kv, size=(T, 40)).astype(np.int32)
+    _check_tile_plan(routes, T_kv)
+
+
 # ---------------------------------------------------------------------------
 # edge cases
 # ---------------------------------------------------------------------------

@@ -41,10 +41,17 @@ void dkdv_phases(int64_t T, int H, int* P, int* C) {
 }
 
 struct Layout {
-  size_t status = 0, row_cnt = 0, row_cols = 0, quad_cnt = 0, quad_ptr = 0, quad_fill = 0, quad_ent = 0,
-         delta = 0, pds = 0, phase_ptr = 0, wl_cnt = 0, wl = 0, partial = 0, total = 0;
+  size_t status = 0, row_cnt = 0, row_cols = 0, tile_ctr = 0, tile_ptr = 0, tile_fill = 0, tile_ent = 0, delta = 0,
+         prec = 0, dsrec = 0, phase_ptr = 0, wl = 0, partial = 0, total = 0;
   int P = 1, C = 1;
 };
+
+// Counters zeroed by one memset at the start of a backward call: per-tile row
+// counts [n_tiles], per-phase work-list sizes [P], the dK/dV unit claim counter
+// [1], and per (tile, group, tensor) the number of phases accumulated [n_tiles * 2G].
+size_t tile_ctr_ints(int64_t n_tiles, int P, int G) {
+  return static_cast<size_t>(n_tiles) * (1 + 2 * static_cast<size_t>(G)) + static_cast<size_t>(P) + 1;
+}
 
 Layout make_layout(int64_t T, int64_t T_kv, int H, int G, int n_sel, bool backward) {
   Layout L;
@@ -54,23 +61,23 @@ Layout make_layout(int64_t T, int64_t T_kv, int H, int G, int n_sel, bool backwa
     off = align256(off + bytes);
     return at;
   };
-  const size_t nq = static_cast<size_t>((T_kv + 3) / 4);
+  const size_t nt = static_cast<size_t>((T_kv + 127) / 128);  // 128-key tiles
   const size_t pairs = static_cast<size_t>(T) * static_cast<size_t>(n_sel);
   L.status = take(4);
   L.row_cnt = take(static_cast<size_t>(T) * 4);
   L.row_cols = take(pairs * 4);
   if (backward) {
-    L.quad_cnt = take(nq * 4);
-    L.quad_ptr = take((nq + 1) * 4);
-    L.quad_fill = take(nq * 4);
-    L.quad_ent = take(pairs * 8);
-    L.delta = take(static_cast<size_t>(T) * H * 4);
-    L.pds = take(pairs * G * 48);
     dkdv_phases(T, H, &L.P, &L.C);
-    L.phase_ptr = take(nq * (L.P + 1) * 4);
-    L.wl_cnt = take(static_cast<size_t>(L.P) * 4);
-    L.wl = take(static_cast<size_t>(L.P) * nq * 16);
-    L.partial = take(nq * G * 2048 * 4);
+    L.tile_ctr = take(tile_ctr_ints(static_cast<int64_t>(nt), L.P, G) * 4);
+    L.tile_ptr = take((nt + 1) * 4);
+    L.tile_fill = take(nt * 4);
+    L.tile_ent = take(pairs * 8);  // at most one entry per routed pair
+    L.delta = take(static_cast<size_t>(T) * H * 4);
+    L.prec = take(pairs * G * 24);   // BF16 P of every routed pair, 12 heads
+    L.dsrec = take(pairs * G * 24);  // BF16 dS
+    L.phase_ptr = take(nt * (L.P + 1) * 4);
+    L.wl = take(static_cast<size_t>(L.P) * nt * 16);
+    L.partial = take(nt * G * 2 * 128 * 256 * 4);  // FP32 dK and dV of every (tile, group)
   }
   L.total = off;
   return L;
@@ -118,39 +125,41 @@ static qsa_status_t backward_impl(const void* grad_out, const void* q, const voi
   const Layout L = make_layout(T, T_kv, H, G, n_sel, true);
   if (workspace_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t nq = (T_kv + 3) / 4;
+  const int64_t nt = (T_kv + 127) / 128;
   int* status = at<int>(workspace, L.status);
   int32_t* row_cnt = at<int32_t>(workspace, L.row_cnt);
   int32_t* row_cols = at<int32_t>(workspace, L.row_cols);
-  int32_t* quad_cnt = at<int32_t>(workspace, L.quad_cnt);
-  int32_t* quad_ptr = at<int32_t>(workspace, L.quad_ptr);
-  int32_t* quad_fill = at<int32_t>(workspace, L.quad_fill);
-  int64_t* quad_ent = at<int64_t>(workspace, L.quad_ent);
+  int32_t* tile_cnt = at<int32_t>(workspace, L.tile_ctr);
+  int32_t* wl_cnt = tile_cnt + nt;
+  int32_t* claim = wl_cnt + L.P;
+  int32_t* done = claim + 1;
+  int32_t* tile_ptr = at<int32_t>(workspace, L.tile_ptr);
+  int32_t* tile_fill = at<int32_t>(workspace, L.tile_fill);
+  int64_t* tile_ent = at<int64_t>(workspace, L.tile_ent);
   float* delta = at<float>(workspace, L.delta);
-  uint16_t* pds = at<uint16_t>(workspace, L.pds);
+  uint16_t* prec = at<uint16_t>(workspace, L.prec);    // P  [T, G, n_sel, 12]
+  uint16_t* dsrec = at<uint16_t>(workspace, L.dsrec);  // dS [T, G, n_sel, 12]
   int32_t* phase_ptr = at<int32_t>(workspace, L.phase_ptr);
-  int32_t* wl_cnt = at<int32_t>(workspace, L.wl_cnt);
   int4* wl = at<int4>(workspace, L.wl);
   float* partial = at<float>(workspace, L.partial);
   const StageEvents ev{stage_events, n_stage_events, s};
-  QSA_TRY(cudaMemsetAsync(quad_cnt, 0, static_cast<size_t>(nq) * 4, s));
-  QSA_TRY(cudaMemsetAsync(wl_cnt, 0, static_cast<size_t>(L.P) * 4, s));
-  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, quad_cnt, status, grad_out, out, delta,
+  QSA_TRY(cudaMemsetAsync(tile_cnt, 0, tile_ctr_ints(nt, L.P, G) * 4, s));
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 0, status, grad_out, out, delta,
                                  H, s));
   QSA_TRY(ev.mark(0));
-  QSA_TRY(qsa::launch_quad_scan(quad_cnt, nq, quad_ptr, quad_fill, s));
+  QSA_TRY(qsa::launch_tile_count(row_cnt, row_cols, T, n_sel, nt, tile_cnt, s));
+  QSA_TRY(qsa::launch_quad_scan(tile_cnt, nt, tile_ptr, tile_fill, s));
   QSA_TRY(ev.mark(1));
-  QSA_TRY(qsa::launch_quad_fill(row_cnt, row_cols, T, n_sel, quad_fill, quad_ent, s));
+  QSA_TRY(qsa::launch_tile_fill(row_cnt, row_cols, T, n_sel, nt, tile_fill, tile_ent, s));
   QSA_TRY(ev.mark(2));
-  QSA_TRY(qsa::launch_quad_sort(quad_ptr, nq, quad_ent, L.P, L.C, phase_ptr, s));
-  QSA_TRY(qsa::launch_quad_worklist(quad_ptr, phase_ptr, nq, T_kv, G, L.P, wl_cnt, wl, dk, dv, kv_f32, s));
+  QSA_TRY(qsa::launch_tile_sort(tile_ptr, nt, tile_ent, L.P, L.C, phase_ptr, s));
+  QSA_TRY(qsa::launch_tile_worklist(tile_ptr, phase_ptr, nt, T_kv, G, L.P, wl_cnt, wl, dk, dv, kv_f32, s));
   QSA_TRY(ev.mark(3));
-  QSA_TRY(qsa::launch_backward_dq(grad_out, q, k, v, lse, delta, row_cnt, row_cols, T, G, n_sel, scale, dq, pds,
-                                  s));
+  QSA_TRY(qsa::launch_backward_dq(grad_out, q, k, v, lse, delta, row_cnt, row_cols, T, G, n_sel, scale, dq, prec,
+                                  dsrec, s));
   QSA_TRY(ev.mark(4));
-  for (int p = 0; p < L.P; ++p)
-    QSA_TRY(qsa::launch_backward_dkdv(grad_out, q, pds, quad_ent, wl_cnt, wl, p, nq, T_kv, G, n_sel, scale, partial,
-                                      dk, dv, kv_f32, s));
+  QSA_TRY(qsa::launch_backward_dkdv_union(grad_out, q, prec, dsrec, row_cols, tile_ent, wl_cnt, wl, claim, done,
+                                          L.P, nt, T_kv, G, n_sel, scale, partial, dk, dv, kv_f32, status, s));
   QSA_TRY(ev.mark(5));
   return QSA_OK;
 }
@@ -206,7 +215,7 @@ qsa_status_t qsa_forward_ex(const void* q, const void* k, const void* v, const i
   int32_t* row_cnt = at<int32_t>(workspace, L.row_cnt);
   int32_t* row_cols = at<int32_t>(workspace, L.row_cols);
   const StageEvents ev{stage_events, n_stage_events, s};
-  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, status, nullptr, nullptr,
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 2, status, nullptr, nullptr,
                                  nullptr, H, s));
   QSA_TRY(ev.mark(0));
   QSA_TRY(qsa::launch_forward(q, k, v, row_cnt, row_cols, T, G, n_sel, scale, out, lse, status, s));
@@ -241,10 +250,7 @@ qsa_status_t qsa_backward_fp32kv(const void* grad_out, const void* q, const void
 
 int qsa_launch_count(int64_t T, int64_t T_kv, int H, int G, int n_sel, int backward) {
   if (check_sizes(T, T_kv, H, G, n_sel) != QSA_OK) return 0;
-  if (!backward) return 2;
-  int P = 1, C = 1;
-  dkdv_phases(T, H, &P, &C);
-  return 6 + P;
+  return backward ? 8 : 2;  // backward: route rows, tile count, scan, fill, sort + work list, dQ, dK/dV
 }
 
 qsa_status_t qsa_bitmap_routes(const uint8_t* sel_blocks, const int32_t* lo, const int32_t* hi,
@@ -314,11 +320,42 @@ qsa_status_t qsa_route_plan(const int32_t* routes, int64_t T, int64_t T_kv, int 
   int32_t* quad_fill = at<int32_t>(scratch, align256(static_cast<size_t>(nq) * 4));
   int32_t* phase_ptr = at<int32_t>(scratch, 2 * align256(static_cast<size_t>(nq) * 4));
   QSA_TRY(cudaMemsetAsync(quad_cnt, 0, static_cast<size_t>(nq) * 4, s));
-  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, quad_cnt, nullptr, nullptr, nullptr,
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, quad_cnt, 2, nullptr, nullptr, nullptr,
                                  nullptr, qsa::kHeadsPerGroup, s));
   QSA_TRY(qsa::launch_quad_scan(quad_cnt, nq, quad_ptr, quad_fill, s));
   QSA_TRY(qsa::launch_quad_fill(row_cnt, row_cols, T, n_sel, quad_fill, quad_ent, s));
   QSA_TRY(qsa::launch_quad_sort(quad_ptr, nq, quad_ent, 1, static_cast<int>(T), phase_ptr, s));
+  return QSA_OK;
+}
+
+size_t qsa_tile_plan_scratch_size(int64_t T, int64_t T_kv) {
+  if (T < 1 || T_kv < 1 || T_kv > INT32_MAX) return 0;
+  const size_t nt = static_cast<size_t>((T_kv + 127) / 128);
+  return 2 * align256(nt * 4) + align256(nt * 8);
+}
+
+qsa_status_t qsa_tile_plan(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel, int32_t* row_cnt,
+                           int32_t* row_cols, int32_t* tile_ptr, int64_t* tile_ent, void* scratch,
+                           size_t scratch_bytes, qsa_stream_t stream) {
+  if (!routes || !row_cnt || !row_cols || !tile_ptr || !tile_ent || !scratch) return QSA_ERR_INVALID_ARGUMENT;
+  const qsa_status_t st = check_sizes(T, T_kv, qsa::kHeadsPerGroup, 1, n_sel);
+  if (st != QSA_OK) return st;
+  if (!aligned(routes, 4) || !aligned(row_cnt, 4) || !aligned(row_cols, 4) || !aligned(tile_ptr, 4) ||
+      !aligned(tile_ent, 8) || !aligned(scratch, 256))
+    return QSA_ERR_MISALIGNED;
+  if (scratch_bytes < qsa_tile_plan_scratch_size(T, T_kv)) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t nt = (T_kv + 127) / 128;
+  int32_t* tile_cnt = static_cast<int32_t*>(scratch);
+  int32_t* tile_fill = at<int32_t>(scratch, align256(static_cast<size_t>(nt) * 4));
+  int32_t* phase_ptr = at<int32_t>(scratch, 2 * align256(static_cast<size_t>(nt) * 4));
+  QSA_TRY(cudaMemsetAsync(tile_cnt, 0, static_cast<size_t>(nt) * 4, s));
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 0, nullptr, nullptr, nullptr,
+                                 nullptr, qsa::kHeadsPerGroup, s));
+  QSA_TRY(qsa::launch_tile_count(row_cnt, row_cols, T, n_sel, nt, tile_cnt, s));
+  QSA_TRY(qsa::launch_quad_scan(tile_cnt, nt, tile_ptr, tile_fill, s));
+  QSA_TRY(qsa::launch_tile_fill(row_cnt, row_cols, T, n_sel, nt, tile_fill, tile_ent, s));
+  QSA_TRY(qsa::launch_tile_sort(tile_ptr, nt, tile_ent, 1, static_cast<int>(T), phase_ptr, s));
   return QSA_OK;
 }
 

@@ -5,17 +5,12 @@
 //   delta = rowsum(dO * out),  dP = dO V^T,  dS = P * (dP - delta),
 //   dQ = scale dS K,  dK = scale dS^T Q,  dV = P^T dO  (dK/dV summed over heads).
 //
-// Two kernels, neither using floating-point atomics:
-//   * dq_kernel, persistent over (query t, group g) items: recomputes S and dP
-//     over R_t (K/V rows gathered like the forward), forms P and dS with delta
-//     from the route kernel, accumulates dQ, and stores the BF16 P / dS of every
-//     routed pair (`pds`, one 48-byte record [P h0..h11 | dS h0..h11] per
-//     (t, g, position in R_t)).
-//   * dkdv_kernel, persistent over (aligned key quad, group g, query-phase range)
-//     work items: walks the quad's query list in ascending query order, stages
-//     each entry's Q / dO rows and P / dS records in shared memory and
-//     accumulates dK^T = Q^T dS and dV^T = dO^T P on tensor cores; the fixed list
-//     order makes dK/dV bitwise reproducible.
+// This file holds dq_kernel, persistent over (query t, group g) items: it
+// recomputes S and dP over R_t (K/V rows gathered like the forward), forms P
+// and dS with delta from the route kernel, accumulates dQ, and stores the BF16
+// P and dS of every routed pair for the dK/dV pass (qsa_dkdv_union.cu): two
+// arrays of 24-byte records, P [T, G, n_sel, 12] and dS [T, G, n_sel, 12], one
+// record per (t, g, position in R_t).  No floating-point atomics.
 #include "qsa_internal.h"
 #include "qsa_pipe.cuh"
 
@@ -33,7 +28,7 @@ namespace {
 // buffer.  Per chunk, warp w computes S = Q K^T and dP = dO V^T for keys
 // 8w..8w+7, P = exp2(S*scale*log2e - lse*log2e), dS = P (dP - delta), stores the
 // BF16 P / dS records and accumulates dQ[:, DPW*w : DPW*(w+1)] += dS K.
-constexpr int kRec = 24;  // bf16 per (t, g, key) record: 12 P + 12 dS
+constexpr int kRec = 24;  // bf16 per (t, g, key) staged in shared memory: 12 P + 12 dS
 constexpr int kFirst = 1, kLast = 2, kSlot = 4;
 
 template <int NW, int STAGES, int CPS>
@@ -71,7 +66,7 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
           const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
           const float* __restrict__ lse, const float* __restrict__ delta, const int32_t* __restrict__ row_cnt,
           const int32_t* __restrict__ row_cols, int64_t n_items, int G, int n_sel, float scale, float scale_log2,
-          __nv_bfloat16* __restrict__ dq, uint16_t* __restrict__ pds) {
+          __nv_bfloat16* __restrict__ dq, uint16_t* __restrict__ prec, uint16_t* __restrict__ dsrec) {
   using S_ = DqShape<NW, STAGES, CPS>;
   constexpr int KEYS = S_::kKeys, kTile = S_::kTile, kStageBytes = S_::kStageBytes, kDsStride = S_::kDsStride;
   constexpr int kNt = S_::kNt, kKs = S_::kKs, kItemBytes = S_::kItemBytes, kThreads = S_::kThreads;
@@ -205,23 +200,45 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
     const uint32_t D23 = pack_bf16(p2 * (dp[2] - dl1), p3 * (dp[3] - dl1));
     *reinterpret_cast<uint32_t*>(sDS + gq * kDsStride + key0) = D01;
     *reinterpret_cast<uint32_t*>(sDS + (gq + 8) * kDsStride + key0) = D23;
-    // records: [key][P h0..h11 | dS h0..h11]
-    sRec[key0 * kRec + gq] = static_cast<uint16_t>(P01 & 0xffff);
-    sRec[(key0 + 1) * kRec + gq] = static_cast<uint16_t>(P01 >> 16);
-    sRec[key0 * kRec + 12 + gq] = static_cast<uint16_t>(D01 & 0xffff);
-    sRec[(key0 + 1) * kRec + 12 + gq] = static_cast<uint16_t>(D01 >> 16);
+    // records: the chunk's P run [key][h0..h11], then its dS run
+    uint16_t* sD = sRec + KEYS * kHeadsPerGroup;
+    sRec[key0 * kHeadsPerGroup + gq] = static_cast<uint16_t>(P01 & 0xffff);
+    sRec[(key0 + 1) * kHeadsPerGroup + gq] = static_cast<uint16_t>(P01 >> 16);
+    sD[key0 * kHeadsPerGroup + gq] = static_cast<uint16_t>(D01 & 0xffff);
+    sD[(key0 + 1) * kHeadsPerGroup + gq] = static_cast<uint16_t>(D01 >> 16);
     if (gq + 8 < kHeadsPerGroup) {
-      sRec[key0 * kRec + gq + 8] = static_cast<uint16_t>(P23 & 0xffff);
-      sRec[(key0 + 1) * kRec + gq + 8] = static_cast<uint16_t>(P23 >> 16);
-      sRec[key0 * kRec + 20 + gq] = static_cast<uint16_t>(D23 & 0xffff);
-      sRec[(key0 + 1) * kRec + 20 + gq] = static_cast<uint16_t>(D23 >> 16);
+      sRec[key0 * kHeadsPerGroup + gq + 8] = static_cast<uint16_t>(P23 & 0xffff);
+      sRec[(key0 + 1) * kHeadsPerGroup + gq + 8] = static_cast<uint16_t>(P23 >> 16);
+      sD[key0 * kHeadsPerGroup + gq + 8] = static_cast<uint16_t>(D23 & 0xffff);
+      sD[(key0 + 1) * kHeadsPerGroup + gq + 8] = static_cast<uint16_t>(D23 >> 16);
     }
     __syncthreads();
     {
+      // the chunk's staged P and dS runs -> the same runs of the two record arrays
+      // (24 bytes per key; 16-byte stores when the run starts 16-byte aligned)
       const int base = (d.w >> 3) * KEYS;
-      const uint4* src = reinterpret_cast<const uint4*>(sRec);
-      uint4* dst = reinterpret_cast<uint4*>(pds + ((t * G + g) * n_sel + base) * kRec);
-      for (int i = tid; i < nk * 3; i += kThreads) dst[i] = src[i];
+      const int64_t r0 = ((t * G + g) * n_sel + base) * kHeadsPerGroup;
+      uint16_t* dp = prec + r0;
+      uint16_t* dd = dsrec + r0;
+      const uint16_t* sD = sRec + KEYS * kHeadsPerGroup;
+      const int words = nk * 3;  // 8-byte words per run
+      if (((reinterpret_cast<uintptr_t>(dp) | reinterpret_cast<uintptr_t>(dd)) & 15) == 0) {
+        const uint4* s4p = reinterpret_cast<const uint4*>(sRec);
+        const uint4* s4d = reinterpret_cast<const uint4*>(sD);
+        for (int i = tid; i < words / 2; i += kThreads) {
+          reinterpret_cast<uint4*>(dp)[i] = s4p[i];
+          reinterpret_cast<uint4*>(dd)[i] = s4d[i];
+        }
+        if ((words & 1) && tid == kThreads - 1) {
+          reinterpret_cast<uint2*>(dp)[words - 1] = reinterpret_cast<const uint2*>(sRec)[words - 1];
+          reinterpret_cast<uint2*>(dd)[words - 1] = reinterpret_cast<const uint2*>(sD)[words - 1];
+        }
+      } else {
+        for (int i = tid; i < words; i += kThreads) {
+          reinterpret_cast<uint2*>(dp)[i] = reinterpret_cast<const uint2*>(sRec)[i];
+          reinterpret_cast<uint2*>(dd)[i] = reinterpret_cast<const uint2*>(sD)[i];
+        }
+      }
     }
     // dQ[:, DPW*w : DPW*(w+1)] += dS K over the chunk's keys
 #pragma unroll
@@ -251,262 +268,6 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
   cp_async_wait<0>();
 }
 
-// ---------------------------------------------------------------------------
-// dK / dV per key quad, one query phase per launch
-// ---------------------------------------------------------------------------
-// Work item = (quad b, group g, entries [lo, hi) of b's ascending query list that
-// fall in the launch's query phase).  Items are dealt round-robin to persistent
-// CTAs (8 warps); each item's entries flow in chunks of 4 through a 4-stage ring:
-// all 12 Q rows and 12 dO rows of each entry (whole 512-byte rows, cp.async,
-// swizzled) and the entry's P/dS records placed by key slot (absent keys and
-// missing entries zero-filled).  Warp w owns dims [32w, 32w+32) and accumulates
-// dK^T += Q^T dS and dV^T += dO^T P with mma.sync: the A fragments come from
-// ldmatrix.trans of the staged rows and the K dimension packs head rows of
-// different entries of the same quad: k-step 0 = heads 0..7 of entries 0 and 1,
-// k-step 1 = the same for entries 2 and 3, k-step 2 = heads 8..11 of all four,
-// so no MMA slot or shared-memory read is spent on padding heads.  An item
-// starts from zero or from the FP32 partial of the previous phase and ends with
-// a partial or, on its last range, the BF16 result: the summation order is the
-// fixed list order, so dK/dV are bitwise reproducible.
-constexpr int kKvThreads = 256;
-constexpr int kKvStages = 2;
-constexpr int kKvCtasPerSm = 2;
-constexpr int kEnt = 4;                                   // entries per chunk
-constexpr int kKvRows = kEnt * 2 * kHeadsPerGroup;        // 96 staged rows per chunk
-constexpr int kKvRecOff = kKvRows * 512;                  // records after the rows
-constexpr int kKvRecBytes = kEnt * 4 * kRec * 2;          // 4 entries x 4 key slots x 48 B
-constexpr int kKvStageBytes = kKvRecOff + kKvRecBytes;
-constexpr int kKvOffDesc = kKvStages * kKvStageBytes;
-constexpr int kKvSmem = kKvOffDesc + kKvStages * 16;
-static_assert(kKvSmem <= 232448, "shared memory per block");
-static_assert(kKvStageBytes % 128 == 0, "alignment");
-constexpr int kItemFirst = 1, kItemLast = 2, kChFirst = 4, kChLast = 8;
-
-// Byte offset of 16-byte column c of stage row r, which belongs to entry u: the
-// 512-byte-row XOR swizzle with the phase of odd entries shifted by 4.
-__device__ __forceinline__ uint32_t swz_ent(int u, int r, int c) {
-  return static_cast<uint32_t>(r) * 512u + (static_cast<uint32_t>(c ^ ((r & 7) ^ ((u & 1) << 2))) << 4);
-}
-
-struct KvCursor {
-  int64_t w;        // work index (item = w / G, g = w % G); >= n_work when exhausted
-  int64_t wi;       // w / G, kept incrementally (no division in the loop)
-  int wg;           // w % G
-  int dt, dg;       // gridDim.x / G and gridDim.x % G
-  int4 item;        // (quad, lo, hi, flags) of the current work index
-  int4 item_next;   // of the next one (prefetched)
-  int ch, nch;
-};
-
-// Work-list item one grid stride after the cursor's, or zeros past the end.
-__device__ __forceinline__ int4 kv_item_next(const KvCursor& c, const int4* wl, int64_t n_work, int G) {
-  const int64_t wi_next = c.wi + c.dt + (c.wg + c.dg >= G ? 1 : 0);
-  return c.w + gridDim.x < n_work ? __ldg(wl + wi_next) : make_int4(0, 0, 0, 0);
-}
-
-__global__ void __launch_bounds__(kKvThreads, kKvCtasPerSm)
-dkdv_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ q,
-            const uint16_t* __restrict__ pds, const int64_t* __restrict__ quad_ent,
-            const int32_t* __restrict__ wl_cnt, const int4* __restrict__ wl, int64_t T_kv, int G, int n_sel,
-            float scale, float* __restrict__ partial, void* __restrict__ dk_out, void* __restrict__ dv_out,
-            bool f32_out) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const uint32_t sbase = smem_u32(smem);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int gq = lane >> 2, cq = lane & 3, mat = lane >> 3, rr = lane & 7;
-  const int H = G * kHeadsPerGroup;
-  int4* desc = reinterpret_cast<int4*>(smem + kKvOffDesc);
-  const int64_t n_work = static_cast<int64_t>(__ldg(wl_cnt)) * G;
-
-  KvCursor cur;
-  cur.w = blockIdx.x;
-  cur.wi = static_cast<int>(blockIdx.x) / G;
-  cur.wg = static_cast<int>(blockIdx.x) % G;
-  cur.dt = static_cast<int>(gridDim.x) / G;
-  cur.dg = static_cast<int>(gridDim.x) % G;
-  cur.item = cur.w < n_work ? __ldg(wl + cur.wi) : make_int4(0, 0, 0, 0);
-  cur.item_next = kv_item_next(cur, wl, n_work, G);
-  cur.ch = 0;
-  cur.nch = (cur.item.z - cur.item.y + kEnt - 1) / kEnt;
-  // Warp w copies the 12 rows (one contiguous 6 KB block) of entry w / 2,
-  // tensor w % 2, to rows u * 24 + tn * 12 + h of the stage; warps 0, 2, 4, 6
-  // also copy their entry's P/dS records.  Each warp loads only its own entry.
-  const int u_w = warp >> 1, tn_w = warp & 1;
-  const uint32_t row_off = static_cast<uint32_t>(u_w * 24 + tn_w * kHeadsPerGroup) * 512;
-  // Stage rows use the 512-byte-row swizzle with the phase of odd entries
-  // shifted by 4 (swz_ent): the k-step that packs heads 8..11 of entries 2j and
-  // 2j + 1 then reads eight distinct 16-byte bank groups.  For row
-  // u*24 + tn*12 + h the phase is (h & 7) ^ 4 (tn ^ (u & 1)).
-  const uint32_t xl4 = static_cast<uint32_t>(lane ^ ((tn_w ^ (u_w & 1)) << 2)) << 4;
-  int64_t ent = -1;
-  auto load_ent = [&]() {
-    const int e = cur.item.y + cur.ch * kEnt + u_w;
-    ent = (cur.w < n_work && e < cur.item.z) ? __ldg(quad_ent + e) : -1;
-  };
-  load_ent();
-
-  auto issue = [&](int stage) {
-    const uint32_t st = sbase + stage * kKvStageBytes;
-    if (cur.w < n_work) {
-      const int g = cur.wg;
-      const int n_ent = min(kEnt, cur.item.z - (cur.item.y + cur.ch * kEnt));
-      const bool live_u = u_w < n_ent;
-      const int64_t t = live_u ? (ent >> 32) : 0;
-      {
-        const __nv_bfloat16* src = (tn_w ? dout : q) + ((t * H + g * kHeadsPerGroup) * kHeadDim + lane * 8);
-        const uint32_t dst = st + row_off;
-#pragma unroll
-        for (int h = 0; h < kHeadsPerGroup; ++h)
-          cp_async16(dst + h * 512 + (xl4 ^ ((h & 7) << 4)), src + h * kHeadDim, live_u);
-      }
-      // records: lanes 0..11 of the tensor-0 warp of entry u copy (key slot, 16-byte part)
-      if (tn_w == 0 && lane < 12) {
-        const int slot = lane / 3, part = lane - 3 * slot;
-        const int mask = static_cast<int>(ent & 15);
-        const bool live = live_u && ((mask >> slot) & 1);
-        const int i0 = static_cast<int>((ent >> 4) & 0x0fffffff);
-        const int idx = live ? i0 + __popc(mask & ((1 << slot) - 1)) : 0;
-        const uint16_t* src = pds + (((live ? t : 0) * G + g) * n_sel + idx) * kRec + part * 8;
-        cp_async16(st + kKvRecOff + (u_w * 4 + slot) * (kRec * 2) + part * 16, src, live);
-      }
-      if (tid == 0) {
-        const int fl = (cur.item.w & 3) | (cur.ch == 0 ? kChFirst : 0) | (cur.ch == cur.nch - 1 ? kChLast : 0);
-        desc[stage] = make_int4(cur.item.x, g, n_ent, fl);
-      }
-    } else if (tid == 0) {
-      desc[stage] = make_int4(0, 0, -1, 0);
-    }
-    cp_async_commit();
-    // advance
-    if (cur.w < n_work && ++cur.ch == cur.nch) {
-      cur.w += gridDim.x;
-      cur.wi += cur.dt;
-      cur.wg += cur.dg;
-      if (cur.wg >= G) {
-        cur.wg -= G;
-        ++cur.wi;
-      }
-      cur.item = cur.item_next;
-      cur.item_next = kv_item_next(cur, wl, n_work, G);
-      cur.ch = 0;
-      cur.nch = (cur.item.z - cur.item.y + kEnt - 1) / kEnt;
-    }
-    load_ent();
-  };
-  for (int s0 = 0; s0 < kKvStages - 1; ++s0) issue(s0);
-
-  float ak[2][4], av[2][4];
-  for (int c = 0;; ++c) {
-    const int stage = c % kKvStages;
-    const uint32_t st = sbase + stage * kKvStageBytes;
-    cp_async_wait<kKvStages - 2>();
-    __syncthreads();  // chunk c has landed; every warp is done with chunk c - 1
-    const int4 d = desc[stage];
-    issue((c + kKvStages - 1) % kKvStages);
-    if (d.z < 0) break;
-    const int64_t b = d.x;
-    const int g = d.y;
-    const int fl = d.w;
-    float* part = partial + ((b * G + g) * 128 + warp * 16 + gq * 2 + (cq & 1)) * 16;
-    if (fl & kChFirst) {
-      if ((fl & kItemFirst) || cq >= 2) {
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-          for (int i = 0; i < 4; ++i) ak[mt][i] = av[mt][i] = 0.f;
-      } else {
-        const float4* src = reinterpret_cast<const float4*>(part);
-        const float4 x0 = src[0], x1 = src[1], x2 = src[2], x3 = src[3];
-        ak[0][0] = x0.x; ak[0][1] = x0.y; ak[0][2] = x0.z; ak[0][3] = x0.w;
-        ak[1][0] = x1.x; ak[1][1] = x1.y; ak[1][2] = x1.z; ak[1][3] = x1.w;
-        av[0][0] = x2.x; av[0][1] = x2.y; av[0][2] = x2.z; av[0][3] = x2.w;
-        av[1][0] = x3.x; av[1][1] = x3.y; av[1][2] = x3.z; av[1][3] = x3.w;
-      }
-    }
-#pragma unroll
-    for (int ks = 0; ks < 3; ++ks) {
-      // B fragments: P (dV) and dS (dK) of key slot gq for the k-step's head slots
-      uint32_t pb0 = 0, pb1 = 0, sb0 = 0, sb1 = 0;
-      if (gq < 4) {
-        int u0, u1, wp;
-        if (ks < 2) {
-          u0 = 2 * ks;
-          u1 = 2 * ks + 1;
-          wp = cq;
-        } else {
-          u0 = cq >> 1;
-          u1 = 2 + (cq >> 1);
-          wp = 4 + (cq & 1);
-        }
-        const uint32_t r0 = st + kKvRecOff + (u0 * 4 + gq) * (kRec * 2);
-        const uint32_t r1 = st + kKvRecOff + (u1 * 4 + gq) * (kRec * 2);
-        asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(pb0) : "r"(r0 + wp * 4));
-        asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(pb1) : "r"(r1 + wp * 4));
-        asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(sb0) : "r"(r0 + (6 + wp) * 4));
-        asm volatile("ld.shared.u32 %0, [%1];\n" : "=r"(sb1) : "r"(r1 + (6 + wp) * 4));
-      }
-      // A fragments: this lane addresses row (entry, head) of matrix `mat`
-      int u, h;
-      if (ks < 2) {
-        u = 2 * ks + (mat >> 1);
-        h = rr;
-      } else {
-        u = 2 * (mat >> 1) + (rr >> 2);
-        h = 8 + (rr & 3);
-      }
-#pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const int dch = warp * 4 + mt * 2 + (mat & 1);
-        uint32_t aq[4], ad[4];
-        ldsm_x4_t(aq, st + swz_ent(u, u * 24 + h, dch));
-        ldsm_x4_t(ad, st + swz_ent(u, u * 24 + kHeadsPerGroup + h, dch));
-        mma_16816(ak[mt], aq, sb0, sb1);
-        mma_16816(av[mt], ad, pb0, pb1);
-      }
-    }
-    if ((fl & kChLast) && cq < 2) {
-      if (fl & kItemLast) {
-        // C fragment of m-tile mt: (dim 32w+16mt+g | +8, key 2c | 2c+1)
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int64_t key = 4 * b + 2 * cq + j;
-          if (key < T_kv) {
-            const int64_t o = (key * G + g) * kHeadDim + warp * 32 + gq;
-            if (f32_out) {  // FP32 sums for callers that add partials before rounding
-              float* rk = static_cast<float*>(dk_out) + o;
-              float* rv = static_cast<float*>(dv_out) + o;
-#pragma unroll
-              for (int mt = 0; mt < 2; ++mt) {
-                rk[16 * mt] = ak[mt][j] * scale;
-                rk[16 * mt + 8] = ak[mt][2 + j] * scale;
-                rv[16 * mt] = av[mt][j];
-                rv[16 * mt + 8] = av[mt][2 + j];
-              }
-            } else {
-              __nv_bfloat16* rk = static_cast<__nv_bfloat16*>(dk_out) + o;
-              __nv_bfloat16* rv = static_cast<__nv_bfloat16*>(dv_out) + o;
-#pragma unroll
-              for (int mt = 0; mt < 2; ++mt) {
-                rk[16 * mt] = __float2bfloat16_rn(ak[mt][j] * scale);
-                rk[16 * mt + 8] = __float2bfloat16_rn(ak[mt][2 + j] * scale);
-                rv[16 * mt] = __float2bfloat16_rn(av[mt][j]);
-                rv[16 * mt + 8] = __float2bfloat16_rn(av[mt][2 + j]);
-              }
-            }
-          }
-        }
-      } else {
-        float4* dst = reinterpret_cast<float4*>(part);
-        dst[0] = make_float4(ak[0][0], ak[0][1], ak[0][2], ak[0][3]);
-        dst[1] = make_float4(ak[1][0], ak[1][1], ak[1][2], ak[1][3]);
-        dst[2] = make_float4(av[0][0], av[0][1], av[0][2], av[0][3]);
-        dst[3] = make_float4(av[1][0], av[1][1], av[1][2], av[1][3]);
-      }
-    }
-  }
-  cp_async_wait<0>();
-}
-
 }  // namespace
 
 // dQ kernel shape used by launch_backward_dq: 2 CTAs of 4 warps per SM, 32-key
@@ -516,7 +277,7 @@ constexpr int kDqWarps = 4, kDqStages = 2, kDqCtasPerSm = 2;
 cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* k, const void* v,
                                const float* lse, const float* delta, const int32_t* row_cnt,
                                const int32_t* row_cols, int64_t T, int G, int n_sel, float scale, void* dq,
-                               uint16_t* pds, cudaStream_t s) {
+                               uint16_t* prec, uint16_t* dsrec, cudaStream_t s) {
   using S_ = DqShape<kDqWarps, kDqStages, kDqCtasPerSm>;
   auto kern = dq_kernel<kDqWarps, kDqStages, kDqCtasPerSm>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S_::kSmemBytes);
@@ -527,19 +288,7 @@ cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* 
   kern<<<static_cast<unsigned>(grid), S_::kThreads, S_::kSmemBytes, s>>>(
       static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q),
       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), lse, delta, row_cnt, row_cols,
-      n_items, G, n_sel, scale, scale * kLog2e, static_cast<__nv_bfloat16*>(dq), pds);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_backward_dkdv(const void* grad_out, const void* q, const uint16_t* pds, const int64_t* quad_ent,
-                                 const int32_t* wl_cnt, const int4* wl, int p, int64_t n_quads, int64_t T_kv,
-                                 int G, int n_sel, float scale, float* partial, void* dk, void* dv,
-                                 bool f32_out, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kKvSmem);
-  if (e != cudaSuccess) return e;
-  dkdv_kernel<<<static_cast<unsigned>(kKvCtasPerSm * sm_count()), kKvThreads, kKvSmem, s>>>(
-      static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q), pds, quad_ent, wl_cnt + p,
-      wl + static_cast<int64_t>(p) * n_quads, T_kv, G, n_sel, scale, partial, dk, dv, f32_out);
+      n_items, G, n_sel, scale, scale * kLog2e, static_cast<__nv_bfloat16*>(dq), prec, dsrec);
   return cudaGetLastError();
 }
 

@@ -1,0 +1,547 @@
+// dK / dV over 128-key tiles on the tensor cores (tcgen05), all query phases in
+// one launch.
+//
+// Backward equations of the cuDNN-Frontend "Query Sparse Attention (QSA)" page
+// ("Selection and components"), per KV group g, summed over its 12 heads:
+//   dK [key] = scale * sum_t sum_h dS[t, h, key] Q[t, h],   dV [key] = sum_t sum_h P[t, h, key] dO[t, h].
+// A work unit is (tile of 128 keys, group g, tensor dK or dV).  Its queries are
+// the tile's transpose list for the phase: one entry per query row that routes
+// into the tile (its "union": the row's keys inside the tile, a contiguous run
+// of the sorted row), so a query's 12 Q (or dO) rows are gathered once per tile
+// however many of the tile's keys it selected.  Per chunk of 4 unions:
+//   D [128 keys x 256 dims] += A [128 keys x 48] . B [48 x 256 dims]
+// with K row 12 u + h = head h of union u; A holds the BF16 dS (for dK) or P
+// (for dV) records the dQ kernel wrote (24 bytes per routed pair), zero where a
+// union did not select the key; B holds the gathered Q (or dO) rows.  That is 3
+// tcgen05.mma kind::f16 (M 128, N 256, K 16), A K-major without swizzle, B MN-major with the 128-byte
+// swizzle, the accumulator in tensor memory (two 256-column buffers, so the
+// epilogue of one unit overlaps the next unit's MMAs).
+//
+// Warp roles (384 threads): warp 6 schedules (claims units, cuts them into
+// chunks of 4 entries, publishes each chunk's descriptor in a shared-memory ring
+// and prefetches its rows, records and keys into L2); warps 0-5 fill whole
+// chunks, warp w the chunks of stage w of the 6-stage shared-memory ring (zero
+// A, gather B rows with cp.async, store the records into their A rows); warp 7
+// (one thread) issues the MMAs; warps 8-11 (tensor-memory lane quarters 0-3)
+// run the epilogue, thread = key row.  Units are claimed from one counter in phase order (phase 0's units, then
+// phase 1's, ...; inside a phase every dK unit before every dV unit), so the
+// CTAs work on about one phase and one tensor at a time and its Q (or dO) rows
+// stay in L2.  A unit sums its entries in list order; its epilogue waits until
+// the unit of the same (tile, group, tensor) in the previous non-empty phase has
+// stored its FP32 partial (a per-(tile, group, tensor) counter in global
+// memory), adds it, and stores its own partial or the final dK / dV.  The
+// summation order is fixed, whichever CTA ran what: no floating-point atomics,
+// bitwise reproducible.  A wait only ever targets a unit claimed earlier, by a
+// CTA that is running, so the waits cannot form a cycle.  Every wait is
+// bounded; on expiry the kernel sets the status word, stops all roles, waits
+// (bounded) for its MMAs, frees its tensor memory and returns.
+#include "qsa_internal.h"
+#include "qsa_device.cuh"
+
+namespace qsa {
+namespace {
+
+constexpr int kUThreads = 384;
+constexpr int kUWorkers = 6;                        // warps 0-5 fill chunks, warp w every stage-w chunk
+constexpr int kUSchedWarp = 6, kUMmaWarp = 7, kUEpiWarp0 = 8;
+constexpr int kURec = 12;                           // bf16 per (t, g, key) record of P or dS: 12 heads
+constexpr int kUKeys = 128;                         // keys per tile (MMA M)
+constexpr int kUUnions = 4;                         // unions per chunk
+constexpr int kUK = kUUnions * kHeadsPerGroup;      // 48 K rows per chunk
+constexpr int kUBBlk = kUK * 128;                   // one 64-dim column block of B (6 KB)
+constexpr int kUBBytes = 4 * kUBBlk;                // 24 KB
+constexpr int kUASbo = (kUK / 8) * 128;             // A: bytes between 8-key core-matrix rows (768)
+constexpr int kUABytes = kUKeys * kUK * 2;          // 12 KB
+constexpr int kUStage = kUBBytes + kUABytes;        // 36 KB
+constexpr int kUStages = 6;
+constexpr int kURing = 16;                          // chunk descriptors the scheduler may run ahead
+constexpr int kUOffCtl = kUStages * kUStage;
+// control block: stage descriptors, accumulator descriptors, the chunk ring
+// (header int4 + 4 list entries), phase prefix, barriers, tmem slot, abort flag
+constexpr int kUOffDesc = kUOffCtl;                          // kUStages x int4
+constexpr int kUOffAcc = kUOffDesc + kUStages * 16;          // 2 x int4
+constexpr int kUOffRing = kUOffAcc + 2 * 16;                 // kURing x 48 bytes
+constexpr int kUMaxPhases = 64;
+constexpr int kUOffPref = kUOffRing + kURing * 48;           // kUMaxPhases + 1 ints: units before each phase
+constexpr int kUOffBar = (kUOffPref + 4 * (kUMaxPhases + 1) + 7) & ~7;
+constexpr int kUBarFull = kUOffBar, kUBarEmpty = kUBarFull + 8 * kUStages;
+constexpr int kUBarRingFull = kUBarEmpty + 8 * kUStages, kUBarRingEmpty = kUBarRingFull + 8 * kURing;
+constexpr int kUBarAccFull = kUBarRingEmpty + 8 * kURing, kUBarAccEmpty = kUBarAccFull + 16;
+constexpr int kUBarDrain = kUBarAccEmpty + 16;
+constexpr int kUOffTmem = kUBarDrain + 8, kUOffAbort = kUOffTmem + 4;
+constexpr int kUSmem = kUOffAbort + 4 + 1024;      // + alignment slack
+static_assert(kUStage % 1024 == 0, "stage alignment (128-byte swizzle atoms)");
+static_assert(kUSmem <= 232448, "shared memory per block");
+// One worker per stage: chunk c goes to warp c % kUStages, so every wait on a
+// stage's barriers comes from one warp, in order, at most one phase ahead of
+// the barrier (a parity wait two phases early would pass at once).  The
+// descriptor ring is at least as deep as the worker count for the same reason.
+static_assert(kUWorkers == kUStages && kURing >= kUWorkers, "one worker per stage");
+static_assert(kUThreads == 32 * (kUEpiWarp0 + 4) && kUEpiWarp0 % 4 == 0 && kUSchedWarp >= kUWorkers &&
+                  kUMmaWarp > kUSchedWarp && kUMmaWarp < kUEpiWarp0,
+              "warp roles (epilogue warps cover tensor-memory lane quarters 0-3 in order)");
+constexpr uint32_t kUSpin = 1u << 22;
+constexpr int kChFirst = 1, kChLast = 2;
+// kind::f16: FP32 accumulate, BF16 A (K-major) and B (MN-major), N = 256, M = 128.
+constexpr uint32_t kUIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
+
+// Bounded wait that also gives up once another role has aborted.
+__device__ __forceinline__ bool u_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  for (uint32_t it = 0; it < kUSpin; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 255) == 255 && *abort_flag) return false;
+  }
+  *abort_flag = 1;
+  return false;
+}
+// A: K-major, no swizzle; core matrices of 8 rows x 16 bytes, 128 bytes apart
+// along K (LBO) and kUASbo apart along M (SBO).
+__device__ __forceinline__ uint64_t u_desc_a(uint32_t addr) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3fff) | (static_cast<uint64_t>(128 >> 4) << 16) |
+         (static_cast<uint64_t>(kUASbo >> 4) << 32) | (static_cast<uint64_t>(1) << 46);
+}
+// B: MN-major, 128-byte swizzle; 64-dim column blocks kUBBlk apart (LBO), 8-row
+// groups 1024 bytes apart (SBO).
+__device__ __forceinline__ uint64_t u_desc_b(uint32_t addr) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3fff) | (static_cast<uint64_t>(kUBBlk >> 4) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) | (static_cast<uint64_t>(2) << 61);
+}
+__device__ __forceinline__ void u_mma(uint32_t d, uint64_t a, uint64_t b, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d),
+      "l"(a), "l"(b), "r"(kUIdesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void u_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void u_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,"
+      "%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__global__ void __launch_bounds__(kUThreads, 1)
+dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ q,
+                  const uint16_t* __restrict__ prec, const uint16_t* __restrict__ dsrec,
+                  const int32_t* __restrict__ row_cols,
+                  const int64_t* __restrict__ ent, const int32_t* __restrict__ wl_cnt, const int4* __restrict__ wl,
+                  int* __restrict__ claim_ctr, int* __restrict__ done, int P, int64_t n_tiles, int64_t T_kv, int G,
+                  int n_sel, float scale,
+                  float* __restrict__ partial, void* __restrict__ dk_out, void* __restrict__ dv_out, bool f32_out,
+                  int* __restrict__ status) {
+  extern __shared__ uint8_t u_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(u_smem_raw) + 1023) & ~uintptr_t{1023});
+  const uint32_t sbase = smem_u32(smem);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int H = G * kHeadsPerGroup;
+  const int units_per_item = 2 * G;
+  volatile int* pref = reinterpret_cast<volatile int*>(smem + kUOffPref);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kUOffAbort);
+  int4* desc = reinterpret_cast<int4*>(smem + kUOffDesc);
+  int4* acc_desc = reinterpret_cast<int4*>(smem + kUOffAcc);
+  uint8_t* ring = smem + kUOffRing;  // chunk c: header int4 at 48 (c % kURing), entries after it
+
+  if (tid == 0) {
+    for (int s = 0; s < kUStages; ++s) {
+      mbar_init(sbase + kUBarFull + 8 * s, 1);   // the worker warp that filled the stage
+      mbar_init(sbase + kUBarEmpty + 8 * s, 1);  // the MMAs that read it
+    }
+    for (int r = 0; r < kURing; ++r) {
+      mbar_init(sbase + kUBarRingFull + 8 * r, 1);   // the scheduler wrote the descriptor
+      mbar_init(sbase + kUBarRingEmpty + 8 * r, 1);  // its worker read it
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(sbase + kUBarAccFull + 8 * b, 2);   // MMA completion + the issuing thread's descriptor arrival
+      mbar_init(sbase + kUBarAccEmpty + 8 * b, 4);  // one arrival per epilogue warp
+    }
+    mbar_init(sbase + kUBarDrain, 1);
+    *abort_flag = 0;
+    int acc = 0;
+    for (int p = 0; p < P; ++p) {
+      pref[p] = acc;
+      acc += __ldg(wl_cnt + p) * units_per_item;
+    }
+    pref[P] = acc;
+    mbar_fence_init();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(sbase + kUOffTmem),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kUOffTmem);
+  const int n_units = pref[P];
+
+  if (warp < kUWorkers) {
+    // ------------------------------------------------------------ workers
+    // Warp w fills chunks w, w + 6, w + 12, ... on its own: it takes the chunk's
+    // descriptor from the scheduler's ring, waits for the chunk's stage to be
+    // free, zeroes A, gathers the 48 Q (or dO) rows of the chunk's 4 unions into
+    // B with cp.async, stores each union's records into the A rows of their keys,
+    // waits for its copies and marks the stage full.  Up to kUStages chunks are
+    // in flight at once, one per warp, with no barrier between warps.
+    for (int c = warp;; c += kUWorkers) {
+      const int rs = c % kURing;
+      bool got = true;
+      if (lane == 0) got = u_wait(sbase + kUBarRingFull + 8 * rs, (c / kURing) & 1, abort_flag);
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      __syncwarp();  // every lane reads the descriptor after lane 0 saw it published
+      const volatile int* hv = reinterpret_cast<const volatile int*>(ring + 48 * rs);
+      const int4 hd = make_int4(hv[0], hv[1], hv[2], hv[3]);
+      int64_t e[kUUnions];
+#pragma unroll
+      for (int u = 0; u < kUUnions; ++u) e[u] = reinterpret_cast<const volatile int64_t*>(ring + 48 * rs + 16)[u];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sbase + kUBarRingEmpty + 8 * rs);
+      const int s = c % kUStages;
+      const bool end = hd.x < 0;
+      if (end && hd.y == 0) break;  // an end marker for a warp whose chunk the MMA never reaches
+      // stage s is free once the MMAs of chunk c - kUStages completed
+      if (c >= kUStages) {
+        if (lane == 0) got = u_wait(sbase + kUBarEmpty + 8 * s, ((c / kUStages) - 1) & 1, abort_flag);
+        if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      }
+      const uint32_t st = sbase + s * kUStage;
+      if (end) {  // the first chunk past the last unit: end marker for the MMA warp
+        if (lane == 0) {
+          desc[s] = make_int4(0, -1, 0, 0);
+          mbar_arrive(sbase + kUBarFull + 8 * s);
+        }
+        break;
+      }
+      const int n = hd.z & 255, r = hd.z >> 10, g = r >> 1, tensor = r & 1, tile = hd.w;
+      // zero A (12 KB): unselected (union, key) slots must read as 0
+      {
+        uint4* a = reinterpret_cast<uint4*>(smem + s * kUStage + kUBBytes);
+#pragma unroll 4
+        for (int i = lane; i < kUABytes / 16; i += 32) a[i] = make_uint4(0, 0, 0, 0);
+      }
+      // B: the 12 head rows of each union (zero-filled for missing unions)
+      {
+        const __nv_bfloat16* base = (tensor ? dout : q) + (g * kHeadsPerGroup * kHeadDim + lane * 8);
+        const uint32_t dst = st + (lane >> 3) * kUBBlk;
+        const int unit = lane & 7;
+#pragma unroll
+        for (int u = 0; u < kUUnions; ++u) {
+          const bool mine = u < n;
+          const __nv_bfloat16* src = base + (mine ? (e[u] >> 32) : 0) * H * kHeadDim;
+#pragma unroll
+          for (int h = 0; h < kHeadsPerGroup; ++h) {
+            const int kr = u * kHeadsPerGroup + h;
+            cp_async16(dst + kr * 128 + ((unit ^ (kr & 7)) << 4), src + h * kHeadDim, mine);
+          }
+        }
+      }
+      cp_async_commit();
+      // A: record j of union u goes to row (key - tile base), K columns 12 u .. 12 u + 11
+      // (24-byte records of 12 heads: dK takes dS, dV takes P)
+      const uint16_t* recs = tensor ? prec : dsrec;
+      const int key0 = tile * kUKeys;
+      int32_t key[kUUnions];
+      uint2 val[kUUnions][3];
+#pragma unroll
+      for (int u = 0; u < kUUnions; ++u) {
+        const int64_t t = e[u] >> 32;
+        const int i0 = static_cast<int>((e[u] >> 8) & 0x3fff), cnt = static_cast<int>(e[u] & 0x7f) + 1;
+        const bool ok_j = u < n && lane < cnt;
+        const uint2* rec = reinterpret_cast<const uint2*>(recs + ((t * G + g) * n_sel + i0) * kURec);
+        key[u] = ok_j ? __ldg(row_cols + t * n_sel + i0 + lane) : -1;
+#pragma unroll
+        for (int hq = 0; hq < 3; ++hq) val[u][hq] = ok_j ? __ldg(rec + lane * 3 + hq) : make_uint2(0, 0);
+      }
+      __syncwarp();  // the zeroing above before the record stores below
+      uint8_t* abase = smem + s * kUStage + kUBBytes;
+      auto put = [&](int u, int32_t k, const uint2 (&v)[3]) {
+        const int m = k - key0;
+        if (k < 0 || static_cast<unsigned>(m) >= static_cast<unsigned>(kUKeys)) return;  // never for a well-formed list
+        uint8_t* row = abase + (m >> 3) * kUASbo + (m & 7) * 16;
+#pragma unroll
+        for (int hq = 0; hq < 3; ++hq) {
+          const int kk = u * kHeadsPerGroup + 4 * hq;
+          *reinterpret_cast<uint2*>(row + (kk >> 3) * 128 + (kk & 7) * 2) = v[hq];
+        }
+      };
+#pragma unroll
+      for (int u = 0; u < kUUnions; ++u) put(u, key[u], val[u]);
+      // unions with more than 32 keys in the tile (rare for sparse routes)
+#pragma unroll
+      for (int u = 0; u < kUUnions; ++u) {
+        const int64_t t = e[u] >> 32;
+        const int i0 = static_cast<int>((e[u] >> 8) & 0x3fff), cnt = static_cast<int>(e[u] & 0x7f) + 1;
+        if (u >= n || cnt <= 32) continue;
+        const uint2* rec = reinterpret_cast<const uint2*>(recs + ((t * G + g) * n_sel + i0) * kURec);
+        for (int j = lane + 32; j < cnt; j += 32) {
+          const uint2 v[3] = {__ldg(rec + j * 3), __ldg(rec + j * 3 + 1), __ldg(rec + j * 3 + 2)};
+          put(u, __ldg(row_cols + t * n_sel + i0 + j), v);
+        }
+      }
+      if (lane == 0) desc[s] = make_int4(hd.x, n, (hd.z >> 8) & 3, r);
+      // the stage is complete once this warp's copies landed: make it visible to
+      // the tensor cores, mark it full
+      cp_async_wait<0>();
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sbase + kUBarFull + 8 * s);
+    }
+  } else if (warp == kUMmaWarp) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      int useq = 0;
+      bool ok = true;
+      for (int c = 0;; ++c) {
+        const int s = c % kUStages;
+        if (!u_wait(sbase + kUBarFull + 8 * s, (c / kUStages) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const int4 d = desc[s];
+        if (d.y < 0) break;
+        const int buf = useq & 1;
+        if ((d.z & kChFirst) && useq >= 2 &&
+            !u_wait(sbase + kUBarAccEmpty + 8 * buf, ((useq >> 1) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+        const uint32_t st = sbase + s * kUStage;
+        const int nks = (d.y * kHeadsPerGroup + 15) / 16;
+        for (int ks = 0; ks < nks; ++ks)
+          u_mma(tmem + buf * 256, u_desc_a(st + kUBBytes + ks * 256), u_desc_b(st + ks * 2048),
+                ((d.z & kChFirst) && ks == 0) ? 0u : 1u);
+        u_commit(sbase + kUBarEmpty + 8 * s);
+        if (d.z & kChLast) {
+          acc_desc[buf] = make_int4(d.x, d.w, 0, 0);
+          u_commit(sbase + kUBarAccFull + 8 * buf);
+          mbar_arrive(sbase + kUBarAccFull + 8 * buf);
+          ++useq;
+        }
+      }
+      if (ok) {  // end marker for the epilogue
+        const int buf = useq & 1;
+        if (useq < 2 || u_wait(sbase + kUBarAccEmpty + 8 * buf, ((useq >> 1) - 1) & 1, abort_flag)) {
+          acc_desc[buf] = make_int4(-1, 0, 0, 0);
+          mbar_arrive(sbase + kUBarAccFull + 8 * buf);
+          mbar_arrive(sbase + kUBarAccFull + 8 * buf);
+        }
+      }
+      // all issued MMAs complete before the tensor memory is released
+      u_commit(sbase + kUBarDrain);
+      for (uint32_t it = 0; it < kUSpin && !mbar_try(sbase + kUBarDrain, 0); ++it) {
+      }
+    }
+    __syncwarp();
+  } else if (warp >= kUEpiWarp0) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp - kUEpiWarp0;      // tensor-memory lanes 32 quarter .. + 31
+    const int m = quarter * 32 + lane;          // key row within the tile
+    const bool leader = quarter == 0 && lane == 0;
+    for (int useq = 0;; ++useq) {
+      const int buf = useq & 1;
+      if (!u_wait(sbase + kUBarAccFull + 8 * buf, (useq >> 1) & 1, abort_flag)) break;
+      const int idx = acc_desc[buf].x, r = acc_desc[buf].y;
+      if (idx < 0) break;
+      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+      const int4 it = __ldg(wl + idx);
+      const int g = r >> 1, tensor = r & 1;
+      const int ord = it.w >> 2;                 // earlier non-empty phases of this tile
+      const bool last = it.w & 2;
+      const int64_t key = static_cast<int64_t>(it.x) * kUKeys + m;
+      const int64_t slot = (static_cast<int64_t>(it.x) * G + g) * 2 + tensor;
+      float* part = partial + slot * (kUKeys * kHeadDim) + static_cast<int64_t>(m) * kHeadDim;
+      const float f = tensor ? 1.f : scale;
+      if (ord > 0) {
+        // the previous phase's partial of this (tile, group, tensor) must be stored
+        bool fail = false;
+        if (leader) {
+          uint32_t it2 = 0;
+          for (;; ++it2) {
+            int v;
+            asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(done + slot) : "memory");
+            if (v >= ord) break;
+            if (it2 >= kUSpin || ((it2 & 255) == 255 && *abort_flag)) {
+              *abort_flag = 1;
+              fail = true;
+              break;
+            }
+            __nanosleep(64);
+          }
+        }
+        if (bar_or(3, 128, fail)) break;
+      }
+      for (int j = 0; j < kHeadDim / 32; ++j) {
+        float v[32];
+        u_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * 256 + j * 32, v);
+        if (ord > 0) {
+          const float4* pr = reinterpret_cast<const float4*>(part + j * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 x = __ldcg(pr + i);
+            v[4 * i] += x.x;
+            v[4 * i + 1] += x.y;
+            v[4 * i + 2] += x.z;
+            v[4 * i + 3] += x.w;
+          }
+        }
+        if (last) {
+          if (key < T_kv) {
+            const int64_t o = (key * G + g) * kHeadDim + j * 32;
+            if (f32_out) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(tensor ? dv_out : dk_out) + o);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                dst[i] = make_float4(v[4 * i] * f, v[4 * i + 1] * f, v[4 * i + 2] * f, v[4 * i + 3] * f);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(tensor ? dv_out : dk_out) + o);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(pack_bf16(v[8 * i] * f, v[8 * i + 1] * f), pack_bf16(v[8 * i + 2] * f, v[8 * i + 3] * f),
+                                    pack_bf16(v[8 * i + 4] * f, v[8 * i + 5] * f),
+                                    pack_bf16(v[8 * i + 6] * f, v[8 * i + 7] * f));
+            }
+          }
+        } else {
+          float4* pw = reinterpret_cast<float4*>(part + j * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) __stcg(pw + i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+        }
+      }
+      asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sbase + kUBarAccEmpty + 8 * buf);
+      if (!last) {
+        // publish the partial: every epilogue thread's stores, then the counter
+        bar_sync(3, 128);
+        if (leader) {
+          __threadfence();
+          asm volatile("st.release.gpu.global.b32 [%0], %1;\n" ::"l"(done + slot), "r"(ord + 1) : "memory");
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ scheduler
+    // Claims units (one ahead) in phase order, cuts them into chunks of up to 4
+    // entries, writes each chunk's descriptor and entries into the ring, and
+    // prefetches into L2 what the chunk's worker will read: the unions' Q (or
+    // dO) rows, record runs and key runs.
+    int claim_p = 0;
+    // unit U -> its phase p, and inside the phase tensor-major order (every dK
+    // unit, then every dV unit, so one tensor's rows are live in L2 at a time):
+    // {work item index, r = 2 g + tensor}; item.x < 0 when the list is exhausted
+    auto claim = [&](int4& item, int& idx, int& r) {
+      int U = 0;
+      if (lane == 0) U = atomicAdd(claim_ctr, 1);
+      U = __shfl_sync(0xffffffffu, U, 0);
+      if (U >= n_units) {
+        item = make_int4(-1, 0, 0, 0);
+        return;
+      }
+      while (pref[claim_p + 1] <= U) ++claim_p;  // claims only grow
+      const int local = U - pref[claim_p];
+      const int per_tensor = (pref[claim_p + 1] - pref[claim_p]) >> 1;  // items x G
+      const int tensor = local >= per_tensor ? 1 : 0;
+      const int rem = local - tensor * per_tensor;
+      idx = static_cast<int>(claim_p * n_tiles) + rem / G;
+      r = 2 * (rem % G) + tensor;
+      item = __ldg(wl + idx);
+    };
+    auto prefetch_l2 = [&](const void* p, int64_t bytes) {  // 16-byte aligned window around [p, p + bytes)
+      const uintptr_t a0 = reinterpret_cast<uintptr_t>(p) & ~uintptr_t{15};
+      const uintptr_t a1 = (reinterpret_cast<uintptr_t>(p) + bytes + 15) & ~uintptr_t{15};
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(a0), "r"(static_cast<uint32_t>(a1 - a0))
+                   : "memory");
+    };
+    int c = 0;
+    bool ok = true;
+    int4 cur, nxt;
+    int cur_idx = 0, cur_r = 0, nxt_idx = 0, nxt_r = 0;
+    claim(cur, cur_idx, cur_r);
+    if (cur.x >= 0) claim(nxt, nxt_idx, nxt_r);
+    while (ok && cur.x >= 0) {
+      const int g = cur_r >> 1, tensor = cur_r & 1;
+      for (int w0 = cur.y; ok && w0 < cur.z; w0 += 32) {
+        // a window of up to 32 entries: lane i holds entry w0 + i
+        const bool have = w0 + lane < cur.z;
+        const int64_t el = have ? __ldg(ent + w0 + lane) : 0;
+        if (have) {
+          const int64_t t = el >> 32;
+          const int i0 = static_cast<int>((el >> 8) & 0x3fff), cnt = static_cast<int>(el & 0x7f) + 1;
+          prefetch_l2((tensor ? dout : q) + (t * H + g * kHeadsPerGroup) * kHeadDim, kHeadsPerGroup * kHeadDim * 2);
+          prefetch_l2((tensor ? prec : dsrec) + ((t * G + g) * n_sel + i0) * kURec, cnt * kURec * 2);
+          prefetch_l2(row_cols + t * n_sel + i0, cnt * 4);
+        }
+        const int w1 = min(cur.z, w0 + 32);
+        for (int p = w0; p < w1; p += kUUnions) {
+          const int n = min(kUUnions, cur.z - p);
+          const int rs = c % kURing;
+          bool got = true;
+          if (c >= kURing && lane == 0) got = u_wait(sbase + kUBarRingEmpty + 8 * rs, ((c / kURing) - 1) & 1, abort_flag);
+          if (!__shfl_sync(0xffffffffu, got, 0)) {
+            ok = false;
+            break;
+          }
+          const int64_t eu = __shfl_sync(0xffffffffu, el, (p - w0) + (lane & 3));
+          if (lane < kUUnions) reinterpret_cast<int64_t*>(ring + 48 * rs + 16)[lane] = lane < n ? eu : 0;
+          const int flags = (p == cur.y ? kChFirst : 0) | (p + n >= cur.z ? kChLast : 0);
+          if (lane == 0) *reinterpret_cast<int4*>(ring + 48 * rs) = make_int4(cur_idx, p, n | (flags << 8) | (cur_r << 10), cur.x);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sbase + kUBarRingFull + 8 * rs);
+          ++c;
+        }
+      }
+      cur = nxt;
+      cur_idx = nxt_idx;
+      cur_r = nxt_r;
+      if (cur.x >= 0) claim(nxt, nxt_idx, nxt_r);
+    }
+    // end markers: chunk c (the first past the list) ends the MMA loop; each of
+    // the other workers gets one that only ends its own loop
+    for (int k = 0; ok && k < kUWorkers; ++k, ++c) {
+      const int rs = c % kURing;
+      bool got = true;
+      if (c >= kURing && lane == 0) got = u_wait(sbase + kUBarRingEmpty + 8 * rs, ((c / kURing) - 1) & 1, abort_flag);
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      if (lane == 0) {
+        *reinterpret_cast<int4*>(ring + 48 * rs) = make_int4(-1, k == 0 ? 1 : 0, 0, 0);
+        mbar_arrive(sbase + kUBarRingFull + 8 * rs);
+      }
+    }
+  }
+
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  if (*abort_flag && tid == 0 && status) atomicExch(status, 3);
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(512));
+}
+
+}  // namespace
+
+cudaError_t launch_backward_dkdv_union(const void* grad_out, const void* q, const uint16_t* prec, const uint16_t* dsrec,
+                                       const int32_t* row_cols, const int64_t* tile_ent, const int32_t* wl_cnt,
+                                       const int4* wl, int* claim_ctr, int* done, int P, int64_t n_tiles,
+                                       int64_t T_kv, int G, int n_sel, float scale, float* partial, void* dk, void* dv,
+                                       bool f32_out, int* status, cudaStream_t s) {
+  if (P < 1 || P > kUMaxPhases) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(dkdv_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUSmem);
+  if (e != cudaSuccess) return e;
+  dkdv_union_kernel<<<static_cast<unsigned>(sm_count()), kUThreads, kUSmem, s>>>(
+      static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q), prec, dsrec, row_cols, tile_ent,
+      wl_cnt, wl, claim_ctr, done, P, n_tiles, T_kv, G, n_sel, scale, partial, dk, dv, f32_out, status);
+  return cudaGetLastError();
+}
+
+}  // namespace qsa

@@ -7,13 +7,14 @@
 namespace qsa {
 
 // Route preprocessing (qsa_routes.cu).
-// Per-row ascending, de-duplicated valid route IDs; optionally counts, per key
-// quad, the rows that meet it (quad_cnt must be zeroed by the caller).
+// Per-row ascending, de-duplicated valid route IDs; optionally counts, per
+// bucket of 2^cnt_shift consecutive keys (2: quads, 7: 128-key tiles), the rows
+// that meet it (bucket_cnt must be zeroed by the caller).
 // `status` (nullable) is zeroed by this kernel, the first of every call.  With
 // `delta` non-null it also writes delta[t, h] = sum_d dO[t,h,d] * out[t,h,d]
 // (FP32 from the BF16 tensors, [T, H]).
 cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel,
-                              int32_t* row_cnt, int32_t* row_cols, int32_t* quad_cnt,
+                              int32_t* row_cnt, int32_t* row_cols, int32_t* bucket_cnt, int cnt_shift,
                               int* status, const void* dout, const void* out, float* delta, int H,
                               cudaStream_t s);
 // quad_cnt -> quad_ptr (exclusive scan, n_quads+1 entries) and quad_fill (copy
@@ -27,32 +28,46 @@ cudaError_t launch_quad_fill(const int32_t* row_cnt, const int32_t* row_cols, in
 // [p*C, (p+1)*C) starts in it: phase_ptr[b*(P+1) + p].
 cudaError_t launch_quad_sort(const int32_t* quad_ptr, int64_t n_quads, int64_t* quad_ent, int P, int C,
                              int32_t* phase_ptr, cudaStream_t s);
-// Per-phase work lists of non-empty (quad, entry range) items (wl_cnt zeroed by
-// the caller); zeroes dK/dV (BF16, or FP32 when f32_out) of quads that no query
-// routes to.
-cudaError_t launch_quad_worklist(const int32_t* quad_ptr, const int32_t* phase_ptr, int64_t n_quads, int64_t T_kv,
+// The key->query transpose over 128-key tiles: one entry per (row, tile) pair,
+// (t << 32) | (i0 << 8) | (n - 1) with row_cols[t][i0, i0 + n) the row's keys in
+// the tile.  Count rows per tile (tile_cnt zeroed by the caller), fill
+// (unordered; tile_fill holds the scanned offsets), then sort each tile's list
+// by query and record its phase starts.
+cudaError_t launch_tile_count(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel,
+                              int64_t n_tiles, int32_t* tile_cnt, cudaStream_t s);
+cudaError_t launch_tile_fill(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel, int64_t n_tiles,
+                             int32_t* tile_fill, int64_t* tile_ent, cudaStream_t s);
+cudaError_t launch_tile_sort(const int32_t* tile_ptr, int64_t n_tiles, int64_t* tile_ent, int P, int C,
+                             int32_t* phase_ptr, cudaStream_t s);
+// Per-phase work lists of non-empty (tile, entry range) items (wl_cnt zeroed by
+// the caller); zeroes dK/dV of tiles that no query routes to.
+cudaError_t launch_tile_worklist(const int32_t* tile_ptr, const int32_t* phase_ptr, int64_t n_tiles, int64_t T_kv,
                                  int G, int P, int32_t* wl_cnt, int4* wl, void* dk, void* dv, bool f32_out,
                                  cudaStream_t s);
 
-// Attention kernels (qsa_forward.cu, qsa_backward.cu).
+// Attention kernels (qsa_forward.cu, qsa_backward.cu, qsa_dkdv_union.cu).
 cudaError_t launch_forward(const void* q, const void* k, const void* v, const int32_t* row_cnt,
                            const int32_t* row_cols, int64_t T, int G, int n_sel, float scale,
                            void* out, float* lse, int* status, cudaStream_t s);
 // dQ per query; also writes the BF16 probabilities / score gradients of every
-// routed pair, pds [T, G, n_sel, 24].
+// routed pair, as two record arrays prec (P) and dsrec (dS), each [T, G, n_sel, 12].
 cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* k, const void* v,
                                const float* lse, const float* delta, const int32_t* row_cnt,
                                const int32_t* row_cols, int64_t T, int G, int n_sel, float scale,
-                               void* dq, uint16_t* pds, cudaStream_t s);
+                               void* dq, uint16_t* prec, uint16_t* dsrec, cudaStream_t s);
 // SM count of the current device (cached).
 int sm_count();
-// dK/dV over the work list of query phase p: accumulates each item's entries
-// onto its quad, reading / writing FP32 partials between phases; the final
-// dK/dV are BF16, or FP32 when f32_out.
-cudaError_t launch_backward_dkdv(const void* grad_out, const void* q, const uint16_t* pds, const int64_t* quad_ent,
-                                 const int32_t* wl_cnt, const int4* wl, int p, int64_t n_quads, int64_t T_kv,
-                                 int G, int n_sel, float scale, float* partial, void* dk, void* dv,
-                                 bool f32_out, cudaStream_t s);
+// dK/dV over 128-key tiles on the tensor cores, all P query phases in one
+// launch: units (tile, group, tensor) of the per-phase work lists claimed from
+// *claim_ctr in phase order; the FP32 partial of a (tile, group, tensor) passes
+// from phase to phase through `partial`, ordered by its counter in `done`
+// (n_tiles * 2G ints; claim_ctr and done zeroed by the caller); final dK/dV BF16,
+// or FP32 when f32_out.  Sets *status = 3 if a bounded wait expired.  P <= 64.
+cudaError_t launch_backward_dkdv_union(const void* grad_out, const void* q, const uint16_t* prec, const uint16_t* dsrec,
+                                       const int32_t* row_cols, const int64_t* tile_ent, const int32_t* wl_cnt,
+                                       const int4* wl, int* claim_ctr, int* done, int P, int64_t n_tiles,
+                                       int64_t T_kv, int G, int n_sel, float scale, float* partial, void* dk, void* dv,
+                                       bool f32_out, int* status, cudaStream_t s);
 
 // Bitmap selection -> route IDs (qsa_bitmap.cu); zeroes *max_cnt first when given.
 cudaError_t launch_bitmap_routes(const uint8_t* sel, const int32_t* lo, const int32_t* hi, const int32_t* blk_base,

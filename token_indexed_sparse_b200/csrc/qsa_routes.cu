@@ -145,11 +145,12 @@ __device__ __forceinline__ void warp_sort(int32_t (&v)[NPL], int lane) {
 }
 
 // One warp per query row (rows of up to 32*NPL route slots): filter, sort in
-// registers, de-duplicate, compact; optional key-quad counts and delta.
+// registers, de-duplicate, compact; optional per-bucket row counts (a bucket is
+// 2^cnt_shift consecutive keys: a quad or a 128-key tile) and delta.
 template <int NPL>
 __global__ void __launch_bounds__(256) route_rows_warp_kernel(
     const int32_t* __restrict__ routes, int64_t T, int32_t T_kv, int n_sel, int32_t* __restrict__ row_cnt,
-    int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt, int* __restrict__ status,
+    int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt, int cnt_shift, int* __restrict__ status,
     const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out, float* __restrict__ delta,
     int H) {
   const int lane = threadIdx.x & 31;
@@ -179,7 +180,8 @@ __global__ void __launch_bounds__(256) route_rows_warp_kernel(
     const int32_t x = v[r];
     if (x != INT_MAX && x != p) {
       ++mine;
-      if (quad_cnt != nullptr && (p == INT_MIN || (p >> 2) != (x >> 2))) atomicAdd(quad_cnt + (x >> 2), 1);
+      if (quad_cnt != nullptr && (p == INT_MIN || (p >> cnt_shift) != (x >> cnt_shift)))
+        atomicAdd(quad_cnt + (x >> cnt_shift), 1);
     }
   }
   int incl = mine;
@@ -215,7 +217,7 @@ __global__ void __launch_bounds__(256) route_rows_warp_kernel(
 // One block per query row: filter invalid IDs, sort, de-duplicate, compact.
 __global__ void __launch_bounds__(kRowThreads) route_rows_kernel(
     const int32_t* __restrict__ routes, int32_t T_kv, int n_sel, int n2,
-    int32_t* __restrict__ row_cnt, int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt,
+    int32_t* __restrict__ row_cnt, int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt, int cnt_shift,
     int* __restrict__ status, const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out,
     float* __restrict__ delta, int H) {
   extern __shared__ int32_t sv[];  // n2 values, then 32 ints of scan scratch
@@ -242,7 +244,8 @@ __global__ void __launch_bounds__(kRowThreads) route_rows_kernel(
     const int32_t x = sv[i];
     if (x != INT_MAX && (i == 0 || sv[i - 1] != x)) {
       ++mine;
-      if (quad_cnt != nullptr && (i == 0 || (sv[i - 1] >> 2) != (x >> 2))) atomicAdd(quad_cnt + (x >> 2), 1);
+      if (quad_cnt != nullptr && (i == 0 || (sv[i - 1] >> cnt_shift) != (x >> cnt_shift)))
+        atomicAdd(quad_cnt + (x >> cnt_shift), 1);
     }
   }
   int total;
@@ -359,35 +362,168 @@ __global__ void __launch_bounds__(kSortThreads) quad_sort_kernel(const int32_t* 
   }
 }
 
-// Thread per quad: append the quad's non-empty phase ranges to the per-phase
-// work lists, wl[p][*] = (quad, first entry, end entry, flags), flags bit 0:
-// no entries before this range, bit 1: no entries after it.  Quads that no query
-// routes to get their dK/dV rows zeroed here.  The order inside a work list
-// does not matter: each item accumulates its own quad, in list order.
-__global__ void __launch_bounds__(256) quad_worklist_kernel(
-    const int32_t* __restrict__ ptr, const int32_t* __restrict__ phase_ptr, int64_t n_quads, int64_t T_kv, int G,
-    int P, int32_t* __restrict__ wl_cnt, int4* __restrict__ wl, uint8_t* __restrict__ dk,
-    uint8_t* __restrict__ dv, int out_bytes) {
-  const int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (b >= n_quads) return;
-  const int q0 = ptr[b], q1 = ptr[b + 1];
-  if (q0 == q1) {
-    const int64_t k_end = min(T_kv, 4 * b + 4);
-    const int64_t row = static_cast<int64_t>(G) * kHeadDim * out_bytes;  // bytes per key
-    for (int64_t key = 4 * b; key < k_end; ++key) {
-      uint4* rk = reinterpret_cast<uint4*>(dk + key * row);
-      uint4* rv = reinterpret_cast<uint4*>(dv + key * row);
-      for (int64_t i = 0; i < row / 16; ++i) rk[i] = rv[i] = make_uint4(0, 0, 0, 0);
+// ---- key->query transpose at the granularity of 128-key tiles ----
+// Entry of a (query row, tile) pair, the "union" of the row's keys in the tile:
+// (t << 32) | (i0 << 8) | (n - 1), where row_cols[t][i0, i0 + n) are the row's
+// keys inside the tile (ascending, so one contiguous run of the sorted row).
+constexpr int kTileShift = 7;
+
+// Rows are taken rows_per_warp per warp (8 warps per block).  With at most
+// kTileBins tiles the block first gathers its per-tile counts in shared memory
+// and touches each global counter once, so rows that meet the same tiles do not
+// contend on one global address per row.
+constexpr int kTileBins = 8192;
+
+// Rows per warp: 8 for rows of up to 1024 slots, else 2 (long rows already give
+// a warp enough work, and more blocks keep more loads in flight).
+inline int tile_rows_per_warp(int n_sel) { return n_sel <= 1024 ? 8 : 2; }
+
+// Calls f(t, cols, cnt, tile, i) for every i where row t's sorted keys enter a
+// new tile.  A warp reads its row 32 keys at a time, the previous key of each
+// lane coming from its neighbour.
+template <typename F>
+__device__ __forceinline__ void for_tile_runs(const int32_t* __restrict__ row_cnt, const int32_t* __restrict__ row_cols,
+                                              int64_t T, int n_sel, int rows_per_warp, F f) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * 8 + warp) * rows_per_warp;
+  for (int r = 0; r < rows_per_warp; ++r) {
+    const int64_t t = t0 + r;
+    if (t >= T) return;
+    const int cnt = row_cnt[t];
+    const int32_t* cols = row_cols + t * n_sel;
+    int32_t carry = -1;  // tile of the last key of the previous 32 (none: -1)
+    for (int base = 0; base < cnt; base += 32) {
+      const int i = base + lane;
+      const int32_t tl = i < cnt ? (cols[i] >> kTileShift) : INT_MAX;
+      int32_t prev = __shfl_up_sync(0xffffffffu, tl, 1);
+      if (lane == 0) prev = carry;
+      carry = __shfl_sync(0xffffffffu, tl, 31);
+      if (i < cnt && tl != prev) f(t, cols, cnt, tl, i);
     }
+  }
+}
+
+// Rows per 128-key tile (tile_cnt zeroed by the caller).
+__global__ void __launch_bounds__(256) tile_count_kernel(const int32_t* __restrict__ row_cnt,
+                                                         const int32_t* __restrict__ row_cols, int64_t T, int n_sel,
+                                                         int rows_per_warp, int64_t n_tiles,
+                                                         int32_t* __restrict__ tile_cnt) {
+  extern __shared__ int32_t hist[];
+  const bool local = n_tiles <= kTileBins;
+  if (local) {
+    for (int b = threadIdx.x; b < n_tiles; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+  }
+  for_tile_runs(row_cnt, row_cols, T, n_sel, rows_per_warp, [&](int64_t, const int32_t*, int, int32_t tl, int) {
+    atomicAdd(local ? hist + tl : tile_cnt + tl, 1);
+  });
+  if (!local) return;
+  __syncthreads();
+  for (int b = threadIdx.x; b < n_tiles; b += blockDim.x)
+    if (hist[b]) atomicAdd(tile_cnt + b, hist[b]);
+}
+
+// One entry per (row, tile) run: (t << 32) | (i0 << 8) | (n - 1), at a slot
+// reserved from the tile's fill cursor (list order is fixed later by the sort).
+__global__ void __launch_bounds__(256) tile_fill_kernel(const int32_t* __restrict__ row_cnt,
+                                                        const int32_t* __restrict__ row_cols, int64_t T,
+                                                        int n_sel, int rows_per_warp, int64_t n_tiles,
+                                                        int32_t* __restrict__ fill, int64_t* __restrict__ ent) {
+  extern __shared__ int32_t tsh[];  // [n_tiles] counts / cursors, [n_tiles] reserved bases
+  const bool local = n_tiles <= kTileBins;
+  int32_t* cnt = tsh;
+  int32_t* base = tsh + (local ? n_tiles : 0);
+  if (local) {
+    for (int b = threadIdx.x; b < n_tiles; b += blockDim.x) cnt[b] = 0;
+    __syncthreads();
+    for_tile_runs(row_cnt, row_cols, T, n_sel, rows_per_warp,
+                  [&](int64_t, const int32_t*, int, int32_t tl, int) { atomicAdd(cnt + tl, 1); });
+    __syncthreads();
+    for (int b = threadIdx.x; b < n_tiles; b += blockDim.x) {
+      if (cnt[b]) base[b] = atomicAdd(fill + b, cnt[b]);
+      cnt[b] = 0;
+    }
+    __syncthreads();
+  }
+  for_tile_runs(row_cnt, row_cols, T, n_sel, rows_per_warp,
+                [&](int64_t t, const int32_t* cols, int n, int32_t tl, int i) {
+    // the run ends at the first key of a later tile; a tile holds at most 128
+    // distinct keys, so it ends within [i + 1, i + 128]
+    int lo = i + 1, hi = min(n, i + 128);
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if ((cols[mid] >> kTileShift) > tl) hi = mid;
+      else lo = mid + 1;
+    }
+    const int p = local ? base[tl] + atomicAdd(cnt + tl, 1) : atomicAdd(fill + tl, 1);
+    ent[p] = (t << 32) | (static_cast<int64_t>(i) << 8) | static_cast<int64_t>(lo - i - 1);
+  });
+}
+
+// One block per tile: sort its list ascending (by query), then record where each
+// query phase starts in it (phase_ptr[tile * (P + 1) + p]).  Lists of up to
+// `cap` entries are sorted in shared memory, longer ones in place in global
+// memory.
+__global__ void __launch_bounds__(1024) tile_sort_kernel(const int32_t* __restrict__ ptr, int64_t* __restrict__ ent,
+                                                         int P, int C, int cap, int32_t* __restrict__ phase_ptr) {
+  extern __shared__ int64_t tsv[];
+  const int64_t b = blockIdx.x;
+  const int lo = ptr[b], len = ptr[b + 1] - lo;
+  int32_t* pp = phase_ptr + b * (P + 1);
+  int64_t* seg = ent + lo;
+  if (len <= 1) {
+    for (int p = threadIdx.x; p <= P; p += blockDim.x)
+      pp[p] = lo + ((len == 1 && (seg[0] >> 32) < static_cast<int64_t>(p) * C) ? 1 : 0);
     return;
   }
+  int n2 = 1;
+  while (n2 < len) n2 <<= 1;
+  if (n2 <= cap) {
+    for (int i = threadIdx.x; i < n2; i += blockDim.x) tsv[i] = i < len ? seg[i] : LLONG_MAX;
+    __syncthreads();
+    block_sort<int64_t>(tsv, n2, n2);
+    for (int i = threadIdx.x; i < len; i += blockDim.x) seg[i] = tsv[i];
+    for (int p = threadIdx.x; p <= P; p += blockDim.x)
+      pp[p] = lo + lower_bound_query(tsv, len, static_cast<int64_t>(p) * C);
+  } else {
+    block_sort<int64_t>(seg, len, n2);
+    for (int p = threadIdx.x; p <= P; p += blockDim.x)
+      pp[p] = lo + lower_bound_query(seg, len, static_cast<int64_t>(p) * C);
+  }
+}
+
+// One warp per tile: lane 0 appends the tile's non-empty phase ranges to the
+// per-phase work lists, wl[p][*] = (tile, first entry, end entry, flags), flags
+// bit 0: no entries of the tile before this range, bit 1: none after it, bits
+// 2..: the number of earlier non-empty phases of the tile (the range's place in
+// the tile's accumulation order).  A tile that no query routes to gets its
+// dK/dV rows zeroed by the warp.
+__global__ void __launch_bounds__(256) tile_worklist_kernel(
+    const int32_t* __restrict__ ptr, const int32_t* __restrict__ phase_ptr, int64_t n_tiles, int64_t T_kv, int G,
+    int P, int32_t* __restrict__ wl_cnt, int4* __restrict__ wl, uint8_t* __restrict__ dk, uint8_t* __restrict__ dv,
+    int out_bytes) {
+  const int lane = threadIdx.x & 31;
+  const int64_t b = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (b >= n_tiles) return;
+  const int q0 = ptr[b], q1 = ptr[b + 1];
+  if (q0 == q1) {
+    const int64_t k0 = b << kTileShift, k1 = min(T_kv, (b + 1) << kTileShift);
+    const int64_t row = static_cast<int64_t>(G) * kHeadDim * out_bytes;  // bytes per key, a multiple of 16
+    uint4* rk = reinterpret_cast<uint4*>(dk + k0 * row);
+    uint4* rv = reinterpret_cast<uint4*>(dv + k0 * row);
+    for (int64_t i = lane; i < (k1 - k0) * row / 16; i += 32) rk[i] = rv[i] = make_uint4(0, 0, 0, 0);
+    return;
+  }
+  if (lane != 0) return;
   const int32_t* pp = phase_ptr + b * (P + 1);
+  int ord = 0;
   for (int p = 0; p < P; ++p) {
     const int lo = pp[p], hi = pp[p + 1];
     if (hi > lo) {
       const int slot = atomicAdd(wl_cnt + p, 1);
-      wl[static_cast<int64_t>(p) * n_quads + slot] =
-          make_int4(static_cast<int>(b), lo, hi, (lo == q0 ? 1 : 0) | (hi == q1 ? 2 : 0));
+      wl[static_cast<int64_t>(p) * n_tiles + slot] =
+          make_int4(static_cast<int>(b), lo, hi, (lo == q0 ? 1 : 0) | (hi == q1 ? 2 : 0) | (ord << 2));
+      ++ord;
     }
   }
 }
@@ -401,15 +537,15 @@ static int next_pow2(int x) {
 }
 
 cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel, int32_t* row_cnt,
-                              int32_t* row_cols, int32_t* quad_cnt, int* status, const void* dout,
+                              int32_t* row_cols, int32_t* bucket_cnt, int cnt_shift, int* status, const void* dout,
                               const void* out, float* delta, int H, cudaStream_t s) {
   const auto* dq = static_cast<const __nv_bfloat16*>(dout);
   const auto* o = static_cast<const __nv_bfloat16*>(out);
   const unsigned wblocks = static_cast<unsigned>((T + 7) / 8);
   const int32_t tkv = static_cast<int32_t>(T_kv);
 #define QSA_ROWS_WARP(NPL)                                                                                       \
-  route_rows_warp_kernel<NPL><<<wblocks, 256, 0, s>>>(routes, T, tkv, n_sel, row_cnt, row_cols, quad_cnt, status, \
-                                                      dq, o, delta, H);                                          \
+  route_rows_warp_kernel<NPL><<<wblocks, 256, 0, s>>>(routes, T, tkv, n_sel, row_cnt, row_cols, bucket_cnt,     \
+                                                      cnt_shift, status, dq, o, delta, H);                       \
   return cudaGetLastError()
   if (n_sel <= 64) { QSA_ROWS_WARP(2); }
   if (n_sel <= 128) { QSA_ROWS_WARP(4); }
@@ -426,7 +562,7 @@ cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, in
     if (e != cudaSuccess) return e;
   }
   route_rows_kernel<<<static_cast<unsigned>(T), kRowThreads, smem, s>>>(
-      routes, tkv, n_sel, n2, row_cnt, row_cols, quad_cnt, status, dq, o, delta, H);
+      routes, tkv, n_sel, n2, row_cnt, row_cols, bucket_cnt, cnt_shift, status, dq, o, delta, H);
   return cudaGetLastError();
 }
 
@@ -449,11 +585,46 @@ cudaError_t launch_quad_sort(const int32_t* quad_ptr, int64_t n_quads, int64_t* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_quad_worklist(const int32_t* quad_ptr, const int32_t* phase_ptr, int64_t n_quads, int64_t T_kv,
+cudaError_t launch_tile_count(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel,
+                              int64_t n_tiles, int32_t* tile_cnt, cudaStream_t s) {
+  const int rpw = tile_rows_per_warp(n_sel);
+  const int64_t blocks = (T + 8 * rpw - 1) / (8 * rpw);
+  const size_t smem = n_tiles <= kTileBins ? static_cast<size_t>(n_tiles) * 4 : 0;
+  tile_count_kernel<<<static_cast<unsigned>(blocks), 256, smem, s>>>(row_cnt, row_cols, T, n_sel, rpw, n_tiles,
+                                                                     tile_cnt);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_fill(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel, int64_t n_tiles,
+                             int32_t* tile_fill, int64_t* tile_ent, cudaStream_t s) {
+  const int rpw = tile_rows_per_warp(n_sel);
+  const int64_t blocks = (T + 8 * rpw - 1) / (8 * rpw);
+  const size_t smem = n_tiles <= kTileBins ? static_cast<size_t>(n_tiles) * 8 : 0;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(tile_fill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  tile_fill_kernel<<<static_cast<unsigned>(blocks), 256, smem, s>>>(row_cnt, row_cols, T, n_sel, rpw, n_tiles,
+                                                                    tile_fill, tile_ent);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_sort(const int32_t* tile_ptr, int64_t n_tiles, int64_t* tile_ent, int P, int C,
+                             int32_t* phase_ptr, cudaStream_t s) {
+  constexpr int kCap = 16384;  // int64 entries sorted in shared memory (128 KB)
+  const int smem = kCap * static_cast<int>(sizeof(int64_t));
+  cudaError_t e = cudaFuncSetAttribute(tile_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  tile_sort_kernel<<<static_cast<unsigned>(n_tiles), 1024, smem, s>>>(tile_ptr, tile_ent, P, C, kCap, phase_ptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_worklist(const int32_t* tile_ptr, const int32_t* phase_ptr, int64_t n_tiles, int64_t T_kv,
                                  int G, int P, int32_t* wl_cnt, int4* wl, void* dk, void* dv, bool f32_out,
                                  cudaStream_t s) {
-  quad_worklist_kernel<<<static_cast<unsigned>((n_quads + 255) / 256), 256, 0, s>>>(
-      quad_ptr, phase_ptr, n_quads, T_kv, G, P, wl_cnt, wl, static_cast<uint8_t*>(dk), static_cast<uint8_t*>(dv),
+  tile_worklist_kernel<<<static_cast<unsigned>((n_tiles * 32 + 255) / 256), 256, 0, s>>>(
+      tile_ptr, phase_ptr, n_tiles, T_kv, G, P, wl_cnt, wl, static_cast<uint8_t*>(dk), static_cast<uint8_t*>(dv),
       f32_out ? 4 : 2);
   return cudaGetLastError();
 }

@@ -69,6 +69,10 @@ def library() -> ctypes.CDLL:
     lib.qsa_route_plan_scratch_size.argtypes = [i64, i64]
     lib.qsa_route_plan.restype = i32
     lib.qsa_route_plan.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp, vp, sz, vp]
+    lib.qsa_tile_plan_scratch_size.restype = sz
+    lib.qsa_tile_plan_scratch_size.argtypes = [i64, i64]
+    lib.qsa_tile_plan.restype = i32
+    lib.qsa_tile_plan.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp, vp, sz, vp]
     _lib = lib
     return lib
 
@@ -222,6 +226,24 @@ def route_plan(routes, T_kv: int):
                             _ptr(quad_ent), _ptr(scratch), scratch.numel(), _stream(dev))
     _check(st, "qsa_route_plan")
     return row_cnt, row_cols, quad_ptr, quad_ent
+
+
+def tile_plan(routes, T_kv: int):
+    """qsa_tile_plan: ``(row_cnt, row_cols, tile_ptr, tile_ent)`` device tensors."""
+    lib = library()
+    routes = _prep(routes, torch.int32, "routes")
+    T, n_sel = routes.shape
+    dev = routes.device
+    nt = (T_kv + 127) // 128
+    row_cnt = torch.empty(T, dtype=torch.int32, device=dev)
+    row_cols = torch.empty(T, n_sel, dtype=torch.int32, device=dev)
+    tile_ptr = torch.empty(nt + 1, dtype=torch.int32, device=dev)
+    tile_ent = torch.empty(T * n_sel, dtype=torch.int64, device=dev)
+    scratch = torch.empty(max(256, lib.qsa_tile_plan_scratch_size(T, T_kv)), dtype=torch.uint8, device=dev)
+    st = lib.qsa_tile_plan(_ptr(routes), T, T_kv, n_sel, _ptr(row_cnt), _ptr(row_cols), _ptr(tile_ptr),
+                           _ptr(tile_ent), _ptr(scratch), scratch.numel(), _stream(dev))
+    _check(st, "qsa_tile_plan")
+    return row_cnt, row_cols, tile_ptr, tile_ent
 
 
 def bitmap_routes(sel_blocks, lo, hi, blk_base, tok_base, T_kv: int, n_sel: int, block_size: int = 4):
