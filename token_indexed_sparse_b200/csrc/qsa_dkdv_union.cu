@@ -19,7 +19,7 @@
 //
 // Warp roles (384 threads): warp 6 schedules (claims units, cuts them into
 // chunks of 4 entries, publishes each chunk's descriptor in a shared-memory ring
-// and prefetches its rows, records and keys into L2); warps 0-5 fill whole
+// and prefetches its records and keys into L2); warps 0-5 fill whole
 // chunks, warp w the chunks of stage w of the 6-stage shared-memory ring (zero
 // A, gather B rows with cp.async, store the records into their A rows); warp 7
 // (one thread) issues the MMAs; warps 8-11 (tensor-memory lane quarters 0-3)
@@ -210,6 +210,25 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
       const int s = c % kUStages;
       const bool end = hd.x < 0;
       if (end && hd.y == 0) break;  // an end marker for a warp whose chunk the MMA never reaches
+      const int n = hd.z & 255, r = hd.z >> 10, g = r >> 1, tensor = r & 1, tile = hd.w;
+      // the records and keys of the chunk's unions (j < 32), loaded first so that
+      // their latency overlaps the wait for the stage, the zeroing and the row
+      // gather; record j of union u goes to A row (key - tile base), K columns
+      // 12 u .. 12 u + 11 (24-byte records of 12 heads: dK takes dS, dV takes P)
+      const uint16_t* recs = tensor ? prec : dsrec;
+      const int key0 = tile * kUKeys;
+      int32_t key[kUUnions];
+      uint2 val[kUUnions][3];
+#pragma unroll
+      for (int u = 0; u < kUUnions; ++u) {
+        const int64_t t = e[u] >> 32;
+        const int i0 = static_cast<int>((e[u] >> 8) & 0x3fff), cnt = static_cast<int>(e[u] & 0x7f) + 1;
+        const bool ok_j = u < n && lane < cnt;
+        const uint2* rec = reinterpret_cast<const uint2*>(recs + ((t * G + g) * n_sel + i0) * kURec);
+        key[u] = ok_j ? __ldg(row_cols + t * n_sel + i0 + lane) : -1;
+#pragma unroll
+        for (int hq = 0; hq < 3; ++hq) val[u][hq] = ok_j ? __ldg(rec + lane * 3 + hq) : make_uint2(0, 0);
+      }
       // stage s is free once the MMAs of chunk c - kUStages completed
       if (c >= kUStages) {
         if (lane == 0) got = u_wait(sbase + kUBarEmpty + 8 * s, ((c / kUStages) - 1) & 1, abort_flag);
@@ -223,7 +242,6 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
         }
         break;
       }
-      const int n = hd.z & 255, r = hd.z >> 10, g = r >> 1, tensor = r & 1, tile = hd.w;
       // zero A (12 KB): unselected (union, key) slots must read as 0
       {
         uint4* a = reinterpret_cast<uint4*>(smem + s * kUStage + kUBBytes);
@@ -247,22 +265,6 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
         }
       }
       cp_async_commit();
-      // A: record j of union u goes to row (key - tile base), K columns 12 u .. 12 u + 11
-      // (24-byte records of 12 heads: dK takes dS, dV takes P)
-      const uint16_t* recs = tensor ? prec : dsrec;
-      const int key0 = tile * kUKeys;
-      int32_t key[kUUnions];
-      uint2 val[kUUnions][3];
-#pragma unroll
-      for (int u = 0; u < kUUnions; ++u) {
-        const int64_t t = e[u] >> 32;
-        const int i0 = static_cast<int>((e[u] >> 8) & 0x3fff), cnt = static_cast<int>(e[u] & 0x7f) + 1;
-        const bool ok_j = u < n && lane < cnt;
-        const uint2* rec = reinterpret_cast<const uint2*>(recs + ((t * G + g) * n_sel + i0) * kURec);
-        key[u] = ok_j ? __ldg(row_cols + t * n_sel + i0 + lane) : -1;
-#pragma unroll
-        for (int hq = 0; hq < 3; ++hq) val[u][hq] = ok_j ? __ldg(rec + lane * 3 + hq) : make_uint2(0, 0);
-      }
       __syncwarp();  // the zeroing above before the record stores below
       uint8_t* abase = smem + s * kUStage + kUBBytes;
       auto put = [&](int u, int32_t k, const uint2 (&v)[3]) {
@@ -435,8 +437,8 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
     // ------------------------------------------------------------ scheduler
     // Claims units (one ahead) in phase order, cuts them into chunks of up to 4
     // entries, writes each chunk's descriptor and entries into the ring, and
-    // prefetches into L2 what the chunk's worker will read: the unions' Q (or
-    // dO) rows, record runs and key runs.
+    // prefetches into L2 the record runs and key runs the chunk's worker will
+    // load into registers (up to kURing chunks ahead).
     int claim_p = 0;
     // unit U -> its phase p, and inside the phase tensor-major order (every dK
     // unit, then every dV unit, so one tensor's rows are live in L2 at a time):
@@ -458,11 +460,12 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
       r = 2 * (rem % G) + tensor;
       item = __ldg(wl + idx);
     };
-    auto prefetch_l2 = [&](const void* p, int64_t bytes) {  // 16-byte aligned window around [p, p + bytes)
-      const uintptr_t a0 = reinterpret_cast<uintptr_t>(p) & ~uintptr_t{15};
-      const uintptr_t a1 = (reinterpret_cast<uintptr_t>(p) + bytes + 15) & ~uintptr_t{15};
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(a0), "r"(static_cast<uint32_t>(a1 - a0))
-                   : "memory");
+    // L2 prefetch of the 128-byte lines of [p, p + bytes) (a plain per-line hint:
+    // the bulk prefetch goes through the bulk-copy unit, one operation at a time)
+    auto prefetch_l2 = [&](const void* p, int64_t bytes) {
+      const uintptr_t a0 = reinterpret_cast<uintptr_t>(p);
+      for (uintptr_t a = a0 & ~uintptr_t{127}; a < a0 + bytes; a += 128)
+        asm volatile("prefetch.global.L2 [%0];\n" ::"l"(a < a0 ? a0 : a) : "memory");
     };
     int c = 0;
     bool ok = true;
@@ -472,14 +475,16 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
     if (cur.x >= 0) claim(nxt, nxt_idx, nxt_r);
     while (ok && cur.x >= 0) {
       const int g = cur_r >> 1, tensor = cur_r & 1;
+      // windows of up to 32 entries, lane i holding entry w0 + i; the next
+      // window's entries are loaded while this one is published
+      int64_t el_next = cur.y + lane < cur.z ? __ldg(ent + cur.y + lane) : 0;
       for (int w0 = cur.y; ok && w0 < cur.z; w0 += 32) {
-        // a window of up to 32 entries: lane i holds entry w0 + i
         const bool have = w0 + lane < cur.z;
-        const int64_t el = have ? __ldg(ent + w0 + lane) : 0;
-        if (have) {
+        const int64_t el = el_next;
+        el_next = w0 + 32 + lane < cur.z ? __ldg(ent + w0 + 32 + lane) : 0;
+        if (have) {  // the records and keys the workers load into registers
           const int64_t t = el >> 32;
           const int i0 = static_cast<int>((el >> 8) & 0x3fff), cnt = static_cast<int>(el & 0x7f) + 1;
-          prefetch_l2((tensor ? dout : q) + (t * H + g * kHeadsPerGroup) * kHeadDim, kHeadsPerGroup * kHeadDim * 2);
           prefetch_l2((tensor ? prec : dsrec) + ((t * G + g) * n_sel + i0) * kURec, cnt * kURec * 2);
           prefetch_l2(row_cols + t * n_sel + i0, cnt * 4);
         }
