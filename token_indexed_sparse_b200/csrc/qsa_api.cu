@@ -42,7 +42,7 @@ void dkdv_phases(int64_t T, int H, int* P, int* C) {
 
 struct Layout {
   size_t status = 0, row_cnt = 0, row_cols = 0, tile_ctr = 0, tile_ptr = 0, tile_fill = 0, tile_ent = 0, delta = 0,
-         prec = 0, dsrec = 0, phase_ptr = 0, wl = 0, partial = 0, total = 0;
+         pds = 0, phase_ptr = 0, wl = 0, partial = 0, total = 0;
   int P = 1, C = 1;
 };
 
@@ -73,8 +73,7 @@ Layout make_layout(int64_t T, int64_t T_kv, int H, int G, int n_sel, bool backwa
     L.tile_fill = take(nt * 4);
     L.tile_ent = take(pairs * 8);  // at most one entry per routed pair
     L.delta = take(static_cast<size_t>(T) * H * 4);
-    L.prec = take(pairs * G * 24);   // BF16 P of every routed pair, 12 heads
-    L.dsrec = take(pairs * G * 24);  // BF16 dS
+    L.pds = take(pairs * G * 48);  // BF16 [P | dS] of every routed pair, 12 heads each
     L.phase_ptr = take(nt * (L.P + 1) * 4);
     L.wl = take(static_cast<size_t>(L.P) * nt * 16);
     L.partial = take(nt * G * 2 * 128 * 256 * 4);  // FP32 dK and dV of every (tile, group)
@@ -137,8 +136,7 @@ static qsa_status_t backward_impl(const void* grad_out, const void* q, const voi
   int32_t* tile_fill = at<int32_t>(workspace, L.tile_fill);
   int64_t* tile_ent = at<int64_t>(workspace, L.tile_ent);
   float* delta = at<float>(workspace, L.delta);
-  uint16_t* prec = at<uint16_t>(workspace, L.prec);    // P  [T, G, n_sel, 12]
-  uint16_t* dsrec = at<uint16_t>(workspace, L.dsrec);  // dS [T, G, n_sel, 12]
+  uint16_t* pds = at<uint16_t>(workspace, L.pds);  // [T, G, n_sel, 24]
   int32_t* phase_ptr = at<int32_t>(workspace, L.phase_ptr);
   int4* wl = at<int4>(workspace, L.wl);
   float* partial = at<float>(workspace, L.partial);
@@ -155,10 +153,10 @@ static qsa_status_t backward_impl(const void* grad_out, const void* q, const voi
   QSA_TRY(qsa::launch_tile_sort(tile_ptr, nt, tile_ent, L.P, L.C, phase_ptr, s));
   QSA_TRY(qsa::launch_tile_worklist(tile_ptr, phase_ptr, nt, T_kv, G, L.P, wl_cnt, wl, dk, dv, kv_f32, s));
   QSA_TRY(ev.mark(3));
-  QSA_TRY(qsa::launch_backward_dq(grad_out, q, k, v, lse, delta, row_cnt, row_cols, T, G, n_sel, scale, dq, prec,
-                                  dsrec, s));
+  QSA_TRY(qsa::launch_backward_dq(grad_out, q, k, v, lse, delta, row_cnt, row_cols, T, G, n_sel, scale, dq, pds,
+                                  s));
   QSA_TRY(ev.mark(4));
-  QSA_TRY(qsa::launch_backward_dkdv_union(grad_out, q, prec, dsrec, row_cols, tile_ent, wl_cnt, wl, claim, done,
+  QSA_TRY(qsa::launch_backward_dkdv_union(grad_out, q, pds, row_cols, tile_ent, wl_cnt, wl, claim, done,
                                           L.P, nt, T_kv, G, n_sel, scale, partial, dk, dv, kv_f32, status, s));
   QSA_TRY(ev.mark(5));
   return QSA_OK;

@@ -8,9 +8,9 @@
 // This file holds dq_kernel, persistent over (query t, group g) items: it
 // recomputes S and dP over R_t (K/V rows gathered like the forward), forms P
 // and dS with delta from the route kernel, accumulates dQ, and stores the BF16
-// P and dS of every routed pair for the dK/dV pass (qsa_dkdv_union.cu): two
-// arrays of 24-byte records, P [T, G, n_sel, 12] and dS [T, G, n_sel, 12], one
-// record per (t, g, position in R_t).  No floating-point atomics.
+// P and dS of every routed pair for the dK/dV pass (qsa_dkdv_union.cu): one
+// 48-byte record [P h0..h11 | dS h0..h11] per (t, g, position in R_t), pds
+// [T, G, n_sel, 24].  No floating-point atomics.
 #include "qsa_internal.h"
 #include "qsa_pipe.cuh"
 
@@ -28,7 +28,7 @@ namespace {
 // buffer.  Per chunk, warp w computes S = Q K^T and dP = dO V^T for keys
 // 8w..8w+7, P = exp2(S*scale*log2e - lse*log2e), dS = P (dP - delta), stores the
 // BF16 P / dS records and accumulates dQ[:, DPW*w : DPW*(w+1)] += dS K.
-constexpr int kRec = 24;  // bf16 per (t, g, key) staged in shared memory: 12 P + 12 dS
+constexpr int kRec = 24;  // bf16 per (t, g, key) record: 12 P + 12 dS
 constexpr int kFirst = 1, kLast = 2, kSlot = 4;
 
 template <int NW, int STAGES, int CPS>
@@ -66,7 +66,7 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
           const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
           const float* __restrict__ lse, const float* __restrict__ delta, const int32_t* __restrict__ row_cnt,
           const int32_t* __restrict__ row_cols, int64_t n_items, int G, int n_sel, float scale, float scale_log2,
-          __nv_bfloat16* __restrict__ dq, uint16_t* __restrict__ prec, uint16_t* __restrict__ dsrec) {
+          __nv_bfloat16* __restrict__ dq, uint16_t* __restrict__ pds) {
   using S_ = DqShape<NW, STAGES, CPS>;
   constexpr int KEYS = S_::kKeys, kTile = S_::kTile, kStageBytes = S_::kStageBytes, kDsStride = S_::kDsStride;
   constexpr int kNt = S_::kNt, kKs = S_::kKs, kItemBytes = S_::kItemBytes, kThreads = S_::kThreads;
@@ -200,45 +200,24 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
     const uint32_t D23 = pack_bf16(p2 * (dp[2] - dl1), p3 * (dp[3] - dl1));
     *reinterpret_cast<uint32_t*>(sDS + gq * kDsStride + key0) = D01;
     *reinterpret_cast<uint32_t*>(sDS + (gq + 8) * kDsStride + key0) = D23;
-    // records: the chunk's P run [key][h0..h11], then its dS run
-    uint16_t* sD = sRec + KEYS * kHeadsPerGroup;
-    sRec[key0 * kHeadsPerGroup + gq] = static_cast<uint16_t>(P01 & 0xffff);
-    sRec[(key0 + 1) * kHeadsPerGroup + gq] = static_cast<uint16_t>(P01 >> 16);
-    sD[key0 * kHeadsPerGroup + gq] = static_cast<uint16_t>(D01 & 0xffff);
-    sD[(key0 + 1) * kHeadsPerGroup + gq] = static_cast<uint16_t>(D01 >> 16);
+    // records: [key][P h0..h11 | dS h0..h11]
+    sRec[key0 * kRec + gq] = static_cast<uint16_t>(P01 & 0xffff);
+    sRec[(key0 + 1) * kRec + gq] = static_cast<uint16_t>(P01 >> 16);
+    sRec[key0 * kRec + 12 + gq] = static_cast<uint16_t>(D01 & 0xffff);
+    sRec[(key0 + 1) * kRec + 12 + gq] = static_cast<uint16_t>(D01 >> 16);
     if (gq + 8 < kHeadsPerGroup) {
-      sRec[key0 * kHeadsPerGroup + gq + 8] = static_cast<uint16_t>(P23 & 0xffff);
-      sRec[(key0 + 1) * kHeadsPerGroup + gq + 8] = static_cast<uint16_t>(P23 >> 16);
-      sD[key0 * kHeadsPerGroup + gq + 8] = static_cast<uint16_t>(D23 & 0xffff);
-      sD[(key0 + 1) * kHeadsPerGroup + gq + 8] = static_cast<uint16_t>(D23 >> 16);
+      sRec[key0 * kRec + gq + 8] = static_cast<uint16_t>(P23 & 0xffff);
+      sRec[(key0 + 1) * kRec + gq + 8] = static_cast<uint16_t>(P23 >> 16);
+      sRec[key0 * kRec + 20 + gq] = static_cast<uint16_t>(D23 & 0xffff);
+      sRec[(key0 + 1) * kRec + 20 + gq] = static_cast<uint16_t>(D23 >> 16);
     }
     __syncthreads();
     {
-      // the chunk's staged P and dS runs -> the same runs of the two record arrays
-      // (24 bytes per key; 16-byte stores when the run starts 16-byte aligned)
+      // the chunk's records, 48 bytes per key, to their run of the record array
       const int base = (d.w >> 3) * KEYS;
-      const int64_t r0 = ((t * G + g) * n_sel + base) * kHeadsPerGroup;
-      uint16_t* dp = prec + r0;
-      uint16_t* dd = dsrec + r0;
-      const uint16_t* sD = sRec + KEYS * kHeadsPerGroup;
-      const int words = nk * 3;  // 8-byte words per run
-      if (((reinterpret_cast<uintptr_t>(dp) | reinterpret_cast<uintptr_t>(dd)) & 15) == 0) {
-        const uint4* s4p = reinterpret_cast<const uint4*>(sRec);
-        const uint4* s4d = reinterpret_cast<const uint4*>(sD);
-        for (int i = tid; i < words / 2; i += kThreads) {
-          reinterpret_cast<uint4*>(dp)[i] = s4p[i];
-          reinterpret_cast<uint4*>(dd)[i] = s4d[i];
-        }
-        if ((words & 1) && tid == kThreads - 1) {
-          reinterpret_cast<uint2*>(dp)[words - 1] = reinterpret_cast<const uint2*>(sRec)[words - 1];
-          reinterpret_cast<uint2*>(dd)[words - 1] = reinterpret_cast<const uint2*>(sD)[words - 1];
-        }
-      } else {
-        for (int i = tid; i < words; i += kThreads) {
-          reinterpret_cast<uint2*>(dp)[i] = reinterpret_cast<const uint2*>(sRec)[i];
-          reinterpret_cast<uint2*>(dd)[i] = reinterpret_cast<const uint2*>(sD)[i];
-        }
-      }
+      const uint4* src = reinterpret_cast<const uint4*>(sRec);
+      uint4* dst = reinterpret_cast<uint4*>(pds + ((t * G + g) * n_sel + base) * kRec);
+      for (int i = tid; i < nk * 3; i += kThreads) dst[i] = src[i];
     }
     // dQ[:, DPW*w : DPW*(w+1)] += dS K over the chunk's keys
 #pragma unroll
@@ -277,7 +256,7 @@ constexpr int kDqWarps = 4, kDqStages = 2, kDqCtasPerSm = 2;
 cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* k, const void* v,
                                const float* lse, const float* delta, const int32_t* row_cnt,
                                const int32_t* row_cols, int64_t T, int G, int n_sel, float scale, void* dq,
-                               uint16_t* prec, uint16_t* dsrec, cudaStream_t s) {
+                               uint16_t* pds, cudaStream_t s) {
   using S_ = DqShape<kDqWarps, kDqStages, kDqCtasPerSm>;
   auto kern = dq_kernel<kDqWarps, kDqStages, kDqCtasPerSm>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S_::kSmemBytes);
@@ -288,7 +267,7 @@ cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* 
   kern<<<static_cast<unsigned>(grid), S_::kThreads, S_::kSmemBytes, s>>>(
       static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q),
       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), lse, delta, row_cnt, row_cols,
-      n_items, G, n_sel, scale, scale * kLog2e, static_cast<__nv_bfloat16*>(dq), prec, dsrec);
+      n_items, G, n_sel, scale, scale * kLog2e, static_cast<__nv_bfloat16*>(dq), pds);
   return cudaGetLastError();
 }
 

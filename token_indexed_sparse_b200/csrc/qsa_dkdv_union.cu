@@ -11,7 +11,7 @@
 // however many of the tile's keys it selected.  Per chunk of 4 unions:
 //   D [128 keys x 256 dims] += A [128 keys x 48] . B [48 x 256 dims]
 // with K row 12 u + h = head h of union u; A holds the BF16 dS (for dK) or P
-// (for dV) records the dQ kernel wrote (24 bytes per routed pair), zero where a
+// (for dV) halves of the 48-byte records the dQ kernel wrote, zero where a
 // union did not select the key; B holds the gathered Q (or dO) rows.  That is 3
 // tcgen05.mma kind::f16 (M 128, N 256, K 16), A K-major without swizzle, B MN-major with the 128-byte
 // swizzle, the accumulator in tensor memory (two 256-column buffers, so the
@@ -44,7 +44,7 @@ namespace {
 constexpr int kUThreads = 384;
 constexpr int kUWorkers = 6;                        // warps 0-5 fill chunks, warp w every stage-w chunk
 constexpr int kUSchedWarp = 6, kUMmaWarp = 7, kUEpiWarp0 = 8;
-constexpr int kURec = 12;                           // bf16 per (t, g, key) record of P or dS: 12 heads
+constexpr int kURec = 24;                           // bf16 per (t, g, key) record: 12 P + 12 dS
 constexpr int kUKeys = 128;                         // keys per tile (MMA M)
 constexpr int kUUnions = 4;                         // unions per chunk
 constexpr int kUK = kUUnions * kHeadsPerGroup;      // 48 K rows per chunk
@@ -133,8 +133,7 @@ __device__ __forceinline__ void u_ld32(uint32_t taddr, float (&v)[32]) {
 
 __global__ void __launch_bounds__(kUThreads, 1)
 dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ q,
-                  const uint16_t* __restrict__ prec, const uint16_t* __restrict__ dsrec,
-                  const int32_t* __restrict__ row_cols,
+                  const uint16_t* __restrict__ pds, const int32_t* __restrict__ row_cols,
                   const int64_t* __restrict__ ent, const int32_t* __restrict__ wl_cnt, const int4* __restrict__ wl,
                   int* __restrict__ claim_ctr, int* __restrict__ done, int P, int64_t n_tiles, int64_t T_kv, int G,
                   int n_sel, float scale,
@@ -194,6 +193,12 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
     // B with cp.async, stores each union's records into the A rows of their keys,
     // waits for its copies and marks the stage full.  Up to kUStages chunks are
     // in flight at once, one per warp, with no barrier between warps.
+    // A rows this lane wrote in the warp's previous chunk (its stage still holds
+    // them): clearing those 24-byte slots restores an all-zero A without
+    // rewriting the 12 KB tile; the whole tile is zeroed on the stage's first
+    // use and after a chunk whose records were not all tracked (runs > 32 keys)
+    int prev_m[kUUnions] = {-1, -1, -1, -1};
+    bool zero_all = true;
     for (int c = warp;; c += kUWorkers) {
       const int rs = c % kURing;
       bool got = true;
@@ -214,8 +219,7 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
       // the records and keys of the chunk's unions (j < 32), loaded first so that
       // their latency overlaps the wait for the stage, the zeroing and the row
       // gather; record j of union u goes to A row (key - tile base), K columns
-      // 12 u .. 12 u + 11 (24-byte records of 12 heads: dK takes dS, dV takes P)
-      const uint16_t* recs = tensor ? prec : dsrec;
+      // 12 u .. 12 u + 11 (dK takes the record's dS half, dV its P half)
       const int key0 = tile * kUKeys;
       int32_t key[kUUnions];
       uint2 val[kUUnions][3];
@@ -224,10 +228,10 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
         const int64_t t = e[u] >> 32;
         const int i0 = static_cast<int>((e[u] >> 8) & 0x3fff), cnt = static_cast<int>(e[u] & 0x7f) + 1;
         const bool ok_j = u < n && lane < cnt;
-        const uint2* rec = reinterpret_cast<const uint2*>(recs + ((t * G + g) * n_sel + i0) * kURec);
+        const uint2* rec = reinterpret_cast<const uint2*>(pds + ((t * G + g) * n_sel + i0) * kURec) + (tensor ? 0 : 3);
         key[u] = ok_j ? __ldg(row_cols + t * n_sel + i0 + lane) : -1;
 #pragma unroll
-        for (int hq = 0; hq < 3; ++hq) val[u][hq] = ok_j ? __ldg(rec + lane * 3 + hq) : make_uint2(0, 0);
+        for (int hq = 0; hq < 3; ++hq) val[u][hq] = ok_j ? __ldg(rec + lane * 6 + hq) : make_uint2(0, 0);
       }
       // stage s is free once the MMAs of chunk c - kUStages completed
       if (c >= kUStages) {
@@ -242,11 +246,23 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
         }
         break;
       }
-      // zero A (12 KB): unselected (union, key) slots must read as 0
-      {
-        uint4* a = reinterpret_cast<uint4*>(smem + s * kUStage + kUBBytes);
+      // A must read 0 in every (union, key) slot this chunk does not fill
+      uint8_t* abase = smem + s * kUStage + kUBBytes;
+      auto slot = [&](int u, int m, int hq) -> uint2* {
+        const int kk = u * kHeadsPerGroup + 4 * hq;
+        return reinterpret_cast<uint2*>(abase + (m >> 3) * kUASbo + (m & 7) * 16 + (kk >> 3) * 128 + (kk & 7) * 2);
+      };
+      if (zero_all) {
+        uint4* a = reinterpret_cast<uint4*>(abase);
 #pragma unroll 4
         for (int i = lane; i < kUABytes / 16; i += 32) a[i] = make_uint4(0, 0, 0, 0);
+      } else {
+#pragma unroll
+        for (int u = 0; u < kUUnions; ++u)
+          if (prev_m[u] >= 0) {
+#pragma unroll
+            for (int hq = 0; hq < 3; ++hq) *slot(u, prev_m[u], hq) = make_uint2(0, 0);
+          }
       }
       // B: the 12 head rows of each union (zero-filled for missing unions)
       {
@@ -266,28 +282,28 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
       }
       cp_async_commit();
       __syncwarp();  // the zeroing above before the record stores below
-      uint8_t* abase = smem + s * kUStage + kUBBytes;
-      auto put = [&](int u, int32_t k, const uint2 (&v)[3]) {
+      // stores record j of union u; returns its A row, or -1
+      auto put = [&](int u, int32_t k, const uint2 (&v)[3]) -> int {
         const int m = k - key0;
-        if (k < 0 || static_cast<unsigned>(m) >= static_cast<unsigned>(kUKeys)) return;  // never for a well-formed list
-        uint8_t* row = abase + (m >> 3) * kUASbo + (m & 7) * 16;
+        if (k < 0 || static_cast<unsigned>(m) >= static_cast<unsigned>(kUKeys)) return -1;  // never for a well-formed list
 #pragma unroll
-        for (int hq = 0; hq < 3; ++hq) {
-          const int kk = u * kHeadsPerGroup + 4 * hq;
-          *reinterpret_cast<uint2*>(row + (kk >> 3) * 128 + (kk & 7) * 2) = v[hq];
-        }
+        for (int hq = 0; hq < 3; ++hq) *slot(u, m, hq) = v[hq];
+        return m;
       };
 #pragma unroll
-      for (int u = 0; u < kUUnions; ++u) put(u, key[u], val[u]);
-      // unions with more than 32 keys in the tile (rare for sparse routes)
+      for (int u = 0; u < kUUnions; ++u) prev_m[u] = put(u, key[u], val[u]);
+      // unions with more than 32 keys in the tile (rare for sparse routes); their
+      // extra rows are not tracked, so the next chunk of this stage zeroes A
+      zero_all = false;
 #pragma unroll
       for (int u = 0; u < kUUnions; ++u) {
         const int64_t t = e[u] >> 32;
         const int i0 = static_cast<int>((e[u] >> 8) & 0x3fff), cnt = static_cast<int>(e[u] & 0x7f) + 1;
         if (u >= n || cnt <= 32) continue;
-        const uint2* rec = reinterpret_cast<const uint2*>(recs + ((t * G + g) * n_sel + i0) * kURec);
+        zero_all = true;
+        const uint2* rec = reinterpret_cast<const uint2*>(pds + ((t * G + g) * n_sel + i0) * kURec) + (tensor ? 0 : 3);
         for (int j = lane + 32; j < cnt; j += 32) {
-          const uint2 v[3] = {__ldg(rec + j * 3), __ldg(rec + j * 3 + 1), __ldg(rec + j * 3 + 2)};
+          const uint2 v[3] = {__ldg(rec + j * 6), __ldg(rec + j * 6 + 1), __ldg(rec + j * 6 + 2)};
           put(u, __ldg(row_cols + t * n_sel + i0 + j), v);
         }
       }
@@ -474,7 +490,7 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
     claim(cur, cur_idx, cur_r);
     if (cur.x >= 0) claim(nxt, nxt_idx, nxt_r);
     while (ok && cur.x >= 0) {
-      const int g = cur_r >> 1, tensor = cur_r & 1;
+      const int g = cur_r >> 1;
       // windows of up to 32 entries, lane i holding entry w0 + i; the next
       // window's entries are loaded while this one is published
       int64_t el_next = cur.y + lane < cur.z ? __ldg(ent + cur.y + lane) : 0;
@@ -485,7 +501,7 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
         if (have) {  // the records and keys the workers load into registers
           const int64_t t = el >> 32;
           const int i0 = static_cast<int>((el >> 8) & 0x3fff), cnt = static_cast<int>(el & 0x7f) + 1;
-          prefetch_l2((tensor ? prec : dsrec) + ((t * G + g) * n_sel + i0) * kURec, cnt * kURec * 2);
+          prefetch_l2(pds + ((t * G + g) * n_sel + i0) * kURec, cnt * kURec * 2);
           prefetch_l2(row_cols + t * n_sel + i0, cnt * 4);
         }
         const int w1 = min(cur.z, w0 + 32);
@@ -535,7 +551,7 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
 
 }  // namespace
 
-cudaError_t launch_backward_dkdv_union(const void* grad_out, const void* q, const uint16_t* prec, const uint16_t* dsrec,
+cudaError_t launch_backward_dkdv_union(const void* grad_out, const void* q, const uint16_t* pds,
                                        const int32_t* row_cols, const int64_t* tile_ent, const int32_t* wl_cnt,
                                        const int4* wl, int* claim_ctr, int* done, int P, int64_t n_tiles,
                                        int64_t T_kv, int G, int n_sel, float scale, float* partial, void* dk, void* dv,
@@ -544,7 +560,7 @@ cudaError_t launch_backward_dkdv_union(const void* grad_out, const void* q, cons
   cudaError_t e = cudaFuncSetAttribute(dkdv_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUSmem);
   if (e != cudaSuccess) return e;
   dkdv_union_kernel<<<static_cast<unsigned>(sm_count()), kUThreads, kUSmem, s>>>(
-      static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q), prec, dsrec, row_cols, tile_ent,
+      static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q), pds, row_cols, tile_ent,
       wl_cnt, wl, claim_ctr, done, P, n_tiles, T_kv, G, n_sel, scale, partial, dk, dv, f32_out, status);
   return cudaGetLastError();
 }

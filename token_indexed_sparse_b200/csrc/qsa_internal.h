@@ -50,11 +50,11 @@ cudaError_t launch_forward(const void* q, const void* k, const void* v, const in
                            const int32_t* row_cols, int64_t T, int G, int n_sel, float scale,
                            void* out, float* lse, int* status, cudaStream_t s);
 // dQ per query; also writes the BF16 probabilities / score gradients of every
-// routed pair, as two record arrays prec (P) and dsrec (dS), each [T, G, n_sel, 12].
+// routed pair, pds [T, G, n_sel, 24] ([P h0..h11 | dS h0..h11] per pair).
 cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* k, const void* v,
                                const float* lse, const float* delta, const int32_t* row_cnt,
                                const int32_t* row_cols, int64_t T, int G, int n_sel, float scale,
-                               void* dq, uint16_t* prec, uint16_t* dsrec, cudaStream_t s);
+                               void* dq, uint16_t* pds, cudaStream_t s);
 // SM count of the current device (cached).
 int sm_count();
 // dK/dV over 128-key tiles on the tensor cores, all P query phases in one
@@ -63,7 +63,7 @@ int sm_count();
 // from phase to phase through `partial`, ordered by its counter in `done`
 // (n_tiles * 2G ints; claim_ctr and done zeroed by the caller); final dK/dV BF16,
 // or FP32 when f32_out.  Sets *status = 3 if a bounded wait expired.  P <= 64.
-cudaError_t launch_backward_dkdv_union(const void* grad_out, const void* q, const uint16_t* prec, const uint16_t* dsrec,
+cudaError_t launch_backward_dkdv_union(const void* grad_out, const void* q, const uint16_t* pds,
                                        const int32_t* row_cols, const int64_t* tile_ent, const int32_t* wl_cnt,
                                        const int4* wl, int* claim_ctr, int* done, int P, int64_t n_tiles,
                                        int64_t T_kv, int G, int n_sel, float scale, float* partial, void* dk, void* dv,
