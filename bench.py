@@ -45,10 +45,10 @@ DKDV_FLOPS_PER_PAIR_HEAD = 4 * 256     # dK = dS^T Q, dV = P^T dO
 # summarised under profiles/, valid only for the kernel source it was taken on:
 # stage -> (bytes per step, source file, sha256 of that file at capture time).
 TRAFFIC = {
-    # one step's 16 dK/dV launches on seq32k: ncu dram__bytes_read.sum + dram__bytes_write.sum
-    # (profiles/dkdv_seq32k.md)
-    "bwd_dkdv": (5471966464, "token_indexed_sparse_b200/csrc/qsa_backward.cu",
-                 "0b663f1ac9daea7b9d38f0222f562e8088daeba11d9a02d65a9a74334b68f9a5"),
+    # the timed step's dK/dV launch on seq32k: ncu dram__bytes_read.sum + dram__bytes_write.sum
+    # (the dK/dV summary under profiles/)
+    "bwd_dkdv": (8614112256, "token_indexed_sparse_b200/csrc/qsa_dkdv_union.cu",
+                 "8d6ec9b097e814e2b3161ffb9569040ec0f4dbbaaae8c064c71bf6b84e3317d3"),
 }
 
 
