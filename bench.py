@@ -42,13 +42,17 @@ FWD_FLOPS_PER_PAIR_HEAD = 4 * 256      # QK^T + PV
 BWD_FLOPS_PER_PAIR_HEAD = 10 * 256     # S recompute, dP, dV, dQ, dK
 DKDV_FLOPS_PER_PAIR_HEAD = 4 * 256     # dK = dS^T Q, dV = P^T dO
 # DRAM bytes (read + write) per step of a stage's kernel, from the ncu capture
-# summarised under profiles/, valid only for the kernel source it was taken on:
-# stage -> (bytes per step, source file, sha256 of that file at capture time).
+# summarised under profiles/, valid only for the sources it was taken on:
+# stage -> (bytes per step, {source file: sha256 of that file at capture time}).
 TRAFFIC = {
     # the timed step's dK/dV launch on seq32k: ncu dram__bytes_read.sum + dram__bytes_write.sum
-    # (the dK/dV summary under profiles/)
-    "bwd_dkdv": (8614112256, "token_indexed_sparse_b200/csrc/qsa_dkdv_union.cu",
-                 "8d6ec9b097e814e2b3161ffb9569040ec0f4dbbaaae8c064c71bf6b84e3317d3"),
+    # (the dK/dV summary under profiles/); the kernel and the phase sizing of its launch
+    "bwd_dkdv": (13116903424, {
+        "token_indexed_sparse_b200/csrc/qsa_dkdv_union.cu":
+            "58c2aa937d264900c09f63146417623e1b87ccaf19d238adc79d5898fb66cddf",
+        "token_indexed_sparse_b200/csrc/qsa_api.cu":
+            "f1767b0adbc801a1f6652ad5362ca555cd832431f6d8ca6a868e67697100fa32",
+    }),
 }
 
 
@@ -56,9 +60,12 @@ def stage_traffic(stage):
     import hashlib
     if stage not in TRAFFIC:
         return None
-    nbytes, rel, digest = TRAFFIC[stage]
-    with open(os.path.join(ROOT, rel), "rb") as f:
-        return nbytes if hashlib.sha256(f.read()).hexdigest() == digest else None
+    nbytes, sources = TRAFFIC[stage]
+    for rel, digest in sources.items():
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != digest:
+                return None
+    return nbytes
 
 
 FWD_STAGES = ["fwd_route_rows", "fwd_attention"]

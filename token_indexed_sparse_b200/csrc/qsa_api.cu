@@ -26,11 +26,15 @@ qsa_status_t check_sizes(int64_t T, int64_t T_kv, int H, int G, int n_sel) {
 }
 
 // Query phases of the dK/dV pass: each phase covers C consecutive queries, chosen
-// so that one phase's Q and dO rows (C * H * 1 KB) stay resident in L2 (48 MiB);
-// at most 64 phases.
+// so that one phase's Q and dO rows (C * H * 1 KB; the pass reads one tensor at
+// a time) stay resident in L2 (48 MiB), but at least 4096 queries: every phase
+// boundary costs an FP32 partial read and write per (tile, group, tensor), and
+// with many heads the L2 bound alone makes phases so short that this dominates
+// (seq32k, 24 heads: 2048 queries per phase ran dK/dV in 7.7 ms, 4096 in 7.1 ms;
+// with 12 heads the bound is 4096 already).  At most 64 phases.
 void dkdv_phases(int64_t T, int H, int* P, int* C) {
   int64_t c = (int64_t{48} << 20) / (static_cast<int64_t>(H) * 1024);
-  c = c < 256 ? 256 : (c / 256) * 256;
+  c = c < 4096 ? 4096 : (c / 256) * 256;
   int64_t p = (T + c - 1) / c;
   if (p > 64) {
     c = (((T + 63) / 64) + 255) / 256 * 256;

@@ -12,19 +12,20 @@
 //   D [128 keys x 256 dims] += A [128 keys x 48] . B [48 x 256 dims]
 // with K row 12 u + h = head h of union u; A holds the BF16 dS (for dK) or P
 // (for dV) halves of the 48-byte records the dQ kernel wrote, zero where a
-// union did not select the key; B holds the gathered Q (or dO) rows.  That is 3
-// tcgen05.mma kind::f16 (M 128, N 256, K 16), A K-major without swizzle, B MN-major with the 128-byte
-// swizzle, the accumulator in tensor memory (two 256-column buffers, so the
-// epilogue of one unit overlaps the next unit's MMAs).
+// union did not select the key; B holds the gathered Q (or dO) rows.  That is
+// 3 tcgen05.mma kind::f16 (M 128, N 256, K 16), A K-major without swizzle, B
+// MN-major with the 128-byte swizzle, the accumulator in tensor memory (two
+// 256-column buffers, so the epilogue of one unit overlaps the next unit's MMAs).
 //
 // Warp roles (384 threads): warp 6 schedules (claims units, cuts them into
 // chunks of 4 entries, publishes each chunk's descriptor in a shared-memory ring
-// and prefetches its records and keys into L2); warps 0-5 fill whole
-// chunks, warp w the chunks of stage w of the 6-stage shared-memory ring (zero
-// A, gather B rows with cp.async, store the records into their A rows); warp 7
+// and prefetches its records and keys into L2); warps 0-5 fill whole chunks,
+// warp w the chunks of stage w of the 6-stage shared-memory ring (clear A,
+// gather B rows with cp.async, store the records into their A rows); warp 7
 // (one thread) issues the MMAs; warps 8-11 (tensor-memory lane quarters 0-3)
-// run the epilogue, thread = key row.  Units are claimed from one counter in phase order (phase 0's units, then
-// phase 1's, ...; inside a phase every dK unit before every dV unit), so the
+// run the epilogue, thread = key row.  Units are claimed from one counter in
+// phase order (phase 0's units, then phase 1's, ...; inside a phase every dK
+// unit before every dV unit), so the
 // CTAs work on about one phase and one tensor at a time and its Q (or dO) rows
 // stay in L2.  A unit sums its entries in list order; its epilogue waits until
 // the unit of the same (tile, group, tensor) in the previous non-empty phase has

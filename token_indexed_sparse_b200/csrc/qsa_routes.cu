@@ -552,7 +552,6 @@ cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, in
   if (n_sel <= 256) { QSA_ROWS_WARP(8); }
   if (n_sel <= 512) { QSA_ROWS_WARP(16); }
   if (n_sel <= 1024) { QSA_ROWS_WARP(32); }
-  if (n_sel <= 2048) { QSA_ROWS_WARP(64); }
 #undef QSA_ROWS_WARP
   const int n2 = next_pow2(n_sel);
   const size_t smem = static_cast<size_t>(n2 + 32) * sizeof(int32_t);
