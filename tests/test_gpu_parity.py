@@ -109,9 +109,13 @@ def test_parity_full_size_sampled(number):
     check_lse(lse[rows].cpu().numpy().astype(np.float64), r_lse)
     assert rel_err(f64(out[rows]), r_out) <= REL_TOL
     assert rel_err(f64(dq[rows]), r_dq) <= REL_TOL
-    # keys: random, the most recent (hot) ones, and one past every route
+    # keys: random, the most recent (hot) ones, one past every route, and a run
+    # of 16 consecutive keys inside one 128-key tile (they share the tile's
+    # query unions in the dK/dV kernel)
+    tile = int(rng.integers(0, wl.T_kv // 128))
     keys = np.unique(np.concatenate([rng.choice(wl.T_kv, 10, replace=False),
-                                     [wl.T_kv - 1, wl.T_kv - 5]]))
+                                     [wl.T_kv - 1, wl.T_kv - 5],
+                                     np.arange(tile * 128 + 40, tile * 128 + 56)]))
     r_dk, r_dv = oracle.backward_keys(dof, qf, kf, vf, routes, wl.scale, keys)
     assert rel_err(f64(dk[keys]), r_dk) <= REL_TOL
     assert rel_err(f64(dv[keys]), r_dv) <= REL_TOL
