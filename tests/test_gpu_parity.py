@@ -36,11 +36,20 @@ def to_dev(routes, *tensors):
     return (r, *[t.to(DEV) for t in tensors])
 
 
+def status_word(ws):
+    # the first int32 of a workspace: 0 unless a kernel gave up on a bounded wait
+    return int(ws[:4].view(torch.int32).item())
+
+
 def run_gpu(q, k, v, do, routes, scale):
     r, qd, kd, vd, dod = to_dev(routes, q, k, v, do)
+    T, H = qd.shape[0], qd.shape[1]
+    ws = torch.empty(qsa.backward_workspace_size(T, kd.shape[0], H, kd.shape[1], r.shape[1]),
+                     dtype=torch.uint8, device=DEV)
     out, lse = qsa.forward(qd, kd, vd, r, scale)
-    dq, dk, dv = qsa.backward(dod, qd, kd, vd, out, lse, r, scale)
+    dq, dk, dv = qsa.backward(dod, qd, kd, vd, out, lse, r, scale, workspace=ws)
     torch.cuda.synchronize()
+    assert status_word(ws) == 0
     return out, lse, dq, dk, dv
 
 
@@ -293,9 +302,13 @@ def test_backward_is_bitwise_deterministic():
     routes, q, k, v, do = inputs(wl)
     r, qd, kd, vd, dod = to_dev(routes, q, k, v, do)
     out, lse = qsa.forward(qd, kd, vd, r, wl.scale)
+    ws = torch.empty(qsa.backward_workspace_size(wl.T, wl.T_kv, wl.H, wl.G, routes.shape[1]),
+                     dtype=torch.uint8, device=DEV)
     first = qsa.backward(dod, qd, kd, vd, out, lse, r, wl.scale)
     for _ in range(2):
-        again = qsa.backward(dod, qd, kd, vd, out, lse, r, wl.scale)
+        again = qsa.backward(dod, qd, kd, vd, out, lse, r, wl.scale, workspace=ws)
+        torch.cuda.synchronize()
+        assert status_word(ws) == 0
         for a, b in zip(first, again):
             assert torch.equal(a, b)
     out2, lse2 = qsa.forward(qd, kd, vd, r, wl.scale)
