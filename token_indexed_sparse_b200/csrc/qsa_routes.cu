@@ -462,8 +462,9 @@ __global__ void __launch_bounds__(256) tile_fill_kernel(const int32_t* __restric
 
 // One block per tile: sort its list ascending (by query), then record where each
 // query phase starts in it (phase_ptr[tile * (P + 1) + p]).  Lists of up to
-// `cap` entries are sorted in shared memory, longer ones in place in global
-// memory.
+// `cap` entries are sorted in shared memory; longer ones run the same network
+// with all comparators inside a `cap`-sized piece in shared memory and only the
+// longer-distance ones in global memory.
 __global__ void __launch_bounds__(1024) tile_sort_kernel(const int32_t* __restrict__ ptr, int64_t* __restrict__ ent,
                                                          int P, int C, int cap, int32_t* __restrict__ phase_ptr) {
   extern __shared__ int64_t tsv[];
@@ -486,7 +487,51 @@ __global__ void __launch_bounds__(1024) tile_sort_kernel(const int32_t* __restri
     for (int p = threadIdx.x; p <= P; p += blockDim.x)
       pp[p] = lo + lower_bound_query(tsv, len, static_cast<int64_t>(p) * C);
   } else {
-    block_sort<int64_t>(seg, len, n2);
+    // the same bitonic network, in `cap`-sized pieces: every comparator whose
+    // two elements lie in one aligned piece runs in shared memory (a piece is
+    // loaded, +infinity past `len`, and written back), only the comparators of
+    // the levels above `cap` with distance >= cap run in global memory
+    auto piece = [&](int c0, bool full_sort, int h_top) {
+      for (int i = threadIdx.x; i < cap; i += blockDim.x) tsv[i] = c0 + i < len ? seg[c0 + i] : LLONG_MAX;
+      __syncthreads();
+      if (full_sort) {
+        block_sort<int64_t>(tsv, cap, cap);
+      } else {
+        for (int h = h_top; h >= 1; h >>= 1) {
+          for (int q = threadIdx.x; q < cap / 2; q += blockDim.x) {
+            const int i = (q / h) * 2 * h + (q % h), j = i + h;
+            const int64_t a = tsv[i], c = tsv[j];
+            if (c < a) { tsv[i] = c; tsv[j] = a; }
+          }
+          __syncthreads();
+        }
+      }
+      for (int i = threadIdx.x; i < cap && c0 + i < len; i += blockDim.x) seg[c0 + i] = tsv[i];
+      __syncthreads();
+    };
+    for (int c0 = 0; c0 < len; c0 += cap) piece(c0, true, 0);
+    for (int k = 2 * cap; k <= n2; k <<= 1) {
+      for (int q = threadIdx.x; q < n2 / 2; q += blockDim.x) {  // flip step of level k
+        const int off = q & (k / 2 - 1), base = (q / (k / 2)) * k;
+        const int i = base + off, j = base + k - 1 - off;
+        if (j < len) {
+          const int64_t a = seg[i], c = seg[j];
+          if (c < a) { seg[i] = c; seg[j] = a; }
+        }
+      }
+      __syncthreads();
+      for (int h = k / 4; h >= cap; h >>= 1) {  // half-cleaners across pieces
+        for (int q = threadIdx.x; q < n2 / 2; q += blockDim.x) {
+          const int i = (q / h) * 2 * h + (q % h), j = i + h;
+          if (j < len) {
+            const int64_t a = seg[i], c = seg[j];
+            if (c < a) { seg[i] = c; seg[j] = a; }
+          }
+        }
+        __syncthreads();
+      }
+      for (int c0 = 0; c0 < len; c0 += cap) piece(c0, false, cap / 2);
+    }
     for (int p = threadIdx.x; p <= P; p += blockDim.x)
       pp[p] = lo + lower_bound_query(seg, len, static_cast<int64_t>(p) * C);
   }
