@@ -42,9 +42,14 @@
 namespace qsa {
 namespace {
 
-constexpr int kUThreads = 384;
+// CTAs per SM and accumulator buffers per CTA (tensor memory: 256 columns per
+// buffer, 512 per SM)
+constexpr int kUCtasPerSm = 1, kUAccBufs = 2;
+constexpr int kUTmemCols = 256 * kUAccBufs;
 constexpr int kUWorkers = 6;                        // warps 0-5 fill chunks, warp w every stage-w chunk
 constexpr int kUSchedWarp = 6, kUMmaWarp = 7, kUEpiWarp0 = 8;
+constexpr int kUWarps = 12;
+constexpr int kUThreads = 32 * kUWarps;
 constexpr int kURec = 24;                           // bf16 per (t, g, key) record: 12 P + 12 dS
 constexpr int kUKeys = 128;                         // keys per tile (MMA M)
 constexpr int kUUnions = 4;                         // unions per chunk
@@ -78,9 +83,13 @@ static_assert(kUSmem <= 232448, "shared memory per block");
 // the barrier (a parity wait two phases early would pass at once).  The
 // descriptor ring is at least as deep as the worker count for the same reason.
 static_assert(kUWorkers == kUStages && kURing >= kUWorkers, "one worker per stage");
-static_assert(kUThreads == 32 * (kUEpiWarp0 + 4) && kUEpiWarp0 % 4 == 0 && kUSchedWarp >= kUWorkers &&
-                  kUMmaWarp > kUSchedWarp && kUMmaWarp < kUEpiWarp0,
+static_assert(kUEpiWarp0 % 4 == 0 && kUEpiWarp0 + 4 <= kUWarps && kUSchedWarp >= kUWorkers &&
+                  kUSchedWarp < kUWarps && kUMmaWarp >= kUWorkers && kUMmaWarp < kUWarps &&
+                  kUSchedWarp != kUMmaWarp && (kUMmaWarp < kUEpiWarp0 || kUMmaWarp >= kUEpiWarp0 + 4) &&
+                  (kUSchedWarp < kUEpiWarp0 || kUSchedWarp >= kUEpiWarp0 + 4),
               "warp roles (epilogue warps cover tensor-memory lane quarters 0-3 in order)");
+static_assert(kUTmemCols * kUCtasPerSm <= 512, "tensor memory per SM");
+static_assert((kUSmem + 1024) * kUCtasPerSm <= 233472, "shared memory per SM");
 constexpr uint32_t kUSpin = 1u << 22;
 constexpr int kChFirst = 1, kChLast = 2;
 // kind::f16: FP32 accumulate, BF16 A (K-major) and B (MN-major), N = 256, M = 128.
@@ -132,7 +141,7 @@ __device__ __forceinline__ void u_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__global__ void __launch_bounds__(kUThreads, 1)
+__global__ void __launch_bounds__(kUThreads, kUCtasPerSm)
 dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ q,
                   const uint16_t* __restrict__ pds, const int32_t* __restrict__ row_cols,
                   const int64_t* __restrict__ ent, const int32_t* __restrict__ wl_cnt, const int4* __restrict__ wl,
@@ -177,7 +186,7 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(sbase + kUOffTmem),
-                 "r"(512));
+                 "r"(kUTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n");
   }
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
@@ -329,9 +338,9 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
         }
         const int4 d = desc[s];
         if (d.y < 0) break;
-        const int buf = useq & 1;
-        if ((d.z & kChFirst) && useq >= 2 &&
-            !u_wait(sbase + kUBarAccEmpty + 8 * buf, ((useq >> 1) - 1) & 1, abort_flag)) {
+        const int buf = useq % kUAccBufs;
+        if ((d.z & kChFirst) && useq >= kUAccBufs &&
+            !u_wait(sbase + kUBarAccEmpty + 8 * buf, ((useq / kUAccBufs) - 1) & 1, abort_flag)) {
           ok = false;
           break;
         }
@@ -350,8 +359,8 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
         }
       }
       if (ok) {  // end marker for the epilogue
-        const int buf = useq & 1;
-        if (useq < 2 || u_wait(sbase + kUBarAccEmpty + 8 * buf, ((useq >> 1) - 1) & 1, abort_flag)) {
+        const int buf = useq % kUAccBufs;
+        if (useq < kUAccBufs || u_wait(sbase + kUBarAccEmpty + 8 * buf, ((useq / kUAccBufs) - 1) & 1, abort_flag)) {
           acc_desc[buf] = make_int4(-1, 0, 0, 0);
           mbar_arrive(sbase + kUBarAccFull + 8 * buf);
           mbar_arrive(sbase + kUBarAccFull + 8 * buf);
@@ -363,14 +372,14 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
       }
     }
     __syncwarp();
-  } else if (warp >= kUEpiWarp0) {
+  } else if (warp >= kUEpiWarp0 && warp < kUEpiWarp0 + 4) {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp - kUEpiWarp0;      // tensor-memory lanes 32 quarter .. + 31
     const int m = quarter * 32 + lane;          // key row within the tile
     const bool leader = quarter == 0 && lane == 0;
     for (int useq = 0;; ++useq) {
-      const int buf = useq & 1;
-      if (!u_wait(sbase + kUBarAccFull + 8 * buf, (useq >> 1) & 1, abort_flag)) break;
+      const int buf = useq % kUAccBufs;
+      if (!u_wait(sbase + kUBarAccFull + 8 * buf, (useq / kUAccBufs) & 1, abort_flag)) break;
       const int idx = acc_desc[buf].x, r = acc_desc[buf].y;
       if (idx < 0) break;
       asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
@@ -450,7 +459,7 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
         }
       }
     }
-  } else {
+  } else if (warp == kUSchedWarp) {
     // ------------------------------------------------------------ scheduler
     // Claims units (one ahead) in phase order, cuts them into chunks of up to 4
     // entries, writes each chunk's descriptor and entries into the ring, and
@@ -547,7 +556,7 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
   if (*abort_flag && tid == 0 && status) atomicExch(status, 3);
-  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(512));
+  if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kUTmemCols));
 }
 
 }  // namespace
@@ -560,7 +569,7 @@ cudaError_t launch_backward_dkdv_union(const void* grad_out, const void* q, cons
   if (P < 1 || P > kUMaxPhases) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(dkdv_union_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUSmem);
   if (e != cudaSuccess) return e;
-  dkdv_union_kernel<<<static_cast<unsigned>(sm_count()), kUThreads, kUSmem, s>>>(
+  dkdv_union_kernel<<<static_cast<unsigned>(kUCtasPerSm * sm_count()), kUThreads, kUSmem, s>>>(
       static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q), pds, row_cols, tile_ent,
       wl_cnt, wl, claim_ctr, done, P, n_tiles, T_kv, G, n_sel, scale, partial, dk, dv, f32_out, status);
   return cudaGetLastError();
