@@ -169,9 +169,11 @@ qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k,
 int qsa_launch_count(int64_t T, int64_t T_kv, int H, int G, int n_sel, int backward);
 
 /*
- * Route preprocessing on its own, exposing the index structures the attention
- * kernels consume.  Cites: "fa4_qsa" page, `_preprocess` (duplicates collapse,
- * invalid IDs discarded; forward and reverse lists).
+ * Route preprocessing on its own.  Cites: "fa4_qsa" page, `_preprocess`
+ * (duplicates collapse, invalid IDs discarded; forward and reverse lists).
+ * row_cnt / row_cols are the per-row lists the forward and dQ kernels consume;
+ * the reverse lists here are grouped by key quad with owner masks (the dK/dV
+ * pass uses the 128-key tile grouping of qsa_tile_plan instead).
  *   row_cnt  [T] int32       : |R_t|
  *   row_cols [T, n_sel] int32: R_t ascending in the first row_cnt[t] slots; the
  *                              remaining slots are left unspecified
