@@ -47,9 +47,9 @@ DKDV_FLOPS_PER_PAIR_HEAD = 4 * 256     # dK = dS^T Q, dV = P^T dO
 TRAFFIC = {
     # the timed step's dK/dV launch on seq32k: ncu dram__bytes_read.sum + dram__bytes_write.sum
     # (the dK/dV summary under profiles/); the kernel and the phase sizing of its launch
-    "bwd_dkdv": (13116903424, {
+    "bwd_dkdv": (13687003648, {
         "token_indexed_sparse_b200/csrc/qsa_dkdv_union.cu":
-            "58c2aa937d264900c09f63146417623e1b87ccaf19d238adc79d5898fb66cddf",
+            "3f17ce8a839d435e88248da8cc1c3393eaa0c76bbf7b119ec93fce2f9c41a17b",
         "token_indexed_sparse_b200/csrc/qsa_api.cu":
             "f1767b0adbc801a1f6652ad5362ca555cd832431f6d8ca6a868e67697100fa32",
     }),
