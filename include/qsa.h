@@ -135,7 +135,7 @@ qsa_status_t qsa_backward_fp32kv(const void* grad_out, const void* q, const void
  * CUDA events (cudaEvent_t, passed as qsa_event_t) on `stream` after each stage,
  * for per-kernel timing.  Stage i's event is recorded right after stage i is
  * enqueued; only the first min(n_stage_events, stage count) are recorded.
- * `stage_events` may be NULL when n_stage_events is 0.  The paper has no
+ * `stage_events` may be NULL when n_stage_events is 0.  The pages have no
  * counterpart: this is an instrumentation hook of this library.
  *   forward stages : 0 route rows (sort/dedup), 1 attention forward
  *   backward stages: 0 route rows (+ delta), 1 tile counts + scan, 2 tile fill,
@@ -289,7 +289,7 @@ qsa_status_t qsa_selector_topk(const float* scores, int64_t score_stride, int64_
  * example an extension running inside a host application that owns the device
  * allocator and offers it no allocation hook, or a latency-critical path that
  * must not call cudaMalloc (which can synchronise the device and has no bounded
- * latency).  The paper has no counterpart: this is an interface convenience of
+ * latency).  The pages have no counterpart: this is an interface convenience of
  * this library.
  *
  * Same arguments and results as qsa_forward, minus the workspace.  The scratch

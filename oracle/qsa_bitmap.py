@@ -11,7 +11,7 @@ block and ``tok_base`` first global token of the query's sequence) and section
 b = blk_base[t] + (j - tok_base[t]) // block_size, and j is allowed iff
 lo[t] <= j <= hi[t], 0 <= b < NB and sel_blocks[t, b] != 0).
 
-Readings where the page leaves a step open (also listed in the design doc):
+Readings where the page leaves a step open:
 
 * ``//`` is floor division (the page's notation is Python's), so a key before
   ``tok_base[t]`` maps to block ``blk_base[t] - 1`` or lower.

@@ -23,7 +23,7 @@ Sources (documentation pages, cited by page title and section):
   PV; empty rows give zero output and -inf LSE; the backward equations
   S, P, delta, dP, dS, dQ, dK, dV).
 
-Readings where the pages leave a step open (also listed in the design doc):
+Readings where the pages leave a step open:
 
 * Query head ``h`` uses KV head ``h // (H // G)`` (contiguous head groups).
 * ``delta`` is formed from the oracle's own exact output.

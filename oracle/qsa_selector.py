@@ -13,7 +13,7 @@ incomplete causal tail and the packed sequence's token origin; and the
 four-slot route group is one distinct complete block or the consecutive causal
 tail padded with -1, and blocks restart at each packed document origin.
 
-Readings where the pages leave a step open (also listed in the design doc):
+Readings where the pages leave a step open:
 
 * Query t sits at key position ``pos[t]`` of a sequence whose first token is
   ``tok_base[t]`` and whose first compressed block is ``blk_base[t]``; its own
