@@ -17,8 +17,10 @@
 // i.e. 256 (query, head) rows of qi.  It loops over 128-block tiles of kbar
 // covering the tile's candidates:  D[128 blocks][256 rows] = kbar_tile .
 // qi_tile^T with K = Di = 128, BF16 operands staged by TMA in 128B-swizzled
-// shared memory (K-major), FP32 accumulators in tensor memory, double-buffered
-// so that the MMA of block tile i + 1 runs under the epilogue of tile i.  The
+// shared memory (K-major; kbar tiles up to four ahead, a stage refilled as soon
+// as the MMA that read it has completed), FP32 accumulators in tensor memory,
+// double-buffered so that the MMA of block tile i + 1 runs under the epilogue
+// of tile i.  The
 // epilogue thread of TMEM lane r (block g0 + r) reads its 256 columns, sums
 // relu over each query's Hi heads and writes the scaled score.
 //
@@ -40,9 +42,13 @@ constexpr int kSelBlk = 128;       // compressed blocks per tile: the MMA M
 constexpr int kSelThreads = 128;   // 4 warps: one TMEM lane quarter each
 constexpr int kQiBytes = kSelRows * kSelDi * 2;   // 64 KB: two [256][64] SW128 K-blocks
 constexpr int kKbBytes = kSelBlk * kSelDi * 2;    // 32 KB: two [128][64] SW128 K-blocks
-constexpr int kSelOffKb = kQiBytes;               // two kbar stages
-constexpr int kSelOffBar = kSelOffKb + 2 * kKbBytes;
-constexpr int kSelSmem = kSelOffBar + 64 + 1024;  // + barriers, TMEM address, 1 KB alignment slack
+constexpr int kSelKbStages = 4;                   // kbar tiles loaded ahead of their MMA
+constexpr int kSelOffKb = kQiBytes;
+constexpr int kSelOffBar = kSelOffKb + kSelKbStages * kKbBytes;
+// barriers: qi, kSelKbStages kbar stages, 2 accumulators; then the TMEM address
+constexpr int kSelBarQ = 0, kSelBarK0 = 8, kSelBarM0 = kSelBarK0 + 8 * kSelKbStages, kSelTmemSlot = kSelBarM0 + 16;
+constexpr int kSelSmem = kSelOffBar + kSelTmemSlot + 8 + 1024;  // + 1 KB alignment slack
+static_assert(kSelSmem <= 232448, "shared memory per block");
 constexpr uint32_t kSelSpin = 1u << 24;
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -131,8 +137,9 @@ selector_scores_kernel(const __grid_constant__ CUtensorMap qi_map, const __grid_
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int Q = kSelRows / Hi;                 // queries per CTA
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * Q;
-  const uint32_t bar_q = sb + kSelOffBar, bar_k0 = bar_q + 8, bar_m0 = bar_q + 24;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSelOffBar + 40);
+  const uint32_t bar_q = sb + kSelOffBar + kSelBarQ, bar_k0 = sb + kSelOffBar + kSelBarK0,
+                 bar_m0 = sb + kSelOffBar + kSelBarM0;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSelOffBar + kSelTmemSlot);
 
   // the tile's global candidate blocks: union over its queries of [blk_base, blk_base + own)
   int64_t g_lo = INT64_MAX, g_hi = 0;
@@ -151,8 +158,7 @@ selector_scores_kernel(const __grid_constant__ CUtensorMap qi_map, const __grid_
 
   if (tid == 0) {
     mbar_init(bar_q, 1);
-    mbar_init(bar_k0, 1);
-    mbar_init(bar_k0 + 8, 1);
+    for (int j = 0; j < kSelKbStages; ++j) mbar_init(bar_k0 + 8 * j, 1);
     mbar_init(bar_m0, 1);
     mbar_init(bar_m0 + 8, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -168,9 +174,9 @@ selector_scores_kernel(const __grid_constant__ CUtensorMap qi_map, const __grid_
   const uint32_t tmem = *tmem_slot;
 
   const int qi_row0 = static_cast<int>(t0 * Hi);
-  auto load_kb = [&](int i) {  // kbar tile i -> stage i & 1
-    const uint32_t bar = bar_k0 + 8 * (i & 1);
-    const uint32_t dst = sb + kSelOffKb + (i & 1) * kKbBytes;
+  auto load_kb = [&](int i) {  // kbar tile i -> stage i % kSelKbStages
+    const uint32_t bar = bar_k0 + 8 * (i % kSelKbStages);
+    const uint32_t dst = sb + kSelOffKb + (i % kSelKbStages) * kKbBytes;
     mbar_expect_tx(bar, kKbBytes);
     const int g = static_cast<int>(g_lo + static_cast<int64_t>(i) * kSelBlk);
     tma_load_2d(dst, &kb_map, 0, g, bar);
@@ -178,7 +184,7 @@ selector_scores_kernel(const __grid_constant__ CUtensorMap qi_map, const __grid_
   };
   auto issue_mma = [&](int i) {  // D[i & 1] = kbar tile i . qi tile^T
     const uint32_t d = tmem + (i & 1) * kSelRows;
-    const uint32_t a0 = sb + kSelOffKb + (i & 1) * kKbBytes, b0 = sb;
+    const uint32_t a0 = sb + kSelOffKb + (i % kSelKbStages) * kKbBytes, b0 = sb;
 #pragma unroll
     for (int kk = 0; kk < kSelDi / 16; ++kk) {
       // k-step kk: K-block kk / 4, byte offset 32 (kk % 4) inside the 128-byte row
@@ -194,8 +200,7 @@ selector_scores_kernel(const __grid_constant__ CUtensorMap qi_map, const __grid_
     mbar_expect_tx(bar_q, kQiBytes);
     tma_load_2d(sb, &qi_map, 0, qi_row0, bar_q);
     tma_load_2d(sb + kQiBytes / 2, &qi_map, 64, qi_row0, bar_q);
-    load_kb(0);
-    if (n_tiles > 1) load_kb(1);
+    for (int j = 0; j < min(n_tiles, kSelKbStages); ++j) load_kb(j);
     ok = mbar_wait(bar_q, 0) && mbar_wait(bar_k0, 0);
     if (ok) {
       asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
@@ -208,7 +213,7 @@ selector_scores_kernel(const __grid_constant__ CUtensorMap qi_map, const __grid_
   for (; ok && i < n_tiles; ++i) {
     // issue the next tile's MMA before this tile's epilogue
     if (tid == 0 && i + 1 < n_tiles) {
-      ok = mbar_wait(bar_k0 + 8 * ((i + 1) & 1), ((i + 1) >> 1) & 1);
+      ok = mbar_wait(bar_k0 + 8 * ((i + 1) % kSelKbStages), ((i + 1) / kSelKbStages) & 1);
       if (ok) {
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
         issue_mma(i + 1);
@@ -217,6 +222,8 @@ selector_scores_kernel(const __grid_constant__ CUtensorMap qi_map, const __grid_
     const bool got = mbar_wait(bar_m0 + 8 * (i & 1), (i >> 1) & 1);
     ok = __syncthreads_and(ok && got) != 0;
     if (!ok) break;
+    // MMA i has read its kbar stage: refill it kSelKbStages tiles ahead, under the epilogue
+    if (tid == 0 && i + kSelKbStages < n_tiles) load_kb(i + kSelKbStages);
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
     // epilogue: thread = TMEM lane = block row r of the tile
     const int r = warp * 32 + lane;
@@ -237,18 +244,15 @@ selector_scores_kernel(const __grid_constant__ CUtensorMap qi_map, const __grid_
       }
     }
     asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-    __syncthreads();  // accumulator i & 1 and kbar stage i & 1 are free again
-    if (tid == 0 && i + 2 < n_tiles) load_kb(i + 2);
+    __syncthreads();  // accumulator i & 1 is free again
   }
   if (!ok) {
     if (tid == 0 && status) atomicExch(status, 2);
     // wait (bounded) for this CTA's copies and MMAs still in flight
     if (tid == 0) {
       mbar_wait(bar_q, 0);
-      for (int j = i; j < min(n_tiles, i + 2); ++j) {
-        mbar_wait(bar_k0 + 8 * (j & 1), (j >> 1) & 1);
-        mbar_wait(bar_m0 + 8 * (j & 1), (j >> 1) & 1);
-      }
+      for (int j = i; j < min(n_tiles, i + kSelKbStages); ++j) mbar_wait(bar_k0 + 8 * (j % kSelKbStages), (j / kSelKbStages) & 1);
+      for (int j = i; j < min(n_tiles, i + 2); ++j) mbar_wait(bar_m0 + 8 * (j & 1), (j >> 1) & 1);
     }
     __syncthreads();
   }
