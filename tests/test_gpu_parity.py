@@ -297,8 +297,9 @@ def test_edge_cases(case):
 # determinism, non-finite isolation, error statuses
 # ---------------------------------------------------------------------------
 
-def test_backward_is_bitwise_deterministic():
-    wl = W.CONFIGS[3]
+@pytest.mark.parametrize("number", [3, 4])  # thd16k: 1 KV group, 4 dK/dV phases; seq32k: 2 groups, 8 phases
+def test_backward_is_bitwise_deterministic(number):
+    wl = W.CONFIGS[number]
     routes, q, k, v, do = inputs(wl)
     r, qd, kd, vd, dod = to_dev(routes, q, k, v, do)
     out, lse = qsa.forward(qd, kd, vd, r, wl.scale)
