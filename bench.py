@@ -35,7 +35,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = 4
+WORKLOAD = "seq32k"
 METRIC = "QSA fwd+bwd selected pairs/s and TFLOP/s at T=32K, 512 sel/query; % roofline"
 UNIT = "pairs/s"
 FWD_FLOPS_PER_PAIR_HEAD = 4 * 256      # QK^T + PV
@@ -183,7 +183,7 @@ def run_reference(args):
     if rank != 0:
         return
     from token_indexed_sparse_b200 import workloads as W
-    wl = W.CONFIGS[WORKLOAD]
+    wl = W.WORKLOADS[WORKLOAD]
     routes, tens = oracle_inputs(wl)
     rng = np.random.default_rng(1)
     rows_per_step = args.reference_rows
@@ -292,7 +292,7 @@ def run_ours(args):
         import datetime
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
 
-    wl = W.CONFIGS[args.workload]
+    wl = W.WORKLOADS[args.workload]
     if args.scale_T:
         wl = wl.scaled(args.scale_T)
     routes_np = np.array(W.make_routes(wl), dtype=np.int32)
@@ -456,7 +456,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
                     help="time the device-resident steps only and print the stage breakdown (profiling runs)")
-    ap.add_argument("--workload", type=int, default=WORKLOAD, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", default=WORKLOAD, choices=["tiny", "seq4k", "thd16k", "seq32k", "cp128k"])
     ap.add_argument("--scale-T", type=int, default=0,
                     help="run the workload's recipe at this many query rows (profiling of smaller cases)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

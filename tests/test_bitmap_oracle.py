@@ -57,8 +57,7 @@ def test_round_trip_of_causal_block_routes():
     # routes made of whole causal four-token blocks plus the causal tail, as the
     # workload recipe draws them: the bitmap of their blocks with bounds
     # [0, t] allows exactly the routed keys
-    for num in (1, 2):
-        wl = W.CONFIGS[num] if num == 1 else W.CONFIGS[num].scaled(256)
+    for wl in (W.WORKLOADS["tiny"], W.WORKLOADS["seq4k"].scaled(256)):
         routes = W.make_routes(wl)
         T, T_kv = routes.shape[0], wl.T_kv
         sel = _block_routes_to_bitmap(routes, T_kv)

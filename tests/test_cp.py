@@ -41,7 +41,7 @@ def _free_port():
 
 
 def _case():
-    wl = W.CONFIGS[2].scaled(256)          # T = T_kv = 256, 12Q/1KV
+    wl = W.WORKLOADS["seq4k"].scaled(256)          # T = T_kv = 256, 12Q/1KV
     routes = np.array(W.make_routes(wl))
     q, k, v, do = (x.double() for x in W.make_tensors(wl))
     return wl, routes, q, k, v, do

@@ -112,7 +112,7 @@ def test_bitmap_attention_matches_dense_oracle():
 def test_full_size_bitmap_of_seq32k_routes():
     # the seq32k routes' blocks as a single-sequence bitmap (T x NB = 32768 x
     # 8192 bytes): the adapter must return exactly each row's unique valid keys
-    wl = W.CONFIGS[4]
+    wl = W.WORKLOADS["seq32k"]
     r = torch.from_numpy(np.array(W.make_routes(wl))).to(DEV)
     T, T_kv = wl.T, wl.T_kv
     NB = T_kv // 4

@@ -23,16 +23,16 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def _inputs(num, T):
-    wl = W.CONFIGS[num].scaled(T)
+def _inputs(name, T):
+    wl = W.WORKLOADS[name].scaled(T)
     routes = torch.from_numpy(np.array(W.make_routes(wl))).to(DEV)
     q, k, v, do = (x.to(DEV) for x in W.make_tensors(wl))
     return wl, routes, q, k, v, do
 
 
-@pytest.mark.parametrize("num,T", [(3, 1024), (5, 256)])
-def test_fp32_kv_backward(num, T):
-    wl, routes, q, k, v, do = _inputs(num, T)
+@pytest.mark.parametrize("name,T", [("thd16k", 1024), ("cp128k", 256)])
+def test_fp32_kv_backward(name, T):
+    wl, routes, q, k, v, do = _inputs(name, T)
     out, lse = qsa.forward(q, k, v, routes, wl.scale)
     dq, dk, dv = qsa.backward(do, q, k, v, out, lse, routes, wl.scale)
     dq32, dk32, dv32 = qsa.backward(do, q, k, v, out, lse, routes, wl.scale, kv_fp32=True)
@@ -55,7 +55,7 @@ def test_cp_single_rank_reproduces_plain_calls():
     dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
                             device_id=torch.device(DEV))
     try:
-        wl, routes, q, k, v, do = _inputs(5, 512)
+        wl, routes, q, k, v, do = _inputs("cp128k", 512)
         out, lse = qsa.forward(q, k, v, routes, wl.scale)
         dq, dk, dv = qsa.backward(do, q, k, v, out, lse, routes, wl.scale)
         c_out, c_lse = cp.cp_forward(q, k, v, routes, wl.scale)

@@ -80,12 +80,12 @@ def inputs(wl):
 # exhaustive parity on every workload recipe at sizes the dense oracle finishes
 # ---------------------------------------------------------------------------
 
-SMALL = {1: None, 2: 512, 3: 1024, 4: 768, 5: 256}
+SMALL = {"tiny": None, "seq4k": 512, "thd16k": 1024, "seq32k": 768, "cp128k": 256}
 
 
-@pytest.mark.parametrize("number", [1, 2, 3, 4, 5])
-def test_parity_dense_oracle(number):
-    wl = W.CONFIGS[number] if SMALL[number] is None else W.CONFIGS[number].scaled(SMALL[number])
+@pytest.mark.parametrize("name", list(SMALL))
+def test_parity_dense_oracle(name):
+    wl = W.WORKLOADS[name] if SMALL[name] is None else W.WORKLOADS[name].scaled(SMALL[name])
     routes, q, k, v, do = inputs(wl)
     res = run_gpu(q, k, v, do, routes, wl.scale)
     ref_out, ref_lse = oracle.forward_dense(f64(q), f64(k), f64(v), routes, wl.scale)
@@ -103,12 +103,12 @@ def test_parity_dense_oracle(number):
 # full workload sizes: sampled rows and keys computed one by one by the oracle
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("number", [2, 3, 4, 5])
-def test_parity_full_size_sampled(number):
-    wl = W.CONFIGS[number]
+@pytest.mark.parametrize("name", ["seq4k", "thd16k", "seq32k", "cp128k"])
+def test_parity_full_size_sampled(name):
+    wl = W.WORKLOADS[name]
     routes, q, k, v, do = inputs(wl)
     out, lse, dq, dk, dv = run_gpu(q, k, v, do, routes, wl.scale)
-    rng = np.random.default_rng(number)
+    rng = np.random.default_rng(wl.seed - 1000)
     counts = oracle.route_rows_csr(routes, wl.T_kv)[0]
     rows = np.unique(np.concatenate([rng.choice(wl.T, 48, replace=False),
                                      [int(np.argmax(counts)), wl.T - 1, 0]]))
@@ -159,9 +159,9 @@ def _check_plan(routes, T_kv):
     np.testing.assert_array_equal((ent >> 4) & 0x0FFFFFFF, i0)
 
 
-@pytest.mark.parametrize("number,T", [(1, None), (2, 512), (3, 1024), (4, 768), (5, 256)])
-def test_route_plan_bitexact(number, T):
-    wl = W.CONFIGS[number] if T is None else W.CONFIGS[number].scaled(T)
+@pytest.mark.parametrize("name,T", list(SMALL.items()))
+def test_route_plan_bitexact(name, T):
+    wl = W.WORKLOADS[name] if T is None else W.WORKLOADS[name].scaled(T)
     _check_plan(W.make_routes(wl), wl.T_kv)
 
 
@@ -197,9 +197,9 @@ def _check_tile_plan(routes, T_kv):
     np.testing.assert_array_equal((ent & 0x7F) + 1, n)
 
 
-@pytest.mark.parametrize("number,T", [(1, None), (2, 512), (3, 1024), (4, 768), (5, 256)])
-def test_tile_plan_bitexact(number, T):
-    wl = W.CONFIGS[number] if T is None else W.CONFIGS[number].scaled(T)
+@pytest.mark.parametrize("name,T", list(SMALL.items()))
+def test_tile_plan_bitexact(name, T):
+    wl = W.WORKLOADS[name] if T is None else W.WORKLOADS[name].scaled(T)
     _check_tile_plan(W.make_routes(wl), wl.T_kv)
 
 
@@ -297,9 +297,9 @@ def test_edge_cases(case):
 # determinism, non-finite isolation, error statuses
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("number", [3, 4])  # thd16k: 1 KV group, 4 dK/dV phases; seq32k: 2 groups, 8 phases
-def test_backward_is_bitwise_deterministic(number):
-    wl = W.CONFIGS[number]
+@pytest.mark.parametrize("name", ["thd16k", "seq32k"])  # 1 KV group, 4 dK/dV phases; 2 groups, 8 phases
+def test_backward_is_bitwise_deterministic(name):
+    wl = W.WORKLOADS[name]
     routes, q, k, v, do = inputs(wl)
     r, qd, kd, vd, dod = to_dev(routes, q, k, v, do)
     out, lse = qsa.forward(qd, kd, vd, r, wl.scale)
@@ -317,7 +317,7 @@ def test_backward_is_bitwise_deterministic(number):
 
 
 def test_unselected_nonfinite_kv_never_read():
-    wl = W.CONFIGS[2].scaled(512)
+    wl = W.WORKLOADS["seq4k"].scaled(512)
     routes, q, k, v, do = inputs(wl)
     rng = np.random.default_rng(2)
     unused = np.sort(rng.choice(wl.T_kv, 64, replace=False))

@@ -260,11 +260,12 @@ def test_backward_matches_finite_differences():
 # row-gather form == dense form; key-sampled backward == full backward
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("number,T", [(1, 256), (2, 256), (3, 384), (4, 192), (5, 128)])
-def test_row_form_matches_dense_form(number, T):
-    wl = W.CONFIGS[number].scaled(T) if T != W.CONFIGS[number].T else W.CONFIGS[number]
+@pytest.mark.parametrize("name,T", [("tiny", 256), ("seq4k", 256), ("thd16k", 384), ("seq32k", 192),
+                                    ("cp128k", 128)])
+def test_row_form_matches_dense_form(name, T):
+    wl = W.WORKLOADS[name].scaled(T) if T != W.WORKLOADS[name].T else W.WORKLOADS[name]
     routes = W.make_routes(wl)
-    rng = np.random.default_rng(number)
+    rng = np.random.default_rng(wl.seed - 1000)
     q, do = _rand(rng, wl.T, wl.H, 256), _rand(rng, wl.T, wl.H, 256)
     k, v = _rand(rng, wl.T_kv, wl.G, 256), _rand(rng, wl.T_kv, wl.G, 256)
     out_d, lse_d = oracle.forward_dense(q, k, v, routes, wl.scale)

@@ -12,9 +12,9 @@ def _doc_start(wl, pos):
     return starts[np.searchsorted(starts, pos, side="right") - 1], starts
 
 
-@pytest.mark.parametrize("number", [1, 2, 3, 4, 5])
-def test_route_structure(number):
-    wl = W.CONFIGS[number]
+@pytest.mark.parametrize("name", list(W.WORKLOADS))
+def test_route_structure(name):
+    wl = W.WORKLOADS[name]
     r = W.make_routes(wl)
     assert r.shape == (wl.T, wl.W) and r.dtype == np.int32
     assert W.make_routes(wl) is r                       # cached, deterministic
@@ -54,7 +54,7 @@ def test_route_structure(number):
                 v = grp[grp >= 0]
                 assert len(v) >= 1 and np.all(np.diff(v) == 1) and (v[0] - doc) % 4 == 0
                 assert np.all(grp[len(v):] == -1)
-    if number == 4:
+    if name == "seq32k":
         # half of a late row's blocks lie in the most recent 512 blocks
         t = wl.T - 1
         uniq = np.unique(r[t][r[t] >= 0])
@@ -64,7 +64,7 @@ def test_route_structure(number):
 
 def test_tensors_are_seeded_bf16():
     import torch
-    wl = W.CONFIGS[1]
+    wl = W.WORKLOADS["tiny"]
     q, k, v, do = W.make_tensors(wl)
     assert q.dtype == torch.bfloat16 and q.shape == (256, 12, 256)
     assert k.shape == v.shape == (256, 1, 256) and do.shape == q.shape

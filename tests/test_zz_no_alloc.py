@@ -62,7 +62,7 @@ def _compare(out, lse, ref_out, ref_lse):
 
 def test_noalloc_forward_matches_workspace_forward_twice():
     lib = _lib()
-    for wl in (W.CONFIGS[2].scaled(1024), W.CONFIGS[1]):
+    for wl in (W.WORKLOADS["seq4k"].scaled(1024), W.WORKLOADS["tiny"]):
         q, k, v, routes = _inputs(wl)
         assert qsa.forward_workspace_size(wl.T, wl.T_kv, wl.H, wl.G, wl.W) <= QSA_NOALLOC_SCRATCH_BYTES
         ref_out, ref_lse = qsa.forward(q, k, v, routes, wl.scale)

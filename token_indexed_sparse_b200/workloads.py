@@ -10,26 +10,26 @@ one four-token block, either complete or the query's own causal tail padded
 with -1, blocks numbered from each packed document's origin, and -1 rows for
 padding queries.  Block choices per configuration:
 
-1. ``tiny``   T=256, 12Q/1KV, W=64: min(16, visible) blocks uniform without
-   replacement over the visible blocks (the tail may or may not be drawn);
-   the last 8 rows all -1.
-2. ``seq4k``  T=4096, 12Q/1KV, W=256: 64 distinct blocks, the own (tail) block
-   always, the rest uniform over the earlier visible blocks.
-3. ``thd16k`` T=16384 packed as 8 documents (7 distinct sorted cut points
-   uniform in [1, T-1], redrawn while a document is shorter than 4 tokens),
-   W=512: 128 blocks within the query's document, own block always; a seeded
-   3% of rows all -1.
-4. ``seq32k`` T=32768, 24Q/2KV (routes shared by both groups), W=564: 128
-   distinct blocks, 64 from the 512 most recent blocks (own block always) and
-   64 uniform over the older visible blocks; where a pool is short the other
-   pool makes up the count.  Then ceil(10%) of each row's valid IDs are
-   appended again as duplicates and the row is shuffled.
-5. ``cp128k`` 8192 local queries at global positions 122880..131071 against
-   131072 K/V rows, 12Q/1KV, W=2048: 512 distinct blocks, own block always,
-   the others without replacement with weight d^-1.1 in the block distance
-   d >= 1; a seeded 5% of rows all -1.
+* ``tiny``   T=256, 12Q/1KV, W=64: min(16, visible) blocks uniform without
+  replacement over the visible blocks (the tail may or may not be drawn);
+  the last 8 rows all -1.
+* ``seq4k``  T=4096, 12Q/1KV, W=256: 64 distinct blocks, the own (tail) block
+  always, the rest uniform over the earlier visible blocks.
+* ``thd16k`` T=16384 packed as 8 documents (7 distinct sorted cut points
+  uniform in [1, T-1], redrawn while a document is shorter than 4 tokens),
+  W=512: 128 blocks within the query's document, own block always; a seeded
+  3% of rows all -1.
+* ``seq32k`` T=32768, 24Q/2KV (routes shared by both groups), W=564: 128
+  distinct blocks, 64 from the 512 most recent blocks (own block always) and
+  64 uniform over the older visible blocks; where a pool is short the other
+  pool makes up the count.  Then ceil(10%) of each row's valid IDs are
+  appended again as duplicates and the row is shuffled.
+* ``cp128k`` 8192 local queries at global positions 122880..131071 against
+  131072 K/V rows, 12Q/1KV, W=2048: 512 distinct blocks, own block always,
+  the others without replacement with weight d^-1.1 in the block distance
+  d >= 1; a seeded 5% of rows all -1.
 
-Seeds are 1000 + config number.  Routes come from numpy's PCG64; q, k, v and
+Seeds are 1001 to 1005, in the order above.  Routes come from numpy's PCG64; q, k, v and
 grad_out are N(0, 1) float32 draws from a seeded torch CPU generator, rounded
 once to BF16 (the BF16 values are what both sides consume).
 """
@@ -48,7 +48,6 @@ HEAD_DIM = 256
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    number: int
     T: int
     T_kv: int
     H: int
@@ -81,15 +80,15 @@ class Workload:
             pad_tail=min(self.pad_tail, T // 4))
 
 
-CONFIGS = {
-    1: Workload("tiny", 1, 256, 256, 12, 1, 64, 16, "uniform", pad_tail=8, seed=1001),
-    2: Workload("seq4k", 2, 4096, 4096, 12, 1, 256, 64, "own_uniform", seed=1002),
-    3: Workload("thd16k", 3, 16384, 16384, 12, 1, 512, 128, "own_uniform", n_docs=8,
-                pad_frac=0.03, seed=1003),
-    4: Workload("seq32k", 4, 32768, 32768, 24, 2, 564, 128, "near_far", dup_frac=0.10,
-                seed=1004),
-    5: Workload("cp128k", 5, 8192, 131072, 12, 1, 2048, 512, "zipf", q_offset=122880,
-                pad_frac=0.05, seed=1005),
+WORKLOADS = {
+    "tiny": Workload("tiny", 256, 256, 12, 1, 64, 16, "uniform", pad_tail=8, seed=1001),
+    "seq4k": Workload("seq4k", 4096, 4096, 12, 1, 256, 64, "own_uniform", seed=1002),
+    "thd16k": Workload("thd16k", 16384, 16384, 12, 1, 512, 128, "own_uniform", n_docs=8,
+                         pad_frac=0.03, seed=1003),
+    "seq32k": Workload("seq32k", 32768, 32768, 24, 2, 564, 128, "near_far", dup_frac=0.10,
+                         seed=1004),
+    "cp128k": Workload("cp128k", 8192, 131072, 12, 1, 2048, 512, "zipf", q_offset=122880,
+                         pad_frac=0.05, seed=1005),
 }
 
 
