@@ -183,7 +183,9 @@ def run_reference(args):
     if rank != 0:
         return
     from token_indexed_sparse_b200 import workloads as W
-    wl = W.WORKLOADS[WORKLOAD]
+    wl = W.WORKLOADS[args.workload]          # the same workload as the CUDA arm
+    if args.scale_T:
+        wl = wl.scaled(args.scale_T)
     routes, tens = oracle_inputs(wl)
     rng = np.random.default_rng(1)
     rows_per_step = args.reference_rows
