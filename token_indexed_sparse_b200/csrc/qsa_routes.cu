@@ -4,11 +4,15 @@
 // duplicates collapse ("fa4_qsa" page, `_preprocess`; "flex_qsa" page,
 // `_routes_to_membership`).  These kernels turn the raw [T, n_sel] routes into
 //   * per-row ascending de-duplicated lists (row_cnt, row_cols), consumed by the
-//     per-query forward and dQ kernels, and
-//   * the key->query transpose at the granularity of aligned key quads
-//     (quad_ptr, quad_ent), each list in ascending query order, consumed by the
-//     per-quad dK/dV kernel.  A fixed list order makes the dK/dV summation order,
-//     and so its result bits, independent of scheduling.
+//     per-query forward and dQ kernels,
+//   * the key->query transpose over aligned 128-key tiles (tile_ptr, tile_ent:
+//     one entry per (row, tile) naming the row's run of keys in the tile), each
+//     list in ascending query order with its query-phase starts, and the
+//     per-phase work lists the dK/dV kernel claims its units from, and
+//   * the same transpose over aligned key quads with 4-bit owner masks
+//     (quad_ptr, quad_ent), exposed by qsa_route_plan.
+// A fixed list order makes the dK/dV summation order, and so its result bits,
+// independent of scheduling.
 #include <climits>
 
 #include "qsa_device.cuh"
