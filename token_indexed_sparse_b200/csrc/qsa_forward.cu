@@ -1,4 +1,5 @@
-// QSA forward: persistent, one CTA (8 warps) per SM.
+// QSA forward: persistent, four CTAs of two warps per SM (the shape set at the
+// launcher below).
 //
 // Computes, for the 12 query heads of every (query token t, KV group g), the
 // softmax attention of the cuDNN-Frontend "Query Sparse Attention (QSA)" page
@@ -6,15 +7,17 @@
 // PV, FP32 output cast to BF16, natural-log LSE; empty rows give zero output and
 // -inf LSE) over the row's de-duplicated route set R_t.
 //
-// Pipeline (qsa_pipe.cuh): the CTA's items are cut into 64-key chunks that flow
-// through a 3-stage ring of swizzled K / V tiles (plus the item's 12 Q rows on
-// its first chunk), gathered with 16-byte cp.async copies two chunks ahead of
-// the compute.  Rows past the end of R_t are zero-filled, so unselected K/V
+// Pipeline (qsa_pipe.cuh): the CTA's items are cut into chunks of 8 keys per
+// warp (16 at the launch shape) that flow through a ring of swizzled K / V tiles
+// (plus the item's 12 Q rows on its first chunk), gathered with 16-byte
+// cp.async copies STAGES - 1 chunks ahead of the compute (one at the launch
+// shape).  Rows past the end of R_t are zero-filled, so unselected K/V
 // values never reach an output.  Per chunk, warp w forms S = Q K^T for keys
 // 8w..8w+7 (mma.sync m16n8k16 BF16, FP32 accumulate, Q fragments held in
 // registers for the whole item), the chunk's row maxima are combined across the
 // warps in shared memory, P = exp2(S*scale*log2e - m) is written as BF16, and
-// warp w accumulates O[:, 32w:32w+32] += P V with running-max rescaling.
+// warp w accumulates O[:, DPW w : DPW (w + 1)] += P V (DPW = 256 / warps, 128 at
+// the launch shape) with running-max rescaling.
 #include "qsa_internal.h"
 #include "qsa_pipe.cuh"
 
