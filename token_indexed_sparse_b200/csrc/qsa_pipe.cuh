@@ -17,10 +17,7 @@
 
 namespace qsa {
 
-constexpr int kPipeKeys = 64;
-constexpr int kPipeThreads = 256;  // 8 warps: every warp computes and gathers
-
-template <int KEYS = kPipeKeys>
+template <int KEYS>
 __device__ __forceinline__ int pipe_chunks(int cnt) { return cnt > 0 ? (cnt + KEYS - 1) / KEYS : 1; }
 
 // The item index is tracked as (t, g) and advanced by the grid stride without
@@ -43,7 +40,7 @@ __device__ __forceinline__ int pipe_cnt_next(const Cursor& c, const int32_t* row
   return c.it + gridDim.x < n_items ? __ldg(row_cnt + t_next) : 0;
 }
 
-template <int KEYS = kPipeKeys>
+template <int KEYS>
 __device__ __forceinline__ void cursor_init(Cursor& c, const int32_t* row_cnt, int64_t n_items, int G) {
   c.it = blockIdx.x;
   c.t = static_cast<int>(blockIdx.x) / G;
@@ -56,7 +53,7 @@ __device__ __forceinline__ void cursor_init(Cursor& c, const int32_t* row_cnt, i
   c.nch = pipe_chunks<KEYS>(c.cnt);
 }
 
-template <int KEYS = kPipeKeys>
+template <int KEYS>
 __device__ __forceinline__ void cursor_next(Cursor& c, const int32_t* row_cnt, int64_t n_items, int G) {
   if (++c.ch == c.nch) {
     c.it += gridDim.x;
@@ -74,7 +71,7 @@ __device__ __forceinline__ void cursor_next(Cursor& c, const int32_t* row_cnt, i
 }
 
 // Keys in the cursor's current chunk (0 for an empty row or past the end).
-template <int KEYS = kPipeKeys>
+template <int KEYS>
 __device__ __forceinline__ int cursor_nk(const Cursor& c, int64_t n_items) {
   if (c.it >= n_items || c.cnt <= 0) return 0;
   return min(KEYS, c.cnt - c.ch * KEYS);
@@ -83,7 +80,7 @@ __device__ __forceinline__ int cursor_nk(const Cursor& c, int64_t n_items) {
 // Key IDs of the rows this thread gathers in the cursor's current chunk: rows
 // 8 * warp + j, j = 0..7 (0 for rows past the end of the chunk, whose copies are
 // then zero-fills).  Every lane of a warp loads the same eight IDs.
-template <int KEYS = kPipeKeys>
+template <int KEYS>
 __device__ __forceinline__ void cursor_keys(int32_t (&key)[8], const Cursor& c, int64_t n_items, int G,
                                             const int32_t* row_cols, int n_sel) {
   const int nk = cursor_nk<KEYS>(c, n_items);
