@@ -72,6 +72,13 @@ FWD_STAGES = ["fwd_route_rows", "fwd_attention"]
 BWD_STAGES = ["bwd_route_rows", "bwd_tile_scan", "bwd_tile_fill", "bwd_tile_sort", "bwd_dq", "bwd_dkdv"]
 
 
+def pass_ms(stage_ms):
+    """Forward, backward and their sum (ms per step) from the per-stage means."""
+    fwd = sum(stage_ms.get(n, 0.0) for n in FWD_STAGES)
+    bwd = sum(stage_ms.get(n, 0.0) for n in BWD_STAGES)
+    return {"forward": fwd, "backward": bwd, "total": fwd + bwd}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -431,6 +438,7 @@ def run_ours(args):
                           "frac": step_tflops / peaks["bf16_tflops_sustained"],
                           "peak": peaks["bf16_tflops_sustained"], "peak_source": peaks["source"]},
         "stage_ms": avg,
+        "pass_ms": pass_ms(avg),
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},

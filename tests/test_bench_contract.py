@@ -40,3 +40,14 @@ def test_reference_line_has_the_contract_keys():
 
 def test_only_rank_zero_prints():
     assert _run({"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+def test_pass_ms_sums_the_stages():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_mod", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    stages = {n: float(i + 1) for i, n in enumerate(bench.FWD_STAGES + bench.BWD_STAGES)}
+    got = bench.pass_ms(stages)
+    assert got == {"forward": 3.0, "backward": 3.0 + 4 + 5 + 6 + 7 + 8, "total": 36.0}
+    assert bench.pass_ms({}) == {"forward": 0.0, "backward": 0.0, "total": 0.0}
