@@ -146,3 +146,28 @@ def test_no_cpu_fallback_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(qsa, "_LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         qsa.library()
+
+
+def test_binding_refuses_output_buffers_the_kernels_would_overrun():
+    # caller-provided outputs are written in place through their pointers: the
+    # binding checks them before any call (CPU tensors stand in for the device)
+    import torch
+    from token_indexed_sparse_b200 import qsa
+    dev = torch.device("cpu")
+    ok = torch.empty(4, 12, 256, dtype=torch.bfloat16)
+    assert qsa._out(ok, (4, 12, 256), torch.bfloat16, dev, "out") is ok
+    with pytest.raises(ValueError, match="shape"):
+        qsa._out(torch.empty(4, 12, 255, dtype=torch.bfloat16), (4, 12, 256), torch.bfloat16, dev, "out")
+    with pytest.raises(TypeError):
+        qsa._out(torch.empty(4, 12, 256, dtype=torch.float32), (4, 12, 256), torch.bfloat16, dev, "out")
+    with pytest.raises(ValueError, match="contiguous"):
+        qsa._out(torch.empty(12, 4, 256, dtype=torch.bfloat16).transpose(0, 1), (4, 12, 256), torch.bfloat16, dev,
+                 "out")
+    with pytest.raises(ValueError, match="on"):
+        qsa._out(ok, (4, 12, 256), torch.bfloat16, torch.device("meta"), "out")
+    ws = torch.empty(1024, dtype=torch.uint8)
+    assert qsa._workspace(1024, dev, ws) is ws
+    with pytest.raises(ValueError):
+        qsa._workspace(1024, dev, torch.empty(256, dtype=torch.float32))
+    with pytest.raises(ValueError):
+        qsa._workspace(1024, dev, torch.empty(2048, dtype=torch.uint8)[::2])

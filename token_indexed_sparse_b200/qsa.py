@@ -102,6 +102,21 @@ def _prep(x: torch.Tensor, dtype, name: str) -> torch.Tensor:
     return x.contiguous()
 
 
+def _out(t: torch.Tensor, shape, dtype, device, name: str) -> torch.Tensor:
+    """A caller-provided output buffer.  The kernels write it in place through its
+    pointer, so it must be exactly the dense tensor they expect: anything else
+    is refused before the call (a strided or short buffer would be overrun)."""
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
 def _sizes(q, k, routes):
     if q.dim() != 3 or k.dim() != 3 or routes.dim() != 2:
         raise ValueError("expected q [T,H,256], k/v [T_kv,G,256], routes [T,n_sel]")
@@ -128,7 +143,9 @@ def launch_count(T, T_kv, H, G, n_sel, backward: bool) -> int:
 
 
 def _workspace(nbytes: int, device, given: torch.Tensor | None) -> torch.Tensor:
-    if given is not None:
+    if given is not None:  # a dense uint8 buffer: its element count is its size in bytes
+        if given.device != device or given.dtype != torch.uint8 or not given.is_contiguous():
+            raise ValueError(f"workspace must be a contiguous uint8 tensor on {device}")
         return given
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
@@ -157,10 +174,9 @@ def forward(q, k, v, routes, scale: float = 1.0 / 16.0, *, out=None, lse=None, w
     v = _prep(v, torch.bfloat16, "v")
     routes = _prep(routes, torch.int32, "routes")
     T, T_kv, H, G, n_sel = _sizes(q, k, routes)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty(T, H, dtype=torch.float32, device=q.device)
+    out = torch.empty_like(q) if out is None else _out(out, q.shape, torch.bfloat16, q.device, "out")
+    lse = (torch.empty(T, H, dtype=torch.float32, device=q.device) if lse is None
+           else _out(lse, (T, H), torch.float32, q.device, "lse"))
     ws_bytes = lib.qsa_forward_workspace_size(T, T_kv, H, G, n_sel)
     ws = _workspace(ws_bytes, q.device, workspace)
     ev, n_ev = _events(stage_events)
@@ -188,11 +204,11 @@ def backward(grad_out, q, k, v, out, lse, routes, scale: float = 1.0 / 16.0, *,
     routes = _prep(routes, torch.int32, "routes")
     T, T_kv, H, G, n_sel = _sizes(q, k, routes)
     kv_dtype = torch.float32 if kv_fp32 else torch.bfloat16
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty(k.shape, dtype=kv_dtype, device=k.device) if dk is None else dk
-    dv = torch.empty(v.shape, dtype=kv_dtype, device=v.device) if dv is None else dv
-    if dk.dtype != kv_dtype or dv.dtype != kv_dtype:
-        raise TypeError(f"dk / dv must be {kv_dtype}")
+    dq = torch.empty_like(q) if dq is None else _out(dq, q.shape, torch.bfloat16, q.device, "dq")
+    dk = (torch.empty(k.shape, dtype=kv_dtype, device=k.device) if dk is None
+          else _out(dk, k.shape, kv_dtype, k.device, "dk"))
+    dv = (torch.empty(v.shape, dtype=kv_dtype, device=v.device) if dv is None
+          else _out(dv, v.shape, kv_dtype, v.device, "dv"))
     ws_bytes = lib.qsa_backward_workspace_size(T, T_kv, H, G, n_sel)
     ws = _workspace(ws_bytes, q.device, workspace)
     if kv_fp32:
@@ -288,8 +304,13 @@ def selector_scores(qi, kbar, scale: float, pos=None, blk_base=None, tok_base=No
                                                            (tok_base, "tok_base")))
     if scores is None:
         scores = torch.full((T, NB), float("nan"), dtype=torch.float32, device=dev)
+    elif (scores.device != dev or scores.dtype != torch.float32 or scores.dim() != 2 or scores.shape[0] != T
+          or scores.shape[1] < NB or scores.stride(1) != 1):
+        raise ValueError(f"scores must be a float32 [{T}, >= {NB}] tensor on {dev} with unit column stride")
     if status is None:
         status = torch.zeros(1, dtype=torch.int32, device=dev)
+    elif status.device != dev or status.dtype != torch.int32 or status.numel() < 1 or not status.is_contiguous():
+        raise ValueError(f"status must be a contiguous int32 tensor on {dev}")
     st = lib.qsa_selector_scores(_ptr(qi), _ptr(kbar), T, NB, Hi, Di, scale, _ptr(pos), _ptr(blk_base),
                                  _ptr(tok_base), _ptr(scores), scores.stride(0), _ptr(status), _stream(dev))
     _check(st, "qsa_selector_scores")
