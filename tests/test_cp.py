@@ -1,4 +1,4 @@
-"""Context-parallel plumbing on CPU processes (gloo, world size 2).
+"""Context-parallel plumbing on CPU processes (gloo, world sizes 2 and 4).
 
 The CP path (``token_indexed_sparse_b200.cp``) gathers K/V, runs the local
 attention of each rank's query rows and reduce-scatters the dK/dV partials.
@@ -75,9 +75,9 @@ def _rank_main(rank, world, port, out_dir):
         dist.destroy_process_group()
 
 
-def test_cp_composition_matches_single_process(tmp_path):
+@pytest.mark.parametrize("world", [2, 4])
+def test_cp_composition_matches_single_process(tmp_path, world):
     from oracle import backward_dense, forward_dense
-    world = 2
     mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
                        start_method="spawn")
     wl, routes, q, k, v, do = _case()
