@@ -79,6 +79,8 @@ ATTENTION_MUTANTS = {
     "row dK unscaled": ("dk[R, g, :] += scale * (dS.T @ q[t, hs, :])", "dk[R, g, :] += dS.T @ q[t, hs, :]"),
     "row dQ against V": ("dq[i, hs, :] = scale * (dS @ Kg)", "dq[i, hs, :] = scale * (dS @ Vg)"),
     "sampled-key dV from dS": ("dv[dst, g, :] += P[:, n] @ do[t, hs, :]", "dv[dst, g, :] += dS[:, n] @ do[t, hs, :]"),
+    "sampled-key dK unscaled": ("dk[dst, g, :] += scale * (dS[:, n] @ q[t, hs, :])", "dk[dst, g, :] += dS[:, n] @ q[t, hs, :]"),
+    "tile run one key long": ("int(pos.size)", "int(pos.size) + 1"),
 }
 
 # ---------------------------------------------------------------------------
