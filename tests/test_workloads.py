@@ -76,3 +76,14 @@ def test_tensors_are_seeded_bf16():
 def test_pair_count():
     r = np.array([[3, 3, -1, 1, 9], [-1, -1, -1, -1, -1], [0, 1, 2, 3, 4]])
     assert W.pair_count(r, 4) == 2 + 0 + 4
+
+
+# the seeded recipes are fixed: their routed-pair counts are the ones the
+# design documentation and the benchmark figures quote
+PAIRS = {"tiny": 13709, "seq4k": 1010176, "thd16k": 7150250, "seq32k": 16598016, "cp128k": 15927894}
+
+
+@pytest.mark.parametrize("name", list(PAIRS))
+def test_seeded_pair_counts(name):
+    wl = W.WORKLOADS[name]
+    assert W.pair_count(W.make_routes(wl), wl.T_kv) == PAIRS[name]
