@@ -301,10 +301,14 @@ qsa_status_t qsa_selector_topk(const float* scores, int64_t score_stride, int64_
  *     (T = 4096 with n_sel = 256 fits; T = 16384 with n_sel = 512 does not).
  *     Larger sizes return QSA_ERR_WORKSPACE_TOO_SMALL and launch nothing; call
  *     qsa_forward with a workspace instead.  Other argument errors return the
- *     same statuses as qsa_forward.
+ *     same statuses as qsa_forward, checked in the same order (a call that is
+ *     both misaligned and too large returns QSA_ERR_MISALIGNED).
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.  Later calls on the device reuse the address.
+ *     before any stream capture.  Later calls on the device reuse the address
+ *     while the CUDA context it was taken in is current; after cudaDeviceReset
+ *     the next call looks it up again in the new context (so, again, make that
+ *     call before any capture).
  *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
  *   - All calls on one device share the array, and it keeps the last call's
  *     contents; nothing in it has to start at zero, because each call overwrites

@@ -106,6 +106,25 @@ def test_host_validation_before_any_launch(lib):
     assert lib.qsa_tile_plan_scratch_size(16, 300) == 2 * 256 + 256
 
 
+def _fwd_noalloc(lib, q=256, T=16, n_sel=4):
+    P = ctypes.c_void_p
+    f = lib.qsa_forward_noalloc
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, P, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_float, P, P, P]
+    return f(P(q), P(256), P(256), P(256), T, T, 12, 1, n_sel, 0.0625, P(256), P(256), None)
+
+
+def test_noalloc_host_validation_order(lib):
+    # the allocation-free forward checks in qsa_forward's order: pointers, sizes,
+    # scale, alignment, and only then its fixed scratch limit
+    assert _fwd_noalloc(lib, q=0) == 1
+    assert _fwd_noalloc(lib, T=0) == 1
+    assert _fwd_noalloc(lib, q=264) == 3                          # misaligned, small
+    assert _fwd_noalloc(lib, T=16384, n_sel=512) == 4             # aligned, needs ~32 MiB of scratch
+    assert _fwd_noalloc(lib, q=264, T=16384, n_sel=512) == 3      # misaligned and too large
+
+
 def test_bitmap_routes_host_validation(lib):
     P = ctypes.c_void_p
 

@@ -6,8 +6,9 @@ scratch from a fixed array inside the library instead of a caller workspace.
 This file runs last so that a failure here leaves every other test already run.
 The entry point is called through the C ABI twice in a row, on different
 inputs (the second smaller than the first, so stale scratch from the first call
-would show), and each result is checked against qsa_forward with a workspace,
-within the parity tolerances of the other GPU tests.
+would show).  It runs the same kernels as qsa_forward on the same inputs, so
+each result must equal qsa_forward's bit for bit; each is also checked against
+the FP64 CPU oracle within the parity tolerances of the other GPU tests.
 """
 
 import ctypes
@@ -16,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from token_indexed_sparse_b200 import qsa
 from token_indexed_sparse_b200 import workloads as W
 
@@ -51,13 +53,16 @@ def _inputs(wl):
     return q.to(DEV), k.to(DEV), v.to(DEV), routes
 
 
-def _compare(out, lse, ref_out, ref_lse):
-    o, r = out.double(), ref_out.double()
-    assert (o - r).abs().max().item() / max(r.abs().max().item(), 1e-3) <= REL_TOL
-    fin = torch.isfinite(ref_lse)
-    assert torch.equal(torch.isfinite(lse), fin)
-    assert torch.all(lse[~fin] == -float("inf"))
-    assert (lse[fin] - ref_lse[fin]).abs().max().item() <= LSE_TOL
+def _compare_oracle(out, lse, q, k, v, routes, scale):
+    f = lambda x: x.float().cpu().numpy().astype(np.float64)  # noqa: E731
+    ref_out, ref_lse = oracle.forward_dense(f(q), f(k), f(v), routes.cpu().numpy(), scale)
+    err = np.abs(f(out) - ref_out).max() / max(np.abs(ref_out).max(), 1e-3)
+    assert err <= REL_TOL
+    got = lse.cpu().numpy().astype(np.float64)
+    fin = np.isfinite(ref_lse)
+    assert np.array_equal(np.isfinite(got), fin)
+    assert np.all(got[~fin] == -np.inf)
+    assert np.abs(got[fin] - ref_lse[fin]).max() <= LSE_TOL
 
 
 def test_noalloc_forward_matches_workspace_forward_twice():
@@ -70,7 +75,9 @@ def test_noalloc_forward_matches_workspace_forward_twice():
         lse = torch.full((wl.T, wl.H), float("nan"), device=DEV)
         assert _call_noalloc(lib, q, k, v, routes, wl.scale, out, lse) == 0
         torch.cuda.synchronize()
-        _compare(out, lse, ref_out, ref_lse)
+        assert torch.equal(out, ref_out)
+        assert torch.equal(lse, ref_lse)
+        _compare_oracle(out, lse, q, k, v, routes, wl.scale)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():

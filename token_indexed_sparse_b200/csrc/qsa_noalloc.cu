@@ -23,24 +23,64 @@ constexpr int kMaxDevices = 64;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[QSA_NOALLOC_SCRATCH_BYTES];
 
 std::mutex g_mutex;
+// Per device: the context the address was taken in (its process-unique ID) and
+// the address.  A context is destroyed by cudaDeviceReset, and the runtime makes
+// a new one (with the module loaded again, possibly elsewhere) on the next call,
+// so an address is reused only while the context it came from is current.
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device, looked up once per
-// device.  In host code the array's name only stands in for the symbol, so the
-// address must come from cudaGetSymbolAddress with that device current.
+// Driver calls reached through the runtime (no link against libcuda): the
+// current context and its ID, which CUDA never gives to a second context.
+using CtxGetCurrentFn = int (*)(void**);
+using CtxGetIdFn = int (*)(void*, unsigned long long*);
+
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult r1 = cudaDriverEntryPointSymbolNotFound, r2 = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &r1) == cudaSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &r2) == cudaSuccess &&
+        r1 == cudaDriverEntryPointSuccess && r2 == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+      get_id = reinterpret_cast<CtxGetIdFn>(f2);
+    }
+    looked_up = true;
+  }
+  if (get_current == nullptr || get_id == nullptr) return false;
+  void* ctx = nullptr;
+  if (get_current(&ctx) != 0 || ctx == nullptr) return false;
+  return get_id(ctx, id) == 0 && *id != 0;
+}
+
+// Device address of the scratch array in the current context.  In host code the
+// array's name only stands in for the symbol, so the address must come from
+// cudaGetSymbolAddress with the device current.  It is looked up once per device
+// and context: the first call on a device (and the first after a device reset)
+// does it, and that call should come before any stream capture.  Should the
+// context ID be unavailable, it is looked up on every call (a host-side lookup
+// that allocates nothing).
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
+  unsigned long long ctx = 0;
+  if (current_context_id(&ctx) && g_scratch_ptr[dev] != nullptr && g_scratch_ctx[dev] == ctx) {
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
   }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_noalloc_scratch);  // makes the device's context current if it was not
+  if (e != cudaSuccess) return e;
+  g_scratch_ptr[dev] = p;
+  g_scratch_ctx[dev] = current_context_id(&ctx) ? ctx : 0;
+  *out = p;
   return cudaSuccess;
 }
 
@@ -63,11 +103,11 @@ extern "C" qsa_status_t qsa_forward_noalloc(const void* q, const void* k, const 
   const size_t need = qsa_forward_workspace_size(T, T_kv, H, G, n_sel);
   if (need == 0) return size_status(T, T_kv, H, G, n_sel);
   if (!(scale > 0.f) || !std::isfinite(scale)) return QSA_ERR_INVALID_ARGUMENT;
-  if (need > QSA_NOALLOC_SCRATCH_BYTES) return QSA_ERR_WORKSPACE_TOO_SMALL;
   const auto aligned = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; };
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(routes, 4) ||
       !aligned(lse, 4))
     return QSA_ERR_MISALIGNED;
+  if (need > QSA_NOALLOC_SCRATCH_BYTES) return QSA_ERR_WORKSPACE_TOO_SMALL;
   void* scratch = nullptr;
   if (scratch_address(&scratch) != cudaSuccess) return QSA_ERR_CUDA;
   // Scratch layout (the same as qsa_forward's workspace): a status word, row
