@@ -41,6 +41,7 @@ UNIT = "pairs/s"
 FWD_FLOPS_PER_PAIR_HEAD = 4 * 256      # QK^T + PV
 BWD_FLOPS_PER_PAIR_HEAD = 10 * 256     # S recompute, dP, dV, dQ, dK
 DKDV_FLOPS_PER_PAIR_HEAD = 4 * 256     # dK = dS^T Q, dV = P^T dO
+SPEC_BF16_TFLOPS = 2250.0              # B200 dense BF16 tensor peak (NVIDIA specification)
 # DRAM bytes (read + write) per step of a stage's kernel, from the ncu capture
 # summarised under profiles/, valid only for the sources it was taken on:
 # stage -> (bytes per step, {source file: sha256 of that file at capture time}).
@@ -69,7 +70,7 @@ def stage_traffic(stage):
 
 
 FWD_STAGES = ["fwd_route_rows", "fwd_attention"]
-BWD_STAGES = ["bwd_route_rows", "bwd_tile_scan", "bwd_tile_fill", "bwd_tile_sort", "bwd_dq", "bwd_dkdv"]
+BWD_STAGES = ["bwd_route_rows", "bwd_tile_lists", "bwd_tile_worklist", "bwd_dq", "bwd_dkdv"]
 
 
 def pass_ms(stage_ms):
@@ -378,23 +379,59 @@ def run_ours(args):
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in res_h)
 
-    def e2e_step():
-        ins = [t.to(dev, non_blocking=True) for t in host_in]
-        o, l_ = qsa.forward(ins[0], ins[1], ins[2], ins[4], wl.scale, workspace=ws_f)
-        g = qsa.backward(ins[3], ins[0], ins[1], ins[2], o, l_, ins[4], wl.scale, workspace=ws_b)
-        for dst, src in zip(res_h, (o, l_, *g)):
-            dst.copy_(src, non_blocking=True)
+    # Pipelined: step i's inputs go in on s_in while step i-1 computes on the bench
+    # stream and step i-2's results come out on s_out (two device buffer sets; the
+    # two copy directions use separate copy engines).  Every step's bytes cross the
+    # bus inside the timed region.
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    d_in = [[torch.empty(t.shape, dtype=t.dtype, device=dev) for t in host_in] for _ in range(2)]
+    d_res = [[torch.empty(t.shape, dtype=t.dtype, device=dev) for t in res_h] for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of set b landed
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]   # set b computed (its inputs consumed)
+    ev_out = [torch.cuda.Event() for _ in range(2)]   # results of set b copied out
 
-    e2e_steps = max(3, args.steps // 4)
-    e2e_step()
+    def e2e_run(n_steps):
+        for i in range(n_steps + 2):
+            if i < n_steps:
+                b = i & 1
+                if i >= 2:
+                    s_in.wait_event(ev_cmp[b])
+                with torch.cuda.stream(s_in):
+                    for d, h in zip(d_in[b], host_in):
+                        d.copy_(h, non_blocking=True)
+                ev_in[b].record(s_in)
+            j = i - 1
+            if 0 <= j < n_steps:
+                b = j & 1
+                stream.wait_event(ev_in[b])
+                if j >= 2:
+                    stream.wait_event(ev_out[b])
+                q_, k_, v_, do_, r_ = d_in[b]
+                o_, l_, dq_, dk_, dv_ = d_res[b]
+                qsa.forward(q_, k_, v_, r_, wl.scale, out=o_, lse=l_, workspace=ws_f)
+                qsa.backward(do_, q_, k_, v_, o_, l_, r_, wl.scale, dq=dq_, dk=dk_, dv=dv_, workspace=ws_b)
+                ev_cmp[b].record(stream)
+            kk = i - 2
+            if 0 <= kk < n_steps:
+                b = kk & 1
+                s_out.wait_event(ev_cmp[b])
+                with torch.cuda.stream(s_out):
+                    for h, d in zip(res_h, d_res[b]):
+                        h.copy_(d, non_blocking=True)
+                ev_out[b].record(s_out)
+
+    e2e_steps = max(3, args.steps // 2)
+    e2e_run(2)
     torch.cuda.synchronize()
     e0, e1 = mk(), mk()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
+    e2e_run(e2e_steps)
+    stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
@@ -403,6 +440,7 @@ def run_ours(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e_value = world * pairs * e2e_steps / (e2e_ms * 1e-3)
+    del d_in, d_res
 
     peaks = load_peaks()
     avg = {n: float(np.mean(v)) for n, v in stage_ms.items()}
@@ -419,10 +457,12 @@ def run_ours(args):
     roofline = None
     if work is not None:
         achieved = work / (avg[dominant] * 1e-3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
+        peak = peaks["bf16_tflops"]
         roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": stage_traffic(dominant),
-                    "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)"}
+                    "peak_source": f"{peaks['source']} bf16_tflops (burst; the timed region is well under a "
+                                   f"second)",
+                    "frac_of_spec": achieved / SPEC_BF16_TFLOPS}
     aux = {"bitmap_routes": bitmap_adapter_aux(qsa, torch, routes, wl, dev, flush, peaks),
            "selector": selector_aux(qsa, torch, dev, flush, peaks)}
     step_tflops = flops / (ms_per_step * 1e-3) / 1e12
@@ -434,14 +474,17 @@ def run_ours(args):
                    "l2": "flushed (256 MiB write) before every timed step, outside its events",
                    "parallelism": f"{world} independent sequences (one per GPU)" if world > 1 else "1 GPU"},
         "tflops": step_tflops * world,
-        "step_roofline": {"flops": flops, "t_roof_ms": flops / (peaks["bf16_tflops_sustained"] * 1e12) * 1e3,
-                          "frac": step_tflops / peaks["bf16_tflops_sustained"],
-                          "peak": peaks["bf16_tflops_sustained"], "peak_source": peaks["source"]},
+        "step_roofline": {"flops": flops, "t_roof_ms": flops / (peaks["bf16_tflops"] * 1e12) * 1e3,
+                          "frac": step_tflops / peaks["bf16_tflops"],
+                          "peak": peaks["bf16_tflops"], "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                          "frac_of_spec": step_tflops / SPEC_BF16_TFLOPS},
         "stage_ms": avg,
         "pass_ms": pass_ms(avg),
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": e2e_steps},
+                "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+                "how": "pinned host -> device inputs, forward + backward through the C ABI, device -> pinned host "
+                       "results, every step; copies of neighbouring steps overlap the kernels on two copy streams"},
         "gpu_launches": args.steps * (qsa.launch_count(wl.T, wl.T_kv, wl.H, wl.G, wl.W, False)
                                       + qsa.launch_count(wl.T, wl.T_kv, wl.H, wl.G, wl.W, True)),
         "clocks": clk,
@@ -455,6 +498,122 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
+
+
+def run_cp(args):
+    """Context parallelism: ONE sequence of the workload (cp128k by default: 8192
+    query rows against 131072 K/V rows) split across the ranks through
+    token_indexed_sparse_b200.cp: each rank owns a pair-balanced range of query
+    rows and an equal slice of K/V; a step is the CP forward (K/V all-gather,
+    local forward) and the CP backward (all-gather, local FP32 dK/dV backward,
+    FP32 reduce-scatter, BF16 rounding of the own slice), collectives inside the
+    timed region.  Total work is fixed as the rank count grows (strong scaling)."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    from token_indexed_sparse_b200 import cp, qsa
+    from token_indexed_sparse_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    else:
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                device_id=dev, timeout=datetime.timedelta(seconds=120))
+    wl = W.WORKLOADS[args.workload if args.workload != WORKLOAD else "cp128k"]
+    if args.scale_T:
+        wl = wl.scaled(args.scale_T)
+    routes_np = np.array(W.make_routes(wl), dtype=np.int32)
+    counts = np.array([np.unique(r[(r >= 0) & (r < wl.T_kv)]).size for r in routes_np])
+    s, e = cp.balanced_query_ranges(counts, world)[rank]
+    ks, ke = cp.kv_slice(wl.T_kv, world, rank)
+    q_h, k_h, v_h, do_h = W.make_tensors(wl)
+    pairs_total = int(counts.sum())
+    host_in = [t.contiguous().pin_memory() for t in (q_h[s:e], k_h[ks:ke], v_h[ks:ke], do_h[s:e],
+                                                     torch.from_numpy(routes_np[s:e]))]
+    q, k, v, do, routes = (t.to(dev) for t in host_in)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(q_, k_, v_, do_, r_):
+        out, lse = cp.cp_forward(q_, k_, v_, r_, wl.scale)
+        return (out, lse, *cp.cp_backward(do_, q_, k_, v_, out, lse, r_, wl.scale))
+
+    for _ in range(args.warmup):
+        step(q, k, v, do, routes)
+        flush.zero_()
+    torch.cuda.synchronize()
+    mk = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    ev = [(mk(), mk()) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()                 # L2 flushed before every timed step (outside its events)
+        ev[i][0].record(stream)
+        step(q, k, v, do, routes)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clk = clocks.stop()
+    t = torch.tensor([sum(a.elapsed_time(b) for a, b in ev)], device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    value = pairs_total * args.steps / (total_ms * 1e-3)
+
+    # end to end: this rank's inputs in from pinned host memory, the CP step,
+    # its results (out, lse, dq, own dk / dv slices) back to pinned host memory
+    res_shapes = [(e - s, wl.H, 256), (e - s, wl.H), (e - s, wl.H, 256), (ke - ks, wl.G, 256), (ke - ks, wl.G, 256)]
+    res_types = [torch.bfloat16, torch.float32, torch.bfloat16, torch.bfloat16, torch.bfloat16]
+    res_h = [torch.empty(sh, dtype=ty, pin_memory=True) for sh, ty in zip(res_shapes, res_types)]
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = sum(x.numel() * x.element_size() for x in res_h)
+    e2e_steps = max(3, args.steps // 2)
+    dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = mk(), mk()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        ins = [x.to(dev, non_blocking=True) for x in host_in]
+        for dst, src in zip(res_h, step(*ins)):
+            dst.copy_(src, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = torch.tensor([e0.elapsed_time(e1)], device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    e2e_value = pairs_total * e2e_steps / (float(t.item()) * 1e-3)
+    flops = (FWD_FLOPS_PER_PAIR_HEAD + BWD_FLOPS_PER_PAIR_HEAD) * wl.H * pairs_total
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {**workload_config(wl), "pairs_per_step": pairs_total, "flops_per_step": flops,
+                   "l2": "flushed (256 MiB write) before every timed step, outside its events",
+                   "parallelism": f"cp{world}: one sequence, query rows balanced by routed pairs, K/V "
+                                  f"all-gather and FP32 dK/dV reduce-scatter over NCCL"},
+        "tflops": flops * args.steps / (total_ms * 1e-3) / 1e12,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps, "how": "per rank: its inputs in, the CP step, its results out, serially"},
+        "gpu_launches": args.steps * (qsa.launch_count(e - s, wl.T_kv, wl.H, wl.G, wl.W, False)
+                                      + qsa.launch_count(e - s, wl.T_kv, wl.H, wl.G, wl.W, True) + 2),
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    dist.destroy_process_group()
 
 
 def main():
@@ -471,9 +630,14 @@ def main():
                     help="run the workload's recipe at this many query rows (profiling of smaller cases)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--reference-rows", type=int, default=96)
+    ap.add_argument("--mode", choices=["replicas", "cp"], default="replicas",
+                    help="replicas: one independent sequence per GPU (default); cp: one sequence split across "
+                         "the GPUs by context parallelism")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.mode == "cp":
+        run_cp(args)
     else:
         run_ours(args)
 

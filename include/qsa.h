@@ -138,13 +138,13 @@ qsa_status_t qsa_backward_fp32kv(const void* grad_out, const void* q, const void
  * `stage_events` may be NULL when n_stage_events is 0.  The pages have no
  * counterpart: this is an instrumentation hook of this library.
  *   forward stages : 0 route rows (sort/dedup), 1 attention forward
- *   backward stages: 0 route rows (+ delta), 1 tile counts + scan, 2 tile fill,
- *                    3 tile sort + work lists, 4 dQ (+ P/dS records), 5 dK/dV
+ *   backward stages: 0 route rows (+ delta), 1 tile lists (masks, column scans,
+ *                    tile scan, fill), 2 work lists, 3 dQ (+ P/dS records), 4 dK/dV
  * A failed eventRecord returns QSA_ERR_CUDA.
  */
 typedef struct CUevent_st* qsa_event_t; /* same type as cudaEvent_t */
 #define QSA_FORWARD_STAGES 2
-#define QSA_BACKWARD_STAGES 6
+#define QSA_BACKWARD_STAGES 5
 
 qsa_status_t qsa_forward_ex(const void* q, const void* k, const void* v, const int32_t* routes,
                             int64_t T, int64_t T_kv, int H, int G, int n_sel, float scale,
@@ -283,6 +283,20 @@ qsa_status_t qsa_selector_scores(const void* qi, const void* kbar, int64_t T, in
 qsa_status_t qsa_selector_topk(const float* scores, int64_t score_stride, int64_t T, int64_t NB, int k,
                                const int32_t* pos, const int32_t* blk_base, const int32_t* tok_base,
                                int32_t* blocks, int32_t* routes, qsa_stream_t stream);
+
+/*
+ * FP32 -> BF16 rounding of n contiguous values, round to nearest with ties to
+ * even: the final cast of dK / dV sums that a caller adds up in FP32 across
+ * several qsa_backward_fp32kv calls (context parallelism reduce-scatters each
+ * rank's FP32 partials, then rounds its own slice once), with the rounding the
+ * backward applies itself ("Selection and components": FP32 accumulation,
+ * BF16 gradients).
+ *   x [n] float32, y [n] bf16 (device, caller-owned, 16-byte aligned; they
+ *   must not overlap).  Enqueued on `stream`.
+ * Errors: n < 0 or a NULL pointer with n > 0: QSA_ERR_INVALID_ARGUMENT;
+ * misaligned pointers: QSA_ERR_MISALIGNED; a failed launch: QSA_ERR_CUDA.
+ */
+qsa_status_t qsa_cast_f32_to_bf16(const float* x, void* y, int64_t n, qsa_stream_t stream);
 
 /*
  * Allocation-free forward, for callers that cannot allocate device memory: for

@@ -68,7 +68,9 @@ def _rank_main(rank, world, port, out_dir):
 
         rl = torch.from_numpy(routes[s:e])
         out, lse = cp.cp_forward(q[s:e], k[ks:ke], v[ks:ke], rl, wl.scale, local_forward=fwd)
-        dq, dk, dv = cp.cp_backward(do[s:e], q[s:e], k[ks:ke], v[ks:ke], out, lse, rl, wl.scale, local_backward=bwd)
+        # FP64 partials from the oracle, summed across ranks and kept in FP64 (no final rounding)
+        dq, dk, dv = cp.cp_backward(do[s:e], q[s:e], k[ks:ke], v[ks:ke], out, lse, rl, wl.scale, local_backward=bwd,
+                                    final_cast=lambda x: x)
         np.savez(os.path.join(out_dir, f"rank{rank}.npz"), s=s, e=e, ks=ks, ke=ke, out=out.numpy(),
                  lse=lse.numpy(), dq=dq.numpy(), dk=dk.numpy(), dv=dv.numpy())
     finally:

@@ -65,3 +65,33 @@ def test_cp_single_rank_reproduces_plain_calls():
         assert torch.equal(c_dq, dq) and torch.equal(c_dk, dk) and torch.equal(c_dv, dv)
     finally:
         dist.destroy_process_group()
+
+
+def _rne_bf16_bits(x32: np.ndarray) -> np.ndarray:
+    """Round-to-nearest-even of FP32 to BF16, as bit patterns: add half an ulp of
+    the BF16 result (minus one when the kept part is even, so that exact ties go
+    to the even neighbour) and drop the low 16 bits; NaNs are left to the caller."""
+    b = x32.view(np.uint32).astype(np.uint64)
+    lsb = (b >> 16) & 1
+    return ((b + 0x7FFF + lsb) >> 16).astype(np.uint16)
+
+
+@pytest.mark.parametrize("n", [0, 1, 7, 8, 9, 31, 4096 + 5, 1 << 20])
+def test_cast_f32_to_bf16_is_round_to_nearest_even(n):
+    rng = np.random.default_rng(n)
+    x = (rng.standard_normal(n) * np.exp2(rng.integers(-140, 120, n))).astype(np.float32)
+    if n >= 31:
+        specials = np.array([0.0, -0.0, np.inf, -np.inf, 1e-45, -1e-45, 3.4028235e38, -3.4028235e38],
+                            dtype=np.float32)
+        x[:8] = specials
+        # exact ties: low half exactly 0x8000 above an even and an odd BF16 value
+        x[8:12] = np.array([0x3F808000, 0x3F818000, 0xBF808000, 0x00018000], dtype=np.uint32).view(np.float32)
+        x[12] = np.nan
+    xd = torch.from_numpy(x).to(DEV)
+    y = qsa.cast_f32_to_bf16(xd)
+    torch.cuda.synchronize()
+    got = y.cpu().view(torch.int16).numpy().view(np.uint16)
+    nan = np.isnan(x)
+    assert np.array_equal(got[~nan], _rne_bf16_bits(x)[~nan])
+    assert np.all(np.isnan(y.cpu().float().numpy()[nan]))
+    assert torch.equal(y[~torch.from_numpy(nan).to(DEV)], xd[~torch.from_numpy(nan).to(DEV)].to(torch.bfloat16))

@@ -103,6 +103,38 @@ def test_parity_dense_oracle(name):
 # full workload sizes: sampled rows and keys computed one by one by the oracle
 # ---------------------------------------------------------------------------
 
+def phase_spanning_tiles(routes, T_kv, C, n=2):
+    """Two 128-key tiles whose query lists reach into at least two dK/dV query
+    phases of C rows (so their dK/dV sum ordered FP32 partials across phases),
+    the ones with the median number of (query, tile) entries among those
+    (when T <= C there is one phase: the median tiles with entries)."""
+    r = np.asarray(routes).astype(np.int64)
+    t = np.repeat(np.arange(r.shape[0], dtype=np.int64), r.shape[1])
+    key = r.ravel()
+    ok = (key >= 0) & (key < T_kv)
+    pair = np.unique(t[ok] * ((T_kv + 127) // 128) + key[ok] // 128)   # distinct (query, tile)
+    tq, tl = pair // ((T_kv + 127) // 128), pair % ((T_kv + 127) // 128)
+    n_ent = np.bincount(tl, minlength=(T_kv + 127) // 128)
+    phases = np.unique(tl * (1 << 20) + tq // C)
+    n_ph = np.bincount(phases >> 20, minlength=(T_kv + 127) // 128)
+    multi = np.nonzero(n_ph >= 2)[0]
+    if len(multi) < n:                      # a single phase (T <= C): any tiles with entries
+        multi = np.nonzero(n_ent > 0)[0]
+    order = multi[np.argsort(n_ent[multi], kind="stable")]
+    mid = len(order) // 2
+    return order[mid : mid + n]
+
+
+def dkdv_phase_rows(T, H):
+    # the library's dK/dV query-phase length: 48 MiB of one tensor's Q rows,
+    # at least 4096 rows, a multiple of 256 (at most 64 phases)
+    c = (48 << 20) // (H * 1024)
+    c = 4096 if c < 4096 else (c // 256) * 256
+    if (T + c - 1) // c > 64:
+        c = (((T + 63) // 64) + 255) // 256 * 256
+    return c
+
+
 @pytest.mark.parametrize("name", ["seq4k", "thd16k", "seq32k", "cp128k"])
 def test_parity_full_size_sampled(name):
     wl = W.WORKLOADS[name]
@@ -110,7 +142,7 @@ def test_parity_full_size_sampled(name):
     out, lse, dq, dk, dv = run_gpu(q, k, v, do, routes, wl.scale)
     rng = np.random.default_rng(wl.seed - 1000)
     counts = oracle.route_rows_csr(routes, wl.T_kv)[0]
-    rows = np.unique(np.concatenate([rng.choice(wl.T, 48, replace=False),
+    rows = np.unique(np.concatenate([rng.choice(wl.T, 509, replace=False),
                                      [int(np.argmax(counts)), wl.T - 1, 0]]))
     qf, kf, vf, dof = f64(q), f64(k), f64(v), f64(do)
     r_out, r_lse = oracle.forward_rows(qf, kf, vf, routes, wl.scale, rows)
@@ -118,13 +150,13 @@ def test_parity_full_size_sampled(name):
     check_lse(lse[rows].cpu().numpy().astype(np.float64), r_lse)
     assert rel_err(f64(out[rows]), r_out) <= REL_TOL
     assert rel_err(f64(dq[rows]), r_dq) <= REL_TOL
-    # keys: random, the most recent (hot) ones, one past every route, and a run
-    # of 16 consecutive keys inside one 128-key tile (they share the tile's
-    # query unions in the dK/dV kernel)
-    tile = int(rng.integers(0, wl.T_kv // 128))
+    # keys: random, the most recent (hot) ones, one past every route, and every
+    # key of two whole 128-key tiles whose dK/dV sums run over several query
+    # phases (ordered FP32 partials between phases)
+    tiles = phase_spanning_tiles(routes, wl.T_kv, dkdv_phase_rows(wl.T, wl.H))
     keys = np.unique(np.concatenate([rng.choice(wl.T_kv, 10, replace=False),
-                                     [wl.T_kv - 1, wl.T_kv - 5],
-                                     np.arange(tile * 128 + 40, tile * 128 + 56)]))
+                                     [wl.T_kv - 1, wl.T_kv - 5]] +
+                                    [np.arange(tl * 128, min(wl.T_kv, tl * 128 + 128)) for tl in tiles]))
     r_dk, r_dv = oracle.backward_keys(dof, qf, kf, vf, routes, wl.scale, keys)
     assert rel_err(f64(dk[keys]), r_dk) <= REL_TOL
     assert rel_err(f64(dv[keys]), r_dv) <= REL_TOL

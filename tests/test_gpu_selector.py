@@ -6,7 +6,10 @@ Scores: FP32 tensor-core accumulation of BF16 products against the FP64
 oracle, max error <= 1e-4 of the row's largest score.  The top-k is an integer
 decision taken from floating-point scores, so it is compared bit for bit
 against the oracle's top-k applied to the GPU's own FP32 scores (the same
-precision on both sides), and the routes against the oracle's expansion.
+precision on both sides), and the routes against the oracle's expansion.  The
+chosen set is also checked against the FP64 oracle scores: it must be a valid
+top-k up to the score tolerance (no unchosen candidate beats a chosen one by
+more than twice the scores' error bound).
 """
 
 import json
@@ -35,6 +38,25 @@ def _check_scores(S_gpu, S_ref, n):
             continue
         a, b = S_gpu[t, :m], S_ref[t, :m]
         assert np.abs(a - b).max() <= 1e-4 * max(np.abs(b).max(), 1e-6), t
+
+
+def _check_topk_valid(blocks, S_ref, n, k):
+    # blocks [T, k] from the GPU against the FP64 scores S_ref: min(k, n_t)
+    # distinct candidates, ascending, -1 after them, and a top-k of S_ref up to
+    # the tolerance (each side's scores are within 1e-4 of the row maximum)
+    for t in range(S_ref.shape[0]):
+        m = int(n[t])
+        want = min(k, m)
+        b = blocks[t]
+        chosen = b[:want]
+        assert np.all(b[want:] == -1), t
+        assert np.all((chosen >= 0) & (chosen < m)) and np.all(np.diff(chosen) > 0), t
+        if want == 0 or want == m:
+            continue
+        row = S_ref[t, :m]
+        tol = 2e-4 * max(np.abs(row).max(), 1e-6)
+        unchosen = np.setdiff1d(np.arange(m), chosen)
+        assert row[chosen].min() >= row[unchosen].max() - tol, t
 
 
 def _check_topk(S_gpu, n, k, blocks, routes, T, pos=None, tok_base=None):
@@ -76,8 +98,10 @@ def test_random_single_sequence(T, Hi, k, seed):
     assert int(status.item()) == 0
     S = S.cpu().numpy()
     n = n_candidates(T, NB)
-    _check_scores(S, selector_scores(qi.double().numpy(), kbar.double().numpy(), scale), n)
+    S_ref = selector_scores(qi.double().numpy(), kbar.double().numpy(), scale)
+    _check_scores(S, S_ref, n)
     _check_topk(S, n, k, blocks.cpu().numpy(), routes.cpu().numpy(), T)
+    _check_topk_valid(blocks.cpu().numpy(), S_ref, n, k)
 
 
 def test_packed_sequences_with_positions():
@@ -99,8 +123,10 @@ def test_packed_sequences_with_positions():
     assert int(status.item()) == 0
     S = S.cpu().numpy()
     n = n_candidates(T, NB, pos, blk_base, tok_base)
-    _check_scores(S, selector_scores(qi.double().numpy(), kbar.double().numpy(), 0.5, pos, blk_base, tok_base), n)
+    S_ref = selector_scores(qi.double().numpy(), kbar.double().numpy(), 0.5, pos, blk_base, tok_base)
+    _check_scores(S, S_ref, n)
     _check_topk(S, n, k, blocks.cpu().numpy(), routes.cpu().numpy(), T, pos, tok_base)
+    _check_topk_valid(blocks.cpu().numpy(), S_ref, n, k)
 
 
 def test_topk_ties_and_short_rows():
@@ -132,6 +158,7 @@ def test_full_size_sampled_rows():
         if n:
             ref = (1 / 64) * np.maximum(qi[t].double().numpy() @ kd[:n].T, 0).sum(axis=0)
             assert np.abs(Sc[t, :n] - ref).max() <= 1e-4 * np.abs(ref).max(), t
+            _check_topk_valid(bc[t:t + 1], ref[None, :], [n], k)
         ref_b = topk_blocks(Sc[t:t + 1].astype(np.float64), [n], k)
         assert np.array_equal(bc[t:t + 1], ref_b), t
         assert np.array_equal(rc[t:t + 1], expand_routes(ref_b, 1, pos=[t])), t

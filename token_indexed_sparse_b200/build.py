@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libqsa_b200.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
-SOURCES = ["qsa_api.cu", "qsa_routes.cu", "qsa_forward.cu", "qsa_backward.cu", "qsa_noalloc.cu", "qsa_bitmap.cu", "qsa_selector.cu", "qsa_dkdv_union.cu"]
+SOURCES = ["qsa_api.cu", "qsa_routes.cu", "qsa_forward.cu", "qsa_backward.cu", "qsa_noalloc.cu", "qsa_bitmap.cu", "qsa_selector.cu", "qsa_dkdv_union.cu", "qsa_cast.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xptxas", "-v"]
 

@@ -96,22 +96,29 @@ def cp_forward(q, k_local, v_local, routes, scale: float, group=None, local_forw
     return local_forward(q, k, v, routes, scale)
 
 
-def cp_backward(grad_out, q, k_local, v_local, out, lse, routes, scale: float, group=None, local_backward=None):
+def cp_backward(grad_out, q, k_local, v_local, out, lse, routes, scale: float, group=None, local_backward=None,
+                final_cast=None):
     """Backward of this rank's query rows; returns ``(dq, dk_local, dv_local)``.
 
     dq covers the local query rows; dk_local / dv_local are the gradients of the
     rank's own K/V slice summed over every rank's queries (FP32 reduce-scatter,
-    then one rounding to the K/V dtype).
+    then one rounding to BF16 by the library's cast kernel).  ``local_backward``
+    must return FP32 (or wider) dK/dV partials; ``final_cast(x)`` rounds the
+    rank's summed slice (both are parameters only so that the collective
+    plumbing can run on CPU processes).
     """
-    if local_backward is None:
+    if local_backward is None or final_cast is None:
         from . import qsa
-
+    if local_backward is None:
         def local_backward(go, q_, k_, v_, o_, l_, r_, s_):
             return qsa.backward(go, q_, k_, v_, o_, l_, r_, s_, kv_fp32=True)
+    if final_cast is None:
+        final_cast = qsa.cast_f32_to_bf16
     k = _all_gather_rows(k_local, group)
     v = _all_gather_rows(v_local, group)
     dq, dk_part, dv_part = local_backward(grad_out, q, k, v, out, lse, routes, scale)
-    wide = (lambda x: x if x.dtype == torch.float64 else x.to(torch.float32))  # noqa: E731
-    dk = _reduce_scatter_rows(wide(dk_part), group).to(k_local.dtype)
-    dv = _reduce_scatter_rows(wide(dv_part), group).to(v_local.dtype)
+    if dk_part.dtype not in (torch.float32, torch.float64) or dv_part.dtype != dk_part.dtype:
+        raise TypeError("local_backward must return FP32 (or FP64) dK/dV partials")
+    dk = final_cast(_reduce_scatter_rows(dk_part, group))
+    dv = final_cast(_reduce_scatter_rows(dv_part, group))
     return dq, dk, dv

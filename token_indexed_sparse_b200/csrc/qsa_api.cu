@@ -46,7 +46,7 @@ void dkdv_phases(int64_t T, int H, int* P, int* C) {
 
 struct Layout {
   size_t status = 0, row_cnt = 0, row_cols = 0, tile_ctr = 0, tile_ptr = 0, tile_fill = 0, tile_ent = 0, delta = 0,
-         pds = 0, phase_ptr = 0, wl = 0, partial = 0, total = 0;
+         pds = 0, lists = 0, wl = 0, partial = 0, total = 0;
   int P = 1, C = 1;
 };
 
@@ -78,7 +78,7 @@ Layout make_layout(int64_t T, int64_t T_kv, int H, int G, int n_sel, bool backwa
     L.tile_ent = take(pairs * 8);  // at most one entry per routed pair
     L.delta = take(static_cast<size_t>(T) * H * 4);
     L.pds = take(pairs * G * 48);  // BF16 [P | dS] of every routed pair, 12 heads each
-    L.phase_ptr = take(nt * (L.P + 1) * 4);
+    L.lists = take(qsa::tile_lists_bytes(T, T_kv));  // masks and block bases of the tile lists
     L.wl = take(static_cast<size_t>(L.P) * nt * 16);
     L.partial = take(nt * G * 2 * 128 * 256 * 4);  // FP32 dK and dV of every (tile, group)
   }
@@ -141,7 +141,7 @@ static qsa_status_t backward_impl(const void* grad_out, const void* q, const voi
   int64_t* tile_ent = at<int64_t>(workspace, L.tile_ent);
   float* delta = at<float>(workspace, L.delta);
   uint16_t* pds = at<uint16_t>(workspace, L.pds);  // [T, G, n_sel, 24]
-  int32_t* phase_ptr = at<int32_t>(workspace, L.phase_ptr);
+  void* lists = at<void>(workspace, L.lists);
   int4* wl = at<int4>(workspace, L.wl);
   float* partial = at<float>(workspace, L.partial);
   const StageEvents ev{stage_events, n_stage_events, s};
@@ -149,20 +149,16 @@ static qsa_status_t backward_impl(const void* grad_out, const void* q, const voi
   QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 0, status, grad_out, out, delta,
                                  H, s));
   QSA_TRY(ev.mark(0));
-  QSA_TRY(qsa::launch_tile_count(row_cnt, row_cols, T, n_sel, nt, tile_cnt, s));
-  QSA_TRY(qsa::launch_quad_scan(tile_cnt, nt, tile_ptr, tile_fill, s));
+  QSA_TRY(qsa::launch_tile_lists(row_cnt, row_cols, T, n_sel, nt, lists, tile_cnt, tile_ptr, tile_fill, tile_ent, s));
   QSA_TRY(ev.mark(1));
-  QSA_TRY(qsa::launch_tile_fill(row_cnt, row_cols, T, n_sel, nt, tile_fill, tile_ent, s));
+  QSA_TRY(qsa::launch_tile_worklist(tile_ptr, lists, T, nt, T_kv, G, L.P, L.C, wl_cnt, wl, dk, dv, kv_f32, s));
   QSA_TRY(ev.mark(2));
-  QSA_TRY(qsa::launch_tile_sort(tile_ptr, nt, tile_ent, L.P, L.C, phase_ptr, s));
-  QSA_TRY(qsa::launch_tile_worklist(tile_ptr, phase_ptr, nt, T_kv, G, L.P, wl_cnt, wl, dk, dv, kv_f32, s));
-  QSA_TRY(ev.mark(3));
   QSA_TRY(qsa::launch_backward_dq(grad_out, q, k, v, lse, delta, row_cnt, row_cols, T, G, n_sel, scale, dq, pds,
                                   s));
-  QSA_TRY(ev.mark(4));
+  QSA_TRY(ev.mark(3));
   QSA_TRY(qsa::launch_backward_dkdv_union(grad_out, q, pds, row_cols, tile_ent, wl_cnt, wl, claim, done,
                                           L.P, nt, T_kv, G, n_sel, scale, partial, dk, dv, kv_f32, status, s));
-  QSA_TRY(ev.mark(5));
+  QSA_TRY(ev.mark(4));
   return QSA_OK;
 }
 
@@ -252,7 +248,8 @@ qsa_status_t qsa_backward_fp32kv(const void* grad_out, const void* q, const void
 
 int qsa_launch_count(int64_t T, int64_t T_kv, int H, int G, int n_sel, int backward) {
   if (check_sizes(T, T_kv, H, G, n_sel) != QSA_OK) return 0;
-  return backward ? 8 : 2;  // backward: route rows, tile count, scan, fill, sort + work list, dQ, dK/dV
+  // backward: route rows, tile masks, column scans, tile scan, tile fill, work lists, dQ, dK/dV
+  return backward ? 8 : 2;
 }
 
 qsa_status_t qsa_bitmap_routes(const uint8_t* sel_blocks, const int32_t* lo, const int32_t* hi,
@@ -333,7 +330,7 @@ qsa_status_t qsa_route_plan(const int32_t* routes, int64_t T, int64_t T_kv, int 
 size_t qsa_tile_plan_scratch_size(int64_t T, int64_t T_kv) {
   if (T < 1 || T_kv < 1 || T_kv > INT32_MAX) return 0;
   const size_t nt = static_cast<size_t>((T_kv + 127) / 128);
-  return 2 * align256(nt * 4) + align256(nt * 8);
+  return 2 * align256(nt * 4) + align256(qsa::tile_lists_bytes(T, T_kv));
 }
 
 qsa_status_t qsa_tile_plan(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel, int32_t* row_cnt,
@@ -350,14 +347,10 @@ qsa_status_t qsa_tile_plan(const int32_t* routes, int64_t T, int64_t T_kv, int n
   const int64_t nt = (T_kv + 127) / 128;
   int32_t* tile_cnt = static_cast<int32_t*>(scratch);
   int32_t* tile_fill = at<int32_t>(scratch, align256(static_cast<size_t>(nt) * 4));
-  int32_t* phase_ptr = at<int32_t>(scratch, 2 * align256(static_cast<size_t>(nt) * 4));
-  QSA_TRY(cudaMemsetAsync(tile_cnt, 0, static_cast<size_t>(nt) * 4, s));
+  void* lists = at<void>(scratch, 2 * align256(static_cast<size_t>(nt) * 4));
   QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 0, nullptr, nullptr, nullptr,
                                  nullptr, qsa::kHeadsPerGroup, s));
-  QSA_TRY(qsa::launch_tile_count(row_cnt, row_cols, T, n_sel, nt, tile_cnt, s));
-  QSA_TRY(qsa::launch_quad_scan(tile_cnt, nt, tile_ptr, tile_fill, s));
-  QSA_TRY(qsa::launch_tile_fill(row_cnt, row_cols, T, n_sel, nt, tile_fill, tile_ent, s));
-  QSA_TRY(qsa::launch_tile_sort(tile_ptr, nt, tile_ent, 1, static_cast<int>(T), phase_ptr, s));
+  QSA_TRY(qsa::launch_tile_lists(row_cnt, row_cols, T, n_sel, nt, lists, tile_cnt, tile_ptr, tile_fill, tile_ent, s));
   return QSA_OK;
 }
 

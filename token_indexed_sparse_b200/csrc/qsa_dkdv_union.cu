@@ -19,11 +19,12 @@
 //
 // Warp roles (384 threads): warp 6 schedules (claims units, cuts them into
 // chunks of 4 entries, publishes each chunk's descriptor in a shared-memory ring
-// and prefetches its records and keys into L2); warps 0-5 fill whole chunks,
-// warp w the chunks of stage w of the 6-stage shared-memory ring (clear A,
-// gather B rows with cp.async, store the records into their A rows); warp 7
-// (one thread) issues the MMAs; warps 8-11 (tensor-memory lane quarters 0-3)
-// run the epilogue, thread = key row.  Units are claimed from one counter in
+// and prefetches its records and keys into L2); warps 0-5 fill the chunks, warp
+// s every chunk of stage s of the 6-stage shared-memory ring (clear A, gather B
+// rows with cp.async, store the records into their A rows); warp 7 (one
+// thread) issues the MMAs; warps 8-11 (tensor-memory lane quarters 0-3) run the
+// epilogue, thread = key row.  The stage fill is written for kUWorkersPerStage
+// warps per stage, each taking an equal share of the chunk's unions.  Units are claimed from one counter in
 // phase order (phase 0's units, then phase 1's, ...; inside a phase every dK
 // unit before every dV unit), so the
 // CTAs work on about one phase and one tensor at a time and its Q (or dO) rows
@@ -46,7 +47,9 @@ namespace {
 // buffer, 512 per SM)
 constexpr int kUCtasPerSm = 1, kUAccBufs = 2;
 constexpr int kUTmemCols = 256 * kUAccBufs;
-constexpr int kUWorkers = 6;                        // warps 0-5 fill chunks, warp w every stage-w chunk
+constexpr int kUStages = 6;
+constexpr int kUWorkersPerStage = 1;                // (two per stage, each two unions: 7.16 -> 7.58 ms on seq32k)
+constexpr int kUWorkers = kUStages * kUWorkersPerStage;  // warps 0-5 fill chunks
 constexpr int kUSchedWarp = 6, kUMmaWarp = 7, kUEpiWarp0 = 8;
 constexpr int kUWarps = 12;
 constexpr int kUThreads = 32 * kUWarps;
@@ -59,7 +62,6 @@ constexpr int kUBBytes = 4 * kUBBlk;                // 24 KB
 constexpr int kUASbo = (kUK / 8) * 128;             // A: bytes between 8-key core-matrix rows (768)
 constexpr int kUABytes = kUKeys * kUK * 2;          // 12 KB
 constexpr int kUStage = kUBBytes + kUABytes;        // 36 KB
-constexpr int kUStages = 6;
 constexpr int kURing = 16;                          // chunk descriptors the scheduler may run ahead
 constexpr int kUOffCtl = kUStages * kUStage;
 // control block: stage descriptors, accumulator descriptors, the chunk ring
@@ -78,11 +80,14 @@ constexpr int kUOffTmem = kUBarDrain + 8, kUOffAbort = kUOffTmem + 4;
 constexpr int kUSmem = kUOffAbort + 4 + 1024;      // + alignment slack
 static_assert(kUStage % 1024 == 0, "stage alignment (128-byte swizzle atoms)");
 static_assert(kUSmem <= 232448, "shared memory per block");
-// One worker per stage: chunk c goes to warp c % kUStages, so every wait on a
-// stage's barriers comes from one warp, in order, at most one phase ahead of
-// the barrier (a parity wait two phases early would pass at once).  The
-// descriptor ring is at least as deep as the worker count for the same reason.
-static_assert(kUWorkers == kUStages && kURing >= kUWorkers, "one worker per stage");
+// kUWorkersPerStage workers per stage: chunk c goes to warps c % kUStages + h
+// kUStages, so every wait on a stage's barriers comes from those warps, each in
+// chunk order, at most one phase ahead of the barrier (a
+// parity wait two phases early would pass at once).  The descriptor ring is at
+// least as deep as the stage count for the same reason.
+static_assert(kUWorkers == kUStages * kUWorkersPerStage && kUUnions % kUWorkersPerStage == 0 &&
+                  kURing >= kUStages,
+              "a fixed set of workers per stage, an equal share of the unions each");
 static_assert(kUEpiWarp0 % 4 == 0 && kUEpiWarp0 + 4 <= kUWarps && kUSchedWarp >= kUWorkers &&
                   kUSchedWarp < kUWarps && kUMmaWarp >= kUWorkers && kUMmaWarp < kUWarps &&
                   kUSchedWarp != kUMmaWarp && (kUMmaWarp < kUEpiWarp0 || kUMmaWarp >= kUEpiWarp0 + 4) &&
@@ -163,12 +168,12 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
 
   if (tid == 0) {
     for (int s = 0; s < kUStages; ++s) {
-      mbar_init(sbase + kUBarFull + 8 * s, 1);   // the worker warp that filled the stage
+      mbar_init(sbase + kUBarFull + 8 * s, kUWorkersPerStage);  // the worker warps that filled the stage
       mbar_init(sbase + kUBarEmpty + 8 * s, 1);  // the MMAs that read it
     }
     for (int r = 0; r < kURing; ++r) {
       mbar_init(sbase + kUBarRingFull + 8 * r, 1);   // the scheduler wrote the descriptor
-      mbar_init(sbase + kUBarRingEmpty + 8 * r, 1);  // its worker read it
+      mbar_init(sbase + kUBarRingEmpty + 8 * r, kUWorkersPerStage);  // its workers read it
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(sbase + kUBarAccFull + 8 * b, 2);   // MMA completion + the issuing thread's descriptor arrival
@@ -197,19 +202,26 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
 
   if (warp < kUWorkers) {
     // ------------------------------------------------------------ workers
-    // Warp w fills chunks w, w + 6, w + 12, ... on its own: it takes the chunk's
-    // descriptor from the scheduler's ring, waits for the chunk's stage to be
-    // free, zeroes A, gathers the 48 Q (or dO) rows of the chunk's 4 unions into
-    // B with cp.async, stores each union's records into the A rows of their keys,
-    // waits for its copies and marks the stage full.  Up to kUStages chunks are
-    // in flight at once, one per warp, with no barrier between warps.
+    // Warps s + 6 h (h < kUWorkersPerStage) fill chunks s, s + 6, s + 12, ...
+    // together, each taking kMy of the chunk's unions: each takes the chunk's descriptor from
+    // the scheduler's ring, waits for the chunk's stage to be free, clears its
+    // unions' A slots, gathers their 24 Q (or dO) rows into B with cp.async,
+    // stores their records into the A rows of their keys, waits for its copies
+    // and arrives on the stage's full barrier (complete when all have).  Up to
+    // kUStages chunks are in flight at once, with no barrier between stages.
+    const int s = warp % kUStages, half = warp / kUStages;
+    constexpr int kMy = kUUnions / kUWorkersPerStage;  // unions per warp
+    const int u0 = kMy * half;                         // this warp's first union of a chunk
     // A rows this lane wrote in the warp's previous chunk (its stage still holds
-    // them): clearing those 24-byte slots restores an all-zero A without
-    // rewriting the 12 KB tile; the whole tile is zeroed on the stage's first
-    // use and after a chunk whose records were not all tracked (runs > 32 keys)
-    int prev_m[kUUnions] = {-1, -1, -1, -1};
+    // them): clearing those 24-byte slots restores zeros in this warp's unions'
+    // columns without rewriting the tile; they are cleared for all 128 rows on
+    // the stage's first use and after a chunk whose records were not all tracked
+    // (runs > 32 keys)
+    int prev_m[kMy];
+#pragma unroll
+    for (int j = 0; j < kMy; ++j) prev_m[j] = -1;
     bool zero_all = true;
-    for (int c = warp;; c += kUWorkers) {
+    for (int c = s;; c += kUStages) {
       const int rs = c % kURing;
       bool got = true;
       if (lane == 0) got = u_wait(sbase + kUBarRingFull + 8 * rs, (c / kURing) & 1, abort_flag);
@@ -217,31 +229,30 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
       __syncwarp();  // every lane reads the descriptor after lane 0 saw it published
       const volatile int* hv = reinterpret_cast<const volatile int*>(ring + 48 * rs);
       const int4 hd = make_int4(hv[0], hv[1], hv[2], hv[3]);
-      int64_t e[kUUnions];
+      int64_t e[kMy];
 #pragma unroll
-      for (int u = 0; u < kUUnions; ++u) e[u] = reinterpret_cast<const volatile int64_t*>(ring + 48 * rs + 16)[u];
+      for (int j = 0; j < kMy; ++j) e[j] = reinterpret_cast<const volatile int64_t*>(ring + 48 * rs + 16)[u0 + j];
       __syncwarp();
       if (lane == 0) mbar_arrive(sbase + kUBarRingEmpty + 8 * rs);
-      const int s = c % kUStages;
       const bool end = hd.x < 0;
-      if (end && hd.y == 0) break;  // an end marker for a warp whose chunk the MMA never reaches
+      if (end && hd.y == 0) break;  // an end marker for a stage whose chunk the MMA never reaches
       const int n = hd.z & 255, r = hd.z >> 10, g = r >> 1, tensor = r & 1, tile = hd.w;
-      // the records and keys of the chunk's unions (j < 32), loaded first so that
-      // their latency overlaps the wait for the stage, the zeroing and the row
-      // gather; record j of union u goes to A row (key - tile base), K columns
-      // 12 u .. 12 u + 11 (dK takes the record's dS half, dV its P half)
+      // the records and keys of this warp's unions (j < 32), loaded first so
+      // that their latency overlaps the wait for the stage, the clearing and the
+      // row gather; record j of union u goes to A row (key - tile base), K
+      // columns 12 u .. 12 u + 11 (dK takes the record's dS half, dV its P half)
       const int key0 = tile * kUKeys;
-      int32_t key[kUUnions];
-      uint2 val[kUUnions][3];
+      int32_t key[kMy];
+      uint2 val[kMy][3];
 #pragma unroll
-      for (int u = 0; u < kUUnions; ++u) {
-        const int64_t t = e[u] >> 32;
-        const int i0 = static_cast<int>((e[u] >> 8) & 0x3fff), cnt = static_cast<int>(e[u] & 0x7f) + 1;
-        const bool ok_j = u < n && lane < cnt;
+      for (int j = 0; j < kMy; ++j) {
+        const int64_t t = e[j] >> 32;
+        const int i0 = static_cast<int>((e[j] >> 8) & 0x3fff), cnt = static_cast<int>(e[j] & 0x7f) + 1;
+        const bool ok_j = u0 + j < n && lane < cnt;
         const uint2* rec = reinterpret_cast<const uint2*>(pds + ((t * G + g) * n_sel + i0) * kURec) + (tensor ? 0 : 3);
-        key[u] = ok_j ? __ldg(row_cols + t * n_sel + i0 + lane) : -1;
+        key[j] = ok_j ? __ldg(row_cols + t * n_sel + i0 + lane) : -1;
 #pragma unroll
-        for (int hq = 0; hq < 3; ++hq) val[u][hq] = ok_j ? __ldg(rec + lane * 6 + hq) : make_uint2(0, 0);
+        for (int hq = 0; hq < 3; ++hq) val[j][hq] = ok_j ? __ldg(rec + lane * 6 + hq) : make_uint2(0, 0);
       }
       // stage s is free once the MMAs of chunk c - kUStages completed
       if (c >= kUStages) {
@@ -251,7 +262,7 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
       const uint32_t st = sbase + s * kUStage;
       if (end) {  // the first chunk past the last unit: end marker for the MMA warp
         if (lane == 0) {
-          desc[s] = make_int4(0, -1, 0, 0);
+          if (half == 0) desc[s] = make_int4(0, -1, 0, 0);
           mbar_arrive(sbase + kUBarFull + 8 * s);
         }
         break;
@@ -263,35 +274,37 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
         return reinterpret_cast<uint2*>(abase + (m >> 3) * kUASbo + (m & 7) * 16 + (kk >> 3) * 128 + (kk & 7) * 2);
       };
       if (zero_all) {
-        uint4* a = reinterpret_cast<uint4*>(abase);
 #pragma unroll 4
-        for (int i = lane; i < kUABytes / 16; i += 32) a[i] = make_uint4(0, 0, 0, 0);
+        for (int i = lane; i < kMy * kUKeys * 3; i += 32) {
+          const int j = i / (kUKeys * 3), rem = i - j * (kUKeys * 3);
+          *slot(u0 + j, rem / 3, rem % 3) = make_uint2(0, 0);
+        }
       } else {
 #pragma unroll
-        for (int u = 0; u < kUUnions; ++u)
-          if (prev_m[u] >= 0) {
+        for (int j = 0; j < kMy; ++j)
+          if (prev_m[j] >= 0) {
 #pragma unroll
-            for (int hq = 0; hq < 3; ++hq) *slot(u, prev_m[u], hq) = make_uint2(0, 0);
+            for (int hq = 0; hq < 3; ++hq) *slot(u0 + j, prev_m[j], hq) = make_uint2(0, 0);
           }
       }
-      // B: the 12 head rows of each union (zero-filled for missing unions)
+      // B: the 12 head rows of each of this warp's unions (zero-filled for missing unions)
       {
         const __nv_bfloat16* base = (tensor ? dout : q) + (g * kHeadsPerGroup * kHeadDim + lane * 8);
         const uint32_t dst = st + (lane >> 3) * kUBBlk;
         const int unit = lane & 7;
 #pragma unroll
-        for (int u = 0; u < kUUnions; ++u) {
-          const bool mine = u < n;
-          const __nv_bfloat16* src = base + (mine ? (e[u] >> 32) : 0) * H * kHeadDim;
+        for (int j = 0; j < kMy; ++j) {
+          const bool mine = u0 + j < n;
+          const __nv_bfloat16* src = base + (mine ? (e[j] >> 32) : 0) * H * kHeadDim;
 #pragma unroll
           for (int h = 0; h < kHeadsPerGroup; ++h) {
-            const int kr = u * kHeadsPerGroup + h;
+            const int kr = (u0 + j) * kHeadsPerGroup + h;
             cp_async16(dst + kr * 128 + ((unit ^ (kr & 7)) << 4), src + h * kHeadDim, mine);
           }
         }
       }
       cp_async_commit();
-      __syncwarp();  // the zeroing above before the record stores below
+      __syncwarp();  // the clearing above before the record stores below
       // stores record j of union u; returns its A row, or -1
       auto put = [&](int u, int32_t k, const uint2 (&v)[3]) -> int {
         const int m = k - key0;
@@ -301,25 +314,26 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
         return m;
       };
 #pragma unroll
-      for (int u = 0; u < kUUnions; ++u) prev_m[u] = put(u, key[u], val[u]);
+      for (int j = 0; j < kMy; ++j) prev_m[j] = put(u0 + j, key[j], val[j]);
       // unions with more than 32 keys in the tile (rare for sparse routes); their
-      // extra rows are not tracked, so the next chunk of this stage zeroes A
+      // extra rows are not tracked, so the next chunk of this stage clears all
+      // of this warp's slots
       zero_all = false;
 #pragma unroll
-      for (int u = 0; u < kUUnions; ++u) {
-        const int64_t t = e[u] >> 32;
-        const int i0 = static_cast<int>((e[u] >> 8) & 0x3fff), cnt = static_cast<int>(e[u] & 0x7f) + 1;
-        if (u >= n || cnt <= 32) continue;
+      for (int j = 0; j < kMy; ++j) {
+        const int64_t t = e[j] >> 32;
+        const int i0 = static_cast<int>((e[j] >> 8) & 0x3fff), cnt = static_cast<int>(e[j] & 0x7f) + 1;
+        if (u0 + j >= n || cnt <= 32) continue;
         zero_all = true;
         const uint2* rec = reinterpret_cast<const uint2*>(pds + ((t * G + g) * n_sel + i0) * kURec) + (tensor ? 0 : 3);
-        for (int j = lane + 32; j < cnt; j += 32) {
-          const uint2 v[3] = {__ldg(rec + j * 6), __ldg(rec + j * 6 + 1), __ldg(rec + j * 6 + 2)};
-          put(u, __ldg(row_cols + t * n_sel + i0 + j), v);
+        for (int jj = lane + 32; jj < cnt; jj += 32) {
+          const uint2 v[3] = {__ldg(rec + jj * 6), __ldg(rec + jj * 6 + 1), __ldg(rec + jj * 6 + 2)};
+          put(u0 + j, __ldg(row_cols + t * n_sel + i0 + jj), v);
         }
       }
-      if (lane == 0) desc[s] = make_int4(hd.x, n, (hd.z >> 8) & 3, r);
-      // the stage is complete once this warp's copies landed: make it visible to
-      // the tensor cores, mark it full
+      if (half == 0 && lane == 0) desc[s] = make_int4(hd.x, n, (hd.z >> 8) & 3, r);
+      // this warp's part of the stage is complete once its copies landed: make
+      // it visible to the tensor cores, arrive on the stage's full barrier
       cp_async_wait<0>();
       fence_proxy_async();
       __syncwarp();
@@ -379,7 +393,10 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
     const bool leader = quarter == 0 && lane == 0;
     for (int useq = 0;; ++useq) {
       const int buf = useq % kUAccBufs;
-      if (!u_wait(sbase + kUBarAccFull + 8 * buf, (useq / kUAccBufs) & 1, abort_flag)) break;
+      // the four warps leave together: one warp whose wait expired must not
+      // leave the others in the named barriers below
+      const bool got = u_wait(sbase + kUBarAccFull + 8 * buf, (useq / kUAccBufs) & 1, abort_flag);
+      if (bar_or(3, 128, !got)) break;
       const int idx = acc_desc[buf].x, r = acc_desc[buf].y;
       if (idx < 0) break;
       asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
@@ -539,8 +556,8 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
       if (cur.x >= 0) claim(nxt, nxt_idx, nxt_r);
     }
     // end markers: chunk c (the first past the list) ends the MMA loop; each of
-    // the other workers gets one that only ends its own loop
-    for (int k = 0; ok && k < kUWorkers; ++k, ++c) {
+    // the other stages' worker pairs gets one that only ends their own loop
+    for (int k = 0; ok && k < kUStages; ++k, ++c) {
       const int rs = c % kURing;
       bool got = true;
       if (c >= kURing && lane == 0) got = u_wait(sbase + kUBarRingEmpty + 8 * rs, ((c / kURing) - 1) & 1, abort_flag);

@@ -30,20 +30,22 @@ cudaError_t launch_quad_sort(const int32_t* quad_ptr, int64_t n_quads, int64_t* 
                              int32_t* phase_ptr, cudaStream_t s);
 // The key->query transpose over 128-key tiles: one entry per (row, tile) pair,
 // (t << 32) | (i0 << 8) | (n - 1) with row_cols[t][i0, i0 + n) the row's keys in
-// the tile.  Count rows per tile (tile_cnt zeroed by the caller), fill
-// (unordered; tile_fill holds the scanned offsets), then sort each tile's list
-// by query and record its phase starts.
-cudaError_t launch_tile_count(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel,
-                              int64_t n_tiles, int32_t* tile_cnt, cudaStream_t s);
-cudaError_t launch_tile_fill(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel, int64_t n_tiles,
-                             int32_t* tile_fill, int64_t* tile_ent, cudaStream_t s);
-cudaError_t launch_tile_sort(const int32_t* tile_ptr, int64_t n_tiles, int64_t* tile_ent, int P, int C,
-                             int32_t* phase_ptr, cudaStream_t s);
+// the tile, every list in ascending query order without a sort: per block of 64
+// rows a mask of the rows meeting each tile, block bases from a scan down each
+// tile's column, ranks from mask popcounts.  `scratch` holds the masks and the
+// block bases (tile_lists_bytes); tile_cnt, tile_ptr (n_tiles + 1) and
+// tile_fill (n_tiles) are written.
+size_t tile_lists_bytes(int64_t T, int64_t T_kv);
+cudaError_t launch_tile_lists(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel,
+                              int64_t n_tiles, void* scratch, int32_t* tile_cnt, int32_t* tile_ptr,
+                              int32_t* tile_fill, int64_t* tile_ent, cudaStream_t s);
 // Per-phase work lists of non-empty (tile, entry range) items (wl_cnt zeroed by
-// the caller); zeroes dK/dV of tiles that no query routes to.
-cudaError_t launch_tile_worklist(const int32_t* tile_ptr, const int32_t* phase_ptr, int64_t n_tiles, int64_t T_kv,
-                                 int G, int P, int32_t* wl_cnt, int4* wl, void* dk, void* dv, bool f32_out,
-                                 cudaStream_t s);
+// the caller), phase p = rows [p C, (p + 1) C) with C a multiple of 64, its
+// start in a tile's list read from the block bases in `scratch` (written by
+// launch_tile_lists); zeroes dK/dV of tiles that no query routes to.
+cudaError_t launch_tile_worklist(const int32_t* tile_ptr, const void* scratch, int64_t T, int64_t n_tiles,
+                                 int64_t T_kv, int G, int P, int C, int32_t* wl_cnt, int4* wl, void* dk, void* dv,
+                                 bool f32_out, cudaStream_t s);
 
 // Attention kernels (qsa_forward.cu, qsa_backward.cu, qsa_dkdv_union.cu).
 cudaError_t launch_forward(const void* q, const void* k, const void* v, const int32_t* row_cnt,
@@ -68,6 +70,10 @@ cudaError_t launch_backward_dkdv_union(const void* grad_out, const void* q, cons
                                        const int4* wl, int* claim_ctr, int* done, int P, int64_t n_tiles,
                                        int64_t T_kv, int G, int n_sel, float scale, float* partial, void* dk, void* dv,
                                        bool f32_out, int* status, cudaStream_t s);
+
+// FP32 -> BF16 (round to nearest even) of n contiguous values (qsa_cast.cu);
+// x and y 16-byte aligned.
+cudaError_t launch_cast_f32_bf16(const float* x, void* y, int64_t n, cudaStream_t s);
 
 // Bitmap selection -> route IDs (qsa_bitmap.cu); zeroes *max_cnt first when given.
 cudaError_t launch_bitmap_routes(const uint8_t* sel, const int32_t* lo, const int32_t* hi, const int32_t* blk_base,

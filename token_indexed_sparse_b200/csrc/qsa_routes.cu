@@ -7,7 +7,7 @@
 //     per-query forward and dQ kernels,
 //   * the key->query transpose over aligned 128-key tiles (tile_ptr, tile_ent:
 //     one entry per (row, tile) naming the row's run of keys in the tile), each
-//     list in ascending query order with its query-phase starts, and the
+//     list written directly in ascending query order (no sort), and the
 //     per-phase work lists the dK/dV kernel claims its units from, and
 //   * the same transpose over aligned key quads with 4-bit owner masks
 //     (quad_ptr, quad_ent), exposed by qsa_route_plan.
@@ -372,25 +372,28 @@ __global__ void __launch_bounds__(kSortThreads) quad_sort_kernel(const int32_t* 
 // keys inside the tile (ascending, so one contiguous run of the sorted row).
 constexpr int kTileShift = 7;
 
-// Rows are taken rows_per_warp per warp (8 warps per block).  With at most
-// kTileBins tiles the block first gathers its per-tile counts in shared memory
-// and touches each global counter once, so rows that meet the same tiles do not
-// contend on one global address per row.
+// Rows come in blocks of 64 (kBlockRows).  Per block and tile, a 64-bit mask of
+// the block's rows that meet the tile; a scan down each tile's column of mask
+// popcounts gives every block its first slot in the tile's list; an entry's
+// place inside its block is the popcount of the mask below its row.  So every
+// (row, tile) entry is written straight to its place in ascending query order,
+// with no sort and no atomics on the list, and a query phase (a multiple of 64
+// rows) starts at a block's first slot.  With at most kTileBins tiles a block
+// builds its masks in shared memory and writes each one once.
+constexpr int kBlockRows = 64;
 constexpr int kTileBins = 8192;
 
-// Rows per warp: 8 for rows of up to 1024 slots, else 2 (long rows already give
-// a warp enough work, and more blocks keep more loads in flight).
-inline int tile_rows_per_warp(int n_sel) { return n_sel <= 1024 ? 8 : 2; }
-
 // Calls f(t, cols, cnt, tile, i) for every i where row t's sorted keys enter a
-// new tile.  A warp reads its row 32 keys at a time, the previous key of each
-// lane coming from its neighbour.
+// new tile, for the 64 rows of block blockIdx.x spread over the CTA's warps.  A
+// warp reads its row 32 keys at a time, the previous key of each lane coming
+// from its neighbour.
 template <typename F>
-__device__ __forceinline__ void for_tile_runs(const int32_t* __restrict__ row_cnt, const int32_t* __restrict__ row_cols,
-                                              int64_t T, int n_sel, int rows_per_warp, F f) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t t0 = (static_cast<int64_t>(blockIdx.x) * 8 + warp) * rows_per_warp;
-  for (int r = 0; r < rows_per_warp; ++r) {
+__device__ __forceinline__ void for_block_runs(const int32_t* __restrict__ row_cnt,
+                                               const int32_t* __restrict__ row_cols, int64_t T, int n_sel, F f) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int rpw = kBlockRows / nw;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kBlockRows + static_cast<int64_t>(warp) * rpw;
+  for (int r = 0; r < rpw; ++r) {
     const int64_t t = t0 + r;
     if (t >= T) return;
     const int cnt = row_cnt[t];
@@ -407,50 +410,58 @@ __device__ __forceinline__ void for_tile_runs(const int32_t* __restrict__ row_cn
   }
 }
 
-// Rows per 128-key tile (tile_cnt zeroed by the caller).
-__global__ void __launch_bounds__(256) tile_count_kernel(const int32_t* __restrict__ row_cnt,
-                                                         const int32_t* __restrict__ row_cols, int64_t T, int n_sel,
-                                                         int rows_per_warp, int64_t n_tiles,
-                                                         int32_t* __restrict__ tile_cnt) {
-  extern __shared__ int32_t hist[];
+// masks[block * n_tiles + tile]: bit (t mod 64) set when row t meets the tile
+// (zeroed by the caller when n_tiles > kTileBins).
+__global__ void __launch_bounds__(512) tile_mask_kernel(const int32_t* __restrict__ row_cnt,
+                                                        const int32_t* __restrict__ row_cols, int64_t T, int n_sel,
+                                                        int64_t n_tiles, unsigned long long* __restrict__ masks) {
+  extern __shared__ unsigned long long msk[];
   const bool local = n_tiles <= kTileBins;
   if (local) {
-    for (int b = threadIdx.x; b < n_tiles; b += blockDim.x) hist[b] = 0;
+    for (int64_t j = threadIdx.x; j < n_tiles; j += blockDim.x) msk[j] = 0ull;
     __syncthreads();
   }
-  for_tile_runs(row_cnt, row_cols, T, n_sel, rows_per_warp, [&](int64_t, const int32_t*, int, int32_t tl, int) {
-    atomicAdd(local ? hist + tl : tile_cnt + tl, 1);
+  unsigned long long* dst = masks + static_cast<int64_t>(blockIdx.x) * n_tiles;
+  for_block_runs(row_cnt, row_cols, T, n_sel, [&](int64_t t, const int32_t*, int, int32_t tl, int) {
+    atomicOr(local ? msk + tl : dst + tl, 1ull << (t & 63));
   });
   if (!local) return;
   __syncthreads();
-  for (int b = threadIdx.x; b < n_tiles; b += blockDim.x)
-    if (hist[b]) atomicAdd(tile_cnt + b, hist[b]);
+  for (int64_t j = threadIdx.x; j < n_tiles; j += blockDim.x) dst[j] = msk[j];
 }
 
-// One entry per (row, tile) run: (t << 32) | (i0 << 8) | (n - 1), at a slot
-// reserved from the tile's fill cursor (list order is fixed later by the sort).
-__global__ void __launch_bounds__(256) tile_fill_kernel(const int32_t* __restrict__ row_cnt,
-                                                        const int32_t* __restrict__ row_cols, int64_t T,
-                                                        int n_sel, int rows_per_warp, int64_t n_tiles,
-                                                        int32_t* __restrict__ fill, int64_t* __restrict__ ent) {
-  extern __shared__ int32_t tsh[];  // [n_tiles] counts / cursors, [n_tiles] reserved bases
-  const bool local = n_tiles <= kTileBins;
-  int32_t* cnt = tsh;
-  int32_t* base = tsh + (local ? n_tiles : 0);
-  if (local) {
-    for (int b = threadIdx.x; b < n_tiles; b += blockDim.x) cnt[b] = 0;
-    __syncthreads();
-    for_tile_runs(row_cnt, row_cols, T, n_sel, rows_per_warp,
-                  [&](int64_t, const int32_t*, int, int32_t tl, int) { atomicAdd(cnt + tl, 1); });
-    __syncthreads();
-    for (int b = threadIdx.x; b < n_tiles; b += blockDim.x) {
-      if (cnt[b]) base[b] = atomicAdd(fill + b, cnt[b]);
-      cnt[b] = 0;
+// One warp per tile: exclusive scan of the blocks' mask popcounts down the
+// tile's column (blk_base), and the tile's row count.
+__global__ void __launch_bounds__(256) tile_scan_kernel(const unsigned long long* __restrict__ masks, int64_t n_blocks,
+                                                        int64_t n_tiles, int32_t* __restrict__ blk_base,
+                                                        int32_t* __restrict__ tile_cnt) {
+  const int lane = threadIdx.x & 31;
+  const int64_t j = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (j >= n_tiles) return;
+  int carry = 0;
+  for (int64_t b0 = 0; b0 < n_blocks; b0 += 32) {
+    const int64_t b = b0 + lane;
+    const int c = b < n_blocks ? __popcll(masks[b * n_tiles + j]) : 0;
+    int x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
-    __syncthreads();
+    if (b < n_blocks) blk_base[b * n_tiles + j] = carry + x - c;
+    carry += __shfl_sync(0xffffffffu, x, 31);
   }
-  for_tile_runs(row_cnt, row_cols, T, n_sel, rows_per_warp,
-                [&](int64_t t, const int32_t* cols, int n, int32_t tl, int i) {
+  if (lane == 0) tile_cnt[j] = carry;
+}
+
+// One entry per (row, tile) run, (t << 32) | (i0 << 8) | (n - 1), at
+// ptr[tile] + blk_base[block, tile] + (rows of the block below t that meet the tile).
+__global__ void __launch_bounds__(512) tile_fill_kernel(const int32_t* __restrict__ row_cnt,
+                                                        const int32_t* __restrict__ row_cols, int64_t T, int n_sel,
+                                                        int64_t n_tiles, const unsigned long long* __restrict__ masks,
+                                                        const int32_t* __restrict__ blk_base,
+                                                        const int32_t* __restrict__ ptr, int64_t* __restrict__ ent) {
+  for_block_runs(row_cnt, row_cols, T, n_sel, [&](int64_t t, const int32_t* cols, int n, int32_t tl, int i) {
     // the run ends at the first key of a later tile; a tile holds at most 128
     // distinct keys, so it ends within [i + 1, i + 128]
     int lo = i + 1, hi = min(n, i + 128);
@@ -459,86 +470,11 @@ __global__ void __launch_bounds__(256) tile_fill_kernel(const int32_t* __restric
       if ((cols[mid] >> kTileShift) > tl) hi = mid;
       else lo = mid + 1;
     }
-    const int p = local ? base[tl] + atomicAdd(cnt + tl, 1) : atomicAdd(fill + tl, 1);
+    const int64_t cell = (t >> 6) * n_tiles + tl;
+    const unsigned long long below = masks[cell] & ((1ull << (t & 63)) - 1ull);
+    const int64_t p = static_cast<int64_t>(ptr[tl]) + blk_base[cell] + __popcll(below);
     ent[p] = (t << 32) | (static_cast<int64_t>(i) << 8) | static_cast<int64_t>(lo - i - 1);
   });
-}
-
-// One block per tile: sort its list ascending (by query), then record where each
-// query phase starts in it (phase_ptr[tile * (P + 1) + p]).  Lists of up to
-// `cap` entries are sorted in shared memory; longer ones run the same network
-// with all comparators inside a `cap`-sized piece in shared memory and only the
-// longer-distance ones in global memory.
-__global__ void __launch_bounds__(1024) tile_sort_kernel(const int32_t* __restrict__ ptr, int64_t* __restrict__ ent,
-                                                         int P, int C, int cap, int32_t* __restrict__ phase_ptr) {
-  extern __shared__ int64_t tsv[];
-  const int64_t b = blockIdx.x;
-  const int lo = ptr[b], len = ptr[b + 1] - lo;
-  int32_t* pp = phase_ptr + b * (P + 1);
-  int64_t* seg = ent + lo;
-  if (len <= 1) {
-    for (int p = threadIdx.x; p <= P; p += blockDim.x)
-      pp[p] = lo + ((len == 1 && (seg[0] >> 32) < static_cast<int64_t>(p) * C) ? 1 : 0);
-    return;
-  }
-  int n2 = 1;
-  while (n2 < len) n2 <<= 1;
-  if (n2 <= cap) {
-    for (int i = threadIdx.x; i < n2; i += blockDim.x) tsv[i] = i < len ? seg[i] : LLONG_MAX;
-    __syncthreads();
-    block_sort<int64_t>(tsv, n2, n2);
-    for (int i = threadIdx.x; i < len; i += blockDim.x) seg[i] = tsv[i];
-    for (int p = threadIdx.x; p <= P; p += blockDim.x)
-      pp[p] = lo + lower_bound_query(tsv, len, static_cast<int64_t>(p) * C);
-  } else {
-    // the same bitonic network, in `cap`-sized pieces: every comparator whose
-    // two elements lie in one aligned piece runs in shared memory (a piece is
-    // loaded, +infinity past `len`, and written back), only the comparators of
-    // the levels above `cap` with distance >= cap run in global memory
-    auto piece = [&](int c0, bool full_sort, int h_top) {
-      for (int i = threadIdx.x; i < cap; i += blockDim.x) tsv[i] = c0 + i < len ? seg[c0 + i] : LLONG_MAX;
-      __syncthreads();
-      if (full_sort) {
-        block_sort<int64_t>(tsv, cap, cap);
-      } else {
-        for (int h = h_top; h >= 1; h >>= 1) {
-          for (int q = threadIdx.x; q < cap / 2; q += blockDim.x) {
-            const int i = (q / h) * 2 * h + (q % h), j = i + h;
-            const int64_t a = tsv[i], c = tsv[j];
-            if (c < a) { tsv[i] = c; tsv[j] = a; }
-          }
-          __syncthreads();
-        }
-      }
-      for (int i = threadIdx.x; i < cap && c0 + i < len; i += blockDim.x) seg[c0 + i] = tsv[i];
-      __syncthreads();
-    };
-    for (int c0 = 0; c0 < len; c0 += cap) piece(c0, true, 0);
-    for (int k = 2 * cap; k <= n2; k <<= 1) {
-      for (int q = threadIdx.x; q < n2 / 2; q += blockDim.x) {  // flip step of level k
-        const int off = q & (k / 2 - 1), base = (q / (k / 2)) * k;
-        const int i = base + off, j = base + k - 1 - off;
-        if (j < len) {
-          const int64_t a = seg[i], c = seg[j];
-          if (c < a) { seg[i] = c; seg[j] = a; }
-        }
-      }
-      __syncthreads();
-      for (int h = k / 4; h >= cap; h >>= 1) {  // half-cleaners across pieces
-        for (int q = threadIdx.x; q < n2 / 2; q += blockDim.x) {
-          const int i = (q / h) * 2 * h + (q % h), j = i + h;
-          if (j < len) {
-            const int64_t a = seg[i], c = seg[j];
-            if (c < a) { seg[i] = c; seg[j] = a; }
-          }
-        }
-        __syncthreads();
-      }
-      for (int c0 = 0; c0 < len; c0 += cap) piece(c0, false, cap / 2);
-    }
-    for (int p = threadIdx.x; p <= P; p += blockDim.x)
-      pp[p] = lo + lower_bound_query(seg, len, static_cast<int64_t>(p) * C);
-  }
 }
 
 // One warp per tile: lane 0 appends the tile's non-empty phase ranges to the
@@ -548,9 +484,9 @@ __global__ void __launch_bounds__(1024) tile_sort_kernel(const int32_t* __restri
 // the tile's accumulation order).  A tile that no query routes to gets its
 // dK/dV rows zeroed by the warp.
 __global__ void __launch_bounds__(256) tile_worklist_kernel(
-    const int32_t* __restrict__ ptr, const int32_t* __restrict__ phase_ptr, int64_t n_tiles, int64_t T_kv, int G,
-    int P, int32_t* __restrict__ wl_cnt, int4* __restrict__ wl, uint8_t* __restrict__ dk, uint8_t* __restrict__ dv,
-    int out_bytes) {
+    const int32_t* __restrict__ ptr, const int32_t* __restrict__ blk_base, int64_t n_blocks, int64_t n_tiles,
+    int64_t T_kv, int G, int P, int C, int32_t* __restrict__ wl_cnt, int4* __restrict__ wl, uint8_t* __restrict__ dk,
+    uint8_t* __restrict__ dv, int out_bytes) {
   const int lane = threadIdx.x & 31;
   const int64_t b = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (b >= n_tiles) return;
@@ -564,10 +500,15 @@ __global__ void __launch_bounds__(256) tile_worklist_kernel(
     return;
   }
   if (lane != 0) return;
-  const int32_t* pp = phase_ptr + b * (P + 1);
+  // phase p (rows p C .. (p + 1) C - 1, C a multiple of 64) starts at the first
+  // slot of block p C / 64 in the tile's list
+  auto start = [&](int p) {
+    const int64_t blk = static_cast<int64_t>(p) * C / kBlockRows;
+    return q0 + (blk < n_blocks ? blk_base[blk * n_tiles + b] : q1 - q0);
+  };
   int ord = 0;
   for (int p = 0; p < P; ++p) {
-    const int lo = pp[p], hi = pp[p + 1];
+    const int lo = start(p), hi = start(p + 1);
     if (hi > lo) {
       const int slot = atomicAdd(wl_cnt + p, 1);
       wl[static_cast<int64_t>(p) * n_tiles + slot] =
@@ -633,46 +574,48 @@ cudaError_t launch_quad_sort(const int32_t* quad_ptr, int64_t n_quads, int64_t* 
   return cudaGetLastError();
 }
 
-cudaError_t launch_tile_count(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel,
-                              int64_t n_tiles, int32_t* tile_cnt, cudaStream_t s) {
-  const int rpw = tile_rows_per_warp(n_sel);
-  const int64_t blocks = (T + 8 * rpw - 1) / (8 * rpw);
-  const size_t smem = n_tiles <= kTileBins ? static_cast<size_t>(n_tiles) * 4 : 0;
-  tile_count_kernel<<<static_cast<unsigned>(blocks), 256, smem, s>>>(row_cnt, row_cols, T, n_sel, rpw, n_tiles,
-                                                                     tile_cnt);
-  return cudaGetLastError();
+size_t tile_lists_bytes(int64_t T, int64_t T_kv) {
+  const size_t nb = static_cast<size_t>((T + kBlockRows - 1) / kBlockRows);
+  const size_t nt = static_cast<size_t>((T_kv + 127) / 128);
+  return nb * nt * 12;  // a mask (8 bytes) and a block base (4 bytes) per (block, tile)
 }
 
-cudaError_t launch_tile_fill(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel, int64_t n_tiles,
-                             int32_t* tile_fill, int64_t* tile_ent, cudaStream_t s) {
-  const int rpw = tile_rows_per_warp(n_sel);
-  const int64_t blocks = (T + 8 * rpw - 1) / (8 * rpw);
-  const size_t smem = n_tiles <= kTileBins ? static_cast<size_t>(n_tiles) * 8 : 0;
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(tile_fill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
+cudaError_t launch_tile_lists(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel,
+                              int64_t n_tiles, void* scratch, int32_t* tile_cnt, int32_t* tile_ptr,
+                              int32_t* tile_fill, int64_t* tile_ent, cudaStream_t s) {
+  const int64_t nb = (T + kBlockRows - 1) / kBlockRows;
+  auto* masks = static_cast<unsigned long long*>(scratch);
+  auto* blk_base = reinterpret_cast<int32_t*>(masks + nb * n_tiles);
+  const int threads = n_sel <= 1024 ? 256 : 512;  // 8 rows per warp, or 4 for long rows
+  const bool local = n_tiles <= kTileBins;
+  cudaError_t e;
+  if (!local) {
+    e = cudaMemsetAsync(masks, 0, static_cast<size_t>(nb * n_tiles) * 8, s);
+  } else {
+    e = cudaFuncSetAttribute(tile_mask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kTileBins * 8));
   }
-  tile_fill_kernel<<<static_cast<unsigned>(blocks), 256, smem, s>>>(row_cnt, row_cols, T, n_sel, rpw, n_tiles,
-                                                                    tile_fill, tile_ent);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_tile_sort(const int32_t* tile_ptr, int64_t n_tiles, int64_t* tile_ent, int P, int C,
-                             int32_t* phase_ptr, cudaStream_t s) {
-  constexpr int kCap = 16384;  // int64 entries sorted in shared memory (128 KB)
-  const int smem = kCap * static_cast<int>(sizeof(int64_t));
-  cudaError_t e = cudaFuncSetAttribute(tile_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  tile_sort_kernel<<<static_cast<unsigned>(n_tiles), 1024, smem, s>>>(tile_ptr, tile_ent, P, C, kCap, phase_ptr);
+  tile_mask_kernel<<<static_cast<unsigned>(nb), threads, local ? static_cast<size_t>(n_tiles) * 8 : 0, s>>>(
+      row_cnt, row_cols, T, n_sel, n_tiles, masks);
+  tile_scan_kernel<<<static_cast<unsigned>((n_tiles * 32 + 255) / 256), 256, 0, s>>>(masks, nb, n_tiles, blk_base,
+                                                                                    tile_cnt);
+  e = launch_quad_scan(tile_cnt, n_tiles, tile_ptr, tile_fill, s);
+  if (e != cudaSuccess) return e;
+  tile_fill_kernel<<<static_cast<unsigned>(nb), threads, 0, s>>>(row_cnt, row_cols, T, n_sel, n_tiles, masks,
+                                                                 blk_base, tile_ptr, tile_ent);
   return cudaGetLastError();
 }
 
-cudaError_t launch_tile_worklist(const int32_t* tile_ptr, const int32_t* phase_ptr, int64_t n_tiles, int64_t T_kv,
-                                 int G, int P, int32_t* wl_cnt, int4* wl, void* dk, void* dv, bool f32_out,
-                                 cudaStream_t s) {
+cudaError_t launch_tile_worklist(const int32_t* tile_ptr, const void* scratch, int64_t T, int64_t n_tiles,
+                                 int64_t T_kv, int G, int P, int C, int32_t* wl_cnt, int4* wl, void* dk, void* dv,
+                                 bool f32_out, cudaStream_t s) {
+  if (C % kBlockRows != 0) return cudaErrorInvalidValue;
+  const int64_t nb = (T + kBlockRows - 1) / kBlockRows;
+  const auto* blk_base =
+      reinterpret_cast<const int32_t*>(static_cast<const unsigned long long*>(scratch) + nb * n_tiles);
   tile_worklist_kernel<<<static_cast<unsigned>((n_tiles * 32 + 255) / 256), 256, 0, s>>>(
-      tile_ptr, phase_ptr, n_tiles, T_kv, G, P, wl_cnt, wl, static_cast<uint8_t*>(dk), static_cast<uint8_t*>(dv),
+      tile_ptr, blk_base, nb, n_tiles, T_kv, G, P, C, wl_cnt, wl, static_cast<uint8_t*>(dk), static_cast<uint8_t*>(dv),
       f32_out ? 4 : 2);
   return cudaGetLastError();
 }

@@ -73,6 +73,8 @@ def library() -> ctypes.CDLL:
     lib.qsa_tile_plan_scratch_size.argtypes = [i64, i64]
     lib.qsa_tile_plan.restype = i32
     lib.qsa_tile_plan.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp, vp, sz, vp]
+    lib.qsa_cast_f32_to_bf16.restype = i32
+    lib.qsa_cast_f32_to_bf16.argtypes = [vp, vp, i64, vp]
     _lib = lib
     return lib
 
@@ -190,7 +192,7 @@ def backward(grad_out, q, k, v, out, lse, routes, scale: float = 1.0 / 16.0, *,
              dq=None, dk=None, dv=None, workspace=None, stage_events=None, kv_fp32: bool = False):
     """qsa_backward: returns ``(dq, dk, dv)`` (bf16, shapes of q, k, v).
 
-    ``stage_events`` (optional, up to 6 torch.cuda.Event) are recorded after
+    ``stage_events`` (optional, up to 5 torch.cuda.Event) are recorded after
     each backward stage (qsa_backward_ex).  With ``kv_fp32`` dk and dv are FP32
     (qsa_backward_fp32kv: the sums before the BF16 rounding, for adding partials
     from several calls)."""
@@ -224,6 +226,21 @@ def backward(grad_out, q, k, v, out, lse, routes, scale: float = 1.0 / 16.0, *,
                                  _ptr(ws), ws.numel(), _stream(q.device), ev, n_ev)
     _check(st, "qsa_backward")
     return dq, dk, dv
+
+
+def cast_f32_to_bf16(x, out=None):
+    """qsa_cast_f32_to_bf16: ``x`` (FP32, CUDA) rounded to BF16, to nearest even.
+
+    The final rounding of FP32 dK/dV sums added up across calls (context
+    parallelism), the same rounding the backward applies itself."""
+    lib = library()
+    x = _prep(x, torch.float32, "x")
+    out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device) if out is None else \
+        _out(out, x.shape, torch.bfloat16, x.device, "out")
+    if x.data_ptr() % 16 or out.data_ptr() % 16:
+        raise ValueError("x and out must be 16-byte aligned")
+    _check(lib.qsa_cast_f32_to_bf16(_ptr(x), _ptr(out), x.numel(), _stream(x.device)), "qsa_cast_f32_to_bf16")
+    return out
 
 
 def route_plan(routes, T_kv: int):
