@@ -1,9 +1,9 @@
 """A model of the dK/dV kernel's synchronisation, run under random interleavings.
 
 ``dkdv_union_kernel`` (``csrc/qsa_dkdv_union.cu``) is a persistent kernel: per
-CTA a scheduler warp, gather warps (a fixed set per stage of a six-stage ring:
-one each as built, or two each taking half of a chunk's unions), one MMA
-thread and four epilogue warps hand chunks and accumulators to one
+CTA a scheduler warp, gather warps (a fixed set per stage of a three-stage
+ring: two each as built, each taking half of a chunk's unions, or one), one
+MMA thread and four epilogue warps hand chunks and accumulators to one
 another through mbarriers, and across CTAs each (tile, group, tensor) passes
 its FP32 partial from query phase to query phase through a counter in global
 memory.  This test restates that protocol as coroutines (one per warp role and
@@ -34,7 +34,7 @@ import random
 
 import pytest
 
-STAGES, RING, ACC_BUFS, UNIONS, HALVES = 6, 16, 2, 4, 2
+STAGES, RING, ACC_BUFS, UNIONS, HALVES = 3, 16, 2, 8, 2
 
 
 class Bar:
@@ -94,12 +94,13 @@ def make_units(rng, n_tiles, P, G):
 
 
 class Model:
-    """`n_workers` warps take the chunks in turn, chunk k to warp k % n_workers
-    (with 12 workers: two per stage, chunk k to the pair of stage k % 6);
+    """With `n_workers` = 2 x STAGES the pair of stage k % STAGES fills chunk k
+    (the kernel); otherwise `n_workers` warps take the chunks in turn, chunk k to
+    warp k % n_workers;
     `collective_exit=False` restates an earlier epilogue in which each warp left
     on its own accumulator wait."""
 
-    def __init__(self, units, n_ctas, seed, n_workers=STAGES, collective_exit=True, expire_at=None,
+    def __init__(self, units, n_ctas, seed, n_workers=STAGES * HALVES, collective_exit=True, expire_at=None,
                  expire_roles=""):
         self.rng = random.Random(seed)
         self.n_workers = n_workers
@@ -432,19 +433,20 @@ def test_the_model_catches_a_per_warp_epilogue_exit():
 
 
 def test_the_model_catches_workers_shared_between_stages():
-    # The first version let 8 gather warps take chunks in turn over 6 stages, so
-    # chunks k and k + 6 (one stage) could go to different warps and a warp
-    # could wait for "stage free" while the stage's barrier was still two phases
-    # behind; the hardware passes such a wait at once.  The model must flag it
-    # (an early pass, a stage overwritten under its MMA, or a stall).
+    # An early version let 8 gather warps take chunks in turn over 6 stages
+    # (here: 4 warps over 3), so chunks k and k + STAGES (one stage) could go to
+    # different warps and a warp could wait for "stage free" while the stage's
+    # barrier was still two phases behind; the hardware passes such a wait at
+    # once.  The model must flag it (an early pass, a stage overwritten under its
+    # MMA, or a stall).
     units = make_units(random.Random(3), 4, 4, 2)
     flagged = 0
     for seed in range(20):
         try:
-            Model(units, 1, seed, n_workers=8).run()
+            Model(units, 1, seed, n_workers=STAGES + 1).run()
         except AssertionError:
             flagged += 1
     assert flagged >= 15
     for seed in range(20):              # the kernel's design: a fixed set of warps per stage
         Model(units, 1, seed).run()
-        Model(units, 1, seed, n_workers=STAGES * HALVES).run()
+        Model(units, 1, seed, n_workers=STAGES).run()

@@ -8,23 +8,26 @@
 // the tile's transpose list for the phase: one entry per query row that routes
 // into the tile (its "union": the row's keys inside the tile, a contiguous run
 // of the sorted row), so a query's 12 Q (or dO) rows are gathered once per tile
-// however many of the tile's keys it selected.  Per chunk of 4 unions:
-//   D [128 keys x 256 dims] += A [128 keys x 48] . B [48 x 256 dims]
+// however many of the tile's keys it selected.  Per chunk of 8 unions:
+//   D [128 keys x 256 dims] += A [128 keys x 96] . B [96 x 256 dims]
 // with K row 12 u + h = head h of union u; A holds the BF16 dS (for dK) or P
 // (for dV) halves of the 48-byte records the dQ kernel wrote, zero where a
 // union did not select the key; B holds the gathered Q (or dO) rows.  That is
-// 3 tcgen05.mma kind::f16 (M 128, N 256, K 16), A K-major without swizzle, B
+// 6 tcgen05.mma kind::f16 (M 128, N 256, K 16), A K-major without swizzle, B
 // MN-major with the 128-byte swizzle, the accumulator in tensor memory (two
 // 256-column buffers, so the epilogue of one unit overlaps the next unit's MMAs).
+// Chunks of 8 unions rather than 4 halve the MMA thread's fixed cost per union
+// (seq32k: 7.3 -> 5.8 ms), at three 72 KB stages instead of six of 36 KB.
 //
 // Warp roles (384 threads): warp 6 schedules (claims units, cuts them into
-// chunks of 4 entries, publishes each chunk's descriptor in a shared-memory ring
-// and prefetches its records and keys into L2); warps 0-5 fill the chunks, warp
-// s every chunk of stage s of the 6-stage shared-memory ring (clear A, gather B
-// rows with cp.async, store the records into their A rows); warp 7 (one
-// thread) issues the MMAs; warps 8-11 (tensor-memory lane quarters 0-3) run the
-// epilogue, thread = key row.  The stage fill is written for kUWorkersPerStage
-// warps per stage, each taking an equal share of the chunk's unions.  Units are claimed from one counter in
+// chunks of 8 entries, publishes each chunk's descriptor in a shared-memory ring
+// and prefetches its records and keys into L2); warps 0-5 fill the chunks, warps
+// s and s + 3 every chunk of stage s of the 3-stage shared-memory ring, each
+// four of its unions (clear A, gather B rows with cp.async, store the records
+// into their A rows; a warp keeps only about eight 512-byte copies in flight,
+// so the rows of a chunk are split over two warps); warp 7 (one thread) issues
+// the MMAs; warps 8-11 (tensor-memory lane quarters 0-3) run the epilogue,
+// thread = key row.  Units are claimed from one counter in
 // phase order (phase 0's units, then phase 1's, ...; inside a phase every dK
 // unit before every dV unit), so the
 // CTAs work on about one phase and one tensor at a time and its Q (or dO) rows
@@ -47,30 +50,31 @@ namespace {
 // buffer, 512 per SM)
 constexpr int kUCtasPerSm = 1, kUAccBufs = 2;
 constexpr int kUTmemCols = 256 * kUAccBufs;
-constexpr int kUStages = 6;
-constexpr int kUWorkersPerStage = 1;                // (two per stage, each two unions: 7.16 -> 7.58 ms on seq32k)
+constexpr int kUStages = 3;
+constexpr int kUWorkersPerStage = 2;                // warps per stage, kUUnions / 2 unions each
 constexpr int kUWorkers = kUStages * kUWorkersPerStage;  // warps 0-5 fill chunks
 constexpr int kUSchedWarp = 6, kUMmaWarp = 7, kUEpiWarp0 = 8;
 constexpr int kUWarps = 12;
 constexpr int kUThreads = 32 * kUWarps;
 constexpr int kURec = 24;                           // bf16 per (t, g, key) record: 12 P + 12 dS
 constexpr int kUKeys = 128;                         // keys per tile (MMA M)
-constexpr int kUUnions = 4;                         // unions per chunk
-constexpr int kUK = kUUnions * kHeadsPerGroup;      // 48 K rows per chunk
-constexpr int kUBBlk = kUK * 128;                   // one 64-dim column block of B (6 KB)
-constexpr int kUBBytes = 4 * kUBBlk;                // 24 KB
+constexpr int kUUnions = 8;                         // unions per chunk
+constexpr int kUK = kUUnions * kHeadsPerGroup;      // 96 K rows per chunk
+constexpr int kUBBlk = kUK * 128;                   // one 64-dim column block of B (12 KB)
+constexpr int kUBBytes = 4 * kUBBlk;                // 48 KB
 constexpr int kUASbo = (kUK / 8) * 128;             // A: bytes between 8-key core-matrix rows (768)
-constexpr int kUABytes = kUKeys * kUK * 2;          // 12 KB
-constexpr int kUStage = kUBBytes + kUABytes;        // 36 KB
+constexpr int kUABytes = kUKeys * kUK * 2;          // 24 KB
+constexpr int kUStage = kUBBytes + kUABytes;        // 72 KB
 constexpr int kURing = 16;                          // chunk descriptors the scheduler may run ahead
 constexpr int kUOffCtl = kUStages * kUStage;
 // control block: stage descriptors, accumulator descriptors, the chunk ring
 // (header int4 + 4 list entries), phase prefix, barriers, tmem slot, abort flag
 constexpr int kUOffDesc = kUOffCtl;                          // kUStages x int4
 constexpr int kUOffAcc = kUOffDesc + kUStages * 16;          // 2 x int4
-constexpr int kUOffRing = kUOffAcc + 2 * 16;                 // kURing x 48 bytes
+constexpr int kURingSlot = 16 + 8 * kUUnions;                // header int4 + the chunk's entries
+constexpr int kUOffRing = kUOffAcc + 2 * 16;                 // kURing x kURingSlot bytes
 constexpr int kUMaxPhases = 64;
-constexpr int kUOffPref = kUOffRing + kURing * 48;           // kUMaxPhases + 1 ints: units before each phase
+constexpr int kUOffPref = kUOffRing + kURing * kURingSlot;   // kUMaxPhases + 1 ints: units before each phase
 constexpr int kUOffBar = (kUOffPref + 4 * (kUMaxPhases + 1) + 7) & ~7;
 constexpr int kUBarFull = kUOffBar, kUBarEmpty = kUBarFull + 8 * kUStages;
 constexpr int kUBarRingFull = kUBarEmpty + 8 * kUStages, kUBarRingEmpty = kUBarRingFull + 8 * kURing;
@@ -80,6 +84,8 @@ constexpr int kUOffTmem = kUBarDrain + 8, kUOffAbort = kUOffTmem + 4;
 constexpr int kUSmem = kUOffAbort + 4 + 1024;      // + alignment slack
 static_assert(kUStage % 1024 == 0, "stage alignment (128-byte swizzle atoms)");
 static_assert(kUSmem <= 232448, "shared memory per block");
+static_assert((kUUnions & (kUUnions - 1)) == 0 && 32 % kUUnions == 0 && kURingSlot % 16 == 0,
+              "chunks of a power-of-two number of unions, a divisor of the scheduler's 32-entry window");
 // kUWorkersPerStage workers per stage: chunk c goes to warps c % kUStages + h
 // kUStages, so every wait on a stage's barriers comes from those warps, each in
 // chunk order, at most one phase ahead of the barrier (a
@@ -164,7 +170,7 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kUOffAbort);
   int4* desc = reinterpret_cast<int4*>(smem + kUOffDesc);
   int4* acc_desc = reinterpret_cast<int4*>(smem + kUOffAcc);
-  uint8_t* ring = smem + kUOffRing;  // chunk c: header int4 at 48 (c % kURing), entries after it
+  uint8_t* ring = smem + kUOffRing;  // chunk c: header int4 at kURingSlot (c % kURing), entries after it
 
   if (tid == 0) {
     for (int s = 0; s < kUStages; ++s) {
@@ -227,11 +233,11 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
       if (lane == 0) got = u_wait(sbase + kUBarRingFull + 8 * rs, (c / kURing) & 1, abort_flag);
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       __syncwarp();  // every lane reads the descriptor after lane 0 saw it published
-      const volatile int* hv = reinterpret_cast<const volatile int*>(ring + 48 * rs);
+      const volatile int* hv = reinterpret_cast<const volatile int*>(ring + kURingSlot * rs);
       const int4 hd = make_int4(hv[0], hv[1], hv[2], hv[3]);
       int64_t e[kMy];
 #pragma unroll
-      for (int j = 0; j < kMy; ++j) e[j] = reinterpret_cast<const volatile int64_t*>(ring + 48 * rs + 16)[u0 + j];
+      for (int j = 0; j < kMy; ++j) e[j] = reinterpret_cast<const volatile int64_t*>(ring + kURingSlot * rs + 16)[u0 + j];
       __syncwarp();
       if (lane == 0) mbar_arrive(sbase + kUBarRingEmpty + 8 * rs);
       const bool end = hd.x < 0;
@@ -541,10 +547,10 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
             ok = false;
             break;
           }
-          const int64_t eu = __shfl_sync(0xffffffffu, el, (p - w0) + (lane & 3));
-          if (lane < kUUnions) reinterpret_cast<int64_t*>(ring + 48 * rs + 16)[lane] = lane < n ? eu : 0;
+          const int64_t eu = __shfl_sync(0xffffffffu, el, (p - w0) + (lane & (kUUnions - 1)));
+          if (lane < kUUnions) reinterpret_cast<int64_t*>(ring + kURingSlot * rs + 16)[lane] = lane < n ? eu : 0;
           const int flags = (p == cur.y ? kChFirst : 0) | (p + n >= cur.z ? kChLast : 0);
-          if (lane == 0) *reinterpret_cast<int4*>(ring + 48 * rs) = make_int4(cur_idx, p, n | (flags << 8) | (cur_r << 10), cur.x);
+          if (lane == 0) *reinterpret_cast<int4*>(ring + kURingSlot * rs) = make_int4(cur_idx, p, n | (flags << 8) | (cur_r << 10), cur.x);
           __syncwarp();
           if (lane == 0) mbar_arrive(sbase + kUBarRingFull + 8 * rs);
           ++c;
@@ -563,7 +569,7 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
       if (c >= kURing && lane == 0) got = u_wait(sbase + kUBarRingEmpty + 8 * rs, ((c / kURing) - 1) & 1, abort_flag);
       if (!__shfl_sync(0xffffffffu, got, 0)) break;
       if (lane == 0) {
-        *reinterpret_cast<int4*>(ring + 48 * rs) = make_int4(-1, k == 0 ? 1 : 0, 0, 0);
+        *reinterpret_cast<int4*>(ring + kURingSlot * rs) = make_int4(-1, k == 0 ? 1 : 0, 0, 0);
         mbar_arrive(sbase + kUBarRingFull + 8 * rs);
       }
     }

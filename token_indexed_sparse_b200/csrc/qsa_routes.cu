@@ -454,27 +454,56 @@ __global__ void __launch_bounds__(256) tile_scan_kernel(const unsigned long long
   if (lane == 0) tile_cnt[j] = carry;
 }
 
+// Writes the entry (t << 32) | (i0 << 8) | (n - 1) of row t's run in tile tl.
+__device__ __forceinline__ void tile_put(int64_t t, int32_t tl, int i0, int n, int64_t n_tiles,
+                                         const unsigned long long* __restrict__ masks,
+                                         const int32_t* __restrict__ blk_base, const int32_t* __restrict__ ptr,
+                                         int64_t* __restrict__ ent) {
+  const int64_t cell = (t >> 6) * n_tiles + tl;
+  const unsigned long long below = masks[cell] & ((1ull << (t & 63)) - 1ull);
+  const int64_t p = static_cast<int64_t>(ptr[tl]) + blk_base[cell] + __popcll(below);
+  ent[p] = (t << 32) | (static_cast<int64_t>(i0) << 8) | static_cast<int64_t>(n - 1);
+}
+
 // One entry per (row, tile) run, (t << 32) | (i0 << 8) | (n - 1), at
 // ptr[tile] + blk_base[block, tile] + (rows of the block below t that meet the tile).
-__global__ void __launch_bounds__(512) tile_fill_kernel(const int32_t* __restrict__ row_cnt,
+// A run ends where the next one starts: within a 32-key window the next start
+// above a lane comes from the window's ballot of starts; the last run of a
+// window stays pending until the first start of a later window (or the row's end).
+__global__ void __launch_bounds__(512, 2) tile_fill_kernel(const int32_t* __restrict__ row_cnt,
                                                         const int32_t* __restrict__ row_cols, int64_t T, int n_sel,
                                                         int64_t n_tiles, const unsigned long long* __restrict__ masks,
                                                         const int32_t* __restrict__ blk_base,
                                                         const int32_t* __restrict__ ptr, int64_t* __restrict__ ent) {
-  for_block_runs(row_cnt, row_cols, T, n_sel, [&](int64_t t, const int32_t* cols, int n, int32_t tl, int i) {
-    // the run ends at the first key of a later tile; a tile holds at most 128
-    // distinct keys, so it ends within [i + 1, i + 128]
-    int lo = i + 1, hi = min(n, i + 128);
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if ((cols[mid] >> kTileShift) > tl) hi = mid;
-      else lo = mid + 1;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int rpw = kBlockRows / nw;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kBlockRows + static_cast<int64_t>(warp) * rpw;
+  for (int r = 0; r < rpw; ++r) {
+    const int64_t t = t0 + r;
+    if (t >= T) return;
+    const int cnt = row_cnt[t];
+    const int32_t* cols = row_cols + t * n_sel;
+    int32_t carry = -1;             // tile of the last key of the previous window (none: -1)
+    int pend_i = -1;                // start of the run still open at the end of the previous windows
+    int32_t pend_tl = 0;
+    for (int base = 0; base < cnt; base += 32) {
+      const int i = base + lane;
+      const int32_t tl = i < cnt ? (cols[i] >> kTileShift) : INT_MAX;
+      int32_t prev = __shfl_up_sync(0xffffffffu, tl, 1);
+      if (lane == 0) prev = carry;
+      carry = __shfl_sync(0xffffffffu, tl, 31);
+      const bool start = i < cnt && tl != prev;
+      const uint32_t m = __ballot_sync(0xffffffffu, start);
+      if (m == 0) continue;
+      const int first = __ffs(m) - 1, last = 31 - __clz(m);
+      if (pend_i >= 0 && lane == 0) tile_put(t, pend_tl, pend_i, base + first - pend_i, n_tiles, masks, blk_base, ptr, ent);
+      const uint32_t above = lane == 31 ? 0u : (m >> (lane + 1)) << (lane + 1);
+      if (start && above != 0) tile_put(t, tl, i, base + __ffs(above) - 1 - i, n_tiles, masks, blk_base, ptr, ent);
+      pend_i = base + last;
+      pend_tl = __shfl_sync(0xffffffffu, tl, last);
     }
-    const int64_t cell = (t >> 6) * n_tiles + tl;
-    const unsigned long long below = masks[cell] & ((1ull << (t & 63)) - 1ull);
-    const int64_t p = static_cast<int64_t>(ptr[tl]) + blk_base[cell] + __popcll(below);
-    ent[p] = (t << 32) | (static_cast<int64_t>(i) << 8) | static_cast<int64_t>(lo - i - 1);
-  });
+    if (pend_i >= 0 && lane == 0) tile_put(t, pend_tl, pend_i, cnt - pend_i, n_tiles, masks, blk_base, ptr, ent);
+  }
 }
 
 // One warp per tile: lane 0 appends the tile's non-empty phase ranges to the
