@@ -2,8 +2,8 @@
 
 ``dkdv_union_kernel`` (``csrc/qsa_dkdv_union.cu``) is a persistent kernel: per
 CTA a scheduler warp, gather warps (a fixed set per stage of a three-stage
-ring: two each as built, each taking half of a chunk's unions, or one), one
-MMA thread and four epilogue warps hand chunks and accumulators to one
+ring: four each as built, each taking a quarter of a chunk's unions, or one),
+one MMA thread and four epilogue warps hand chunks and accumulators to one
 another through mbarriers, and across CTAs each (tile, group, tensor) passes
 its FP32 partial from query phase to query phase through a counter in global
 memory.  This test restates that protocol as coroutines (one per warp role and
@@ -34,7 +34,7 @@ import random
 
 import pytest
 
-STAGES, RING, ACC_BUFS, UNIONS, HALVES = 3, 16, 2, 8, 2
+STAGES, RING, ACC_BUFS, UNIONS, PER_STAGE = 3, 16, 2, 8, 4
 
 
 class Bar:
@@ -94,13 +94,13 @@ def make_units(rng, n_tiles, P, G):
 
 
 class Model:
-    """With `n_workers` = 2 x STAGES the pair of stage k % STAGES fills chunk k
-    (the kernel); otherwise `n_workers` warps take the chunks in turn, chunk k to
-    warp k % n_workers;
+    """With `n_workers` = PER_STAGE x STAGES the warps of stage k % STAGES fill
+    chunk k together (the kernel); otherwise `n_workers` warps take the chunks
+    in turn, chunk k to warp k % n_workers;
     `collective_exit=False` restates an earlier epilogue in which each warp left
     on its own accumulator wait."""
 
-    def __init__(self, units, n_ctas, seed, n_workers=STAGES * HALVES, collective_exit=True, expire_at=None,
+    def __init__(self, units, n_ctas, seed, n_workers=STAGES * PER_STAGE, collective_exit=True, expire_at=None,
                  expire_roles=""):
         self.rng = random.Random(seed)
         self.n_workers = n_workers
@@ -127,12 +127,12 @@ class Model:
         self.n_roles = {i: sum(1 for n in self.roles if n[0] == i) for i in range(n_ctas)}
 
     def cta_state(self):
-        per_stage = HALVES if self.n_workers == STAGES * HALVES else 1
+        per_stage = PER_STAGE if self.n_workers == STAGES * PER_STAGE else 1
         return dict(full=[Bar(per_stage) for _ in range(STAGES)], empty=[Bar(1) for _ in range(STAGES)],
                     ring_full=[Bar(1) for _ in range(RING)], ring_empty=[Bar(per_stage) for _ in range(RING)],
                     acc_full=[Bar(2) for _ in range(ACC_BUFS)], acc_empty=[Bar(4) for _ in range(ACC_BUFS)],
                     drain=Bar(1), ring=[None] * RING, stage=[None] * STAGES,
-                    half=[[None] * HALVES for _ in range(STAGES)], acc=[None] * ACC_BUFS,
+                    half=[[None] * PER_STAGE for _ in range(STAGES)], acc=[None] * ACC_BUFS,
                     acc_desc=[None] * ACC_BUFS, acc_read={}, tc=[], abort=False, named={}, exited=0,
                     freed=False, per_stage=per_stage)
 
@@ -168,7 +168,7 @@ class Model:
                 c["ring"][rs] = dict(k=k, U=U, first=p == 0, last=p + n >= u["n_ent"])
                 c["ring_full"][rs].arrive()
                 k += 1
-        markers = STAGES if c["per_stage"] == HALVES else self.n_workers
+        markers = STAGES if c["per_stage"] == PER_STAGE else self.n_workers
         for j in range(markers if ok else 0):            # end markers; only the first reaches the MMA
             rs = k % RING
             if k >= RING and not (yield self.wait(c["ring_empty"][rs], k // RING - 1)):
@@ -178,7 +178,7 @@ class Model:
             k += 1
 
     def worker(self, c, w):
-        pairs = c["per_stage"] == HALVES
+        pairs = c["per_stage"] == PER_STAGE
         step = STAGES if pairs else self.n_workers
         k = w % STAGES if pairs else w
         h = w // STAGES if pairs else 0
@@ -379,7 +379,7 @@ def _structures():
 
 
 @pytest.mark.parametrize("case", range(12))
-@pytest.mark.parametrize("per_stage", [1, 2])
+@pytest.mark.parametrize("per_stage", [1, PER_STAGE])
 def test_protocol_under_random_schedules(case, per_stage):
     units, n_ctas = _structures()[case]
     expected = {}

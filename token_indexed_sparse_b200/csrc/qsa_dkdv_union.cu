@@ -16,18 +16,19 @@
 // 6 tcgen05.mma kind::f16 (M 128, N 256, K 16), A K-major without swizzle, B
 // MN-major with the 128-byte swizzle, the accumulator in tensor memory (two
 // 256-column buffers, so the epilogue of one unit overlaps the next unit's MMAs).
-// Chunks of 8 unions rather than 4 halve the MMA thread's fixed cost per union
-// (seq32k: 7.3 -> 5.8 ms), at three 72 KB stages instead of six of 36 KB.
+// Chunks of 8 unions rather than 4 halve the MMA thread's fixed cost per union,
+// at three 72 KB stages instead of six of 36 KB, and four warps per stage keep
+// more copies in flight (seq32k 7.3 -> 5.6 ms, thd16k 1.53 -> 1.14 ms).
 //
-// Warp roles (384 threads): warp 6 schedules (claims units, cuts them into
+// Warp roles (576 threads): warp 16 schedules (claims units, cuts them into
 // chunks of 8 entries, publishes each chunk's descriptor in a shared-memory ring
-// and prefetches its records and keys into L2); warps 0-5 fill the chunks, warps
-// s and s + 3 every chunk of stage s of the 3-stage shared-memory ring, each
-// four of its unions (clear A, gather B rows with cp.async, store the records
-// into their A rows; a warp keeps only about eight 512-byte copies in flight,
-// so the rows of a chunk are split over two warps); warp 7 (one thread) issues
-// the MMAs; warps 8-11 (tensor-memory lane quarters 0-3) run the epilogue,
-// thread = key row.  Units are claimed from one counter in
+// and prefetches its records and keys into L2); warps 0-11 fill the chunks,
+// warps s, s + 3, s + 6 and s + 9 every chunk of stage s of the 3-stage
+// shared-memory ring, each two of its unions (clear A, gather B rows with
+// cp.async, store the records into their A rows; a warp keeps only about eight
+// 512-byte copies in flight, so the rows of a chunk are split over four warps);
+// warp 17 (one thread) issues the MMAs; warps 12-15 (tensor-memory lane
+// quarters 0-3) run the epilogue, thread = key row.  Units are claimed from one counter in
 // phase order (phase 0's units, then phase 1's, ...; inside a phase every dK
 // unit before every dV unit), so the
 // CTAs work on about one phase and one tensor at a time and its Q (or dO) rows
@@ -51,10 +52,10 @@ namespace {
 constexpr int kUCtasPerSm = 1, kUAccBufs = 2;
 constexpr int kUTmemCols = 256 * kUAccBufs;
 constexpr int kUStages = 3;
-constexpr int kUWorkersPerStage = 2;                // warps per stage, kUUnions / 2 unions each
-constexpr int kUWorkers = kUStages * kUWorkersPerStage;  // warps 0-5 fill chunks
-constexpr int kUSchedWarp = 6, kUMmaWarp = 7, kUEpiWarp0 = 8;
-constexpr int kUWarps = 12;
+constexpr int kUWorkersPerStage = 4;                // warps per stage, kUUnions / 4 unions each
+constexpr int kUWorkers = kUStages * kUWorkersPerStage;  // warps 0-11 fill chunks
+constexpr int kUEpiWarp0 = 12, kUSchedWarp = 16, kUMmaWarp = 17;
+constexpr int kUWarps = 18;
 constexpr int kUThreads = 32 * kUWarps;
 constexpr int kURec = 24;                           // bf16 per (t, g, key) record: 12 P + 12 dS
 constexpr int kUKeys = 128;                         // keys per tile (MMA M)
