@@ -285,6 +285,24 @@ qsa_status_t qsa_selector_topk(const float* scores, int64_t score_stride, int64_
                                int32_t* blocks, int32_t* routes, qsa_stream_t stream);
 
 /*
+ * The query-union lists the forward walks, on their own: the paired-query
+ * gather of the "Query Sparse Attention (QSA)" page ("Selection and
+ * components": adjacent queries gather the union of their selected keys once,
+ * owner bits keeping each query's own set), for groups of
+ * qsa_union_group(n_sel) adjacent rows (4, or 1 for rows of more than 4096
+ * slots; 0 for an n_sel outside 1..16384).
+ *   row_cnt, row_cols : as qsa_route_plan
+ *   ucnt [ceil(T/group)] int32 : the number of distinct keys in each group's union
+ *   ukey [ceil(T/group) * group * n_sel] int32 : group i's union, ascending, in
+ *       ukey[i * group * n_sel .. + ucnt[i]); the rest is left unspecified
+ *   uown (same shape) uint8 : per union key, bit q set iff row group * i + q selected it
+ * Same size limits and errors as qsa_route_plan (ucnt / ukey 4-byte aligned).
+ */
+int qsa_union_group(int n_sel);
+qsa_status_t qsa_union_plan(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel, int32_t* row_cnt,
+                            int32_t* row_cols, int32_t* ucnt, int32_t* ukey, uint8_t* uown, qsa_stream_t stream);
+
+/*
  * FP32 -> BF16 rounding of n contiguous values, round to nearest with ties to
  * even: the final cast of dK / dV sums that a caller adds up in FP32 across
  * several qsa_backward_fp32kv calls (context parallelism reduce-scatters each

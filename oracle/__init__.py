@@ -20,4 +20,5 @@ from .qsa_oracle import (  # noqa: F401
     route_rows_csr,
     key_quad_lists,
     key_tile_lists,
+    query_union_lists,
 )

@@ -151,6 +151,40 @@ def key_tile_lists(routes, kv_length: int, tile: int = 128):
     cols = np.asarray(flat, dtype=np.int32).reshape(-1, 3)
     return ptr, cols[:, 0].copy(), cols[:, 1].copy(), cols[:, 2].copy()
 
+def query_union_lists(routes, kv_length: int, group: int):
+    """Route sets of adjacent query rows merged, with owner masks.
+
+    The paired-query gather of the [QSA] page ("Selection and components": one
+    program owns adjacent queries and gathers the union of their selected
+    blocks once, with owner bits telling which query selected each) at a group
+    of ``group`` consecutive rows: group ``i`` holds rows ``group*i ..
+    group*i + group - 1`` (the last group may be shorter).  Its list is the
+    union of those rows' route sets R_t in ascending key order, and key j's
+    owner mask has bit ``q`` set iff j is in R_{group*i + q}.
+
+    Returns ``(counts [n_groups] int32, keys list of int32 arrays, owners list
+    of int32 arrays)``, one array pair per group.
+    """
+    sets = row_route_sets(routes, kv_length)
+    T = len(sets)
+    n_groups = (T + group - 1) // group
+    counts = np.zeros(n_groups, dtype=np.int32)
+    keys, owners = [], []
+    for i in range(n_groups):
+        own = {}
+        for q in range(group):
+            t = group * i + q
+            if t >= T:
+                break
+            for j in sets[t]:
+                own[int(j)] = own.get(int(j), 0) | (1 << q)
+        ks = sorted(own)
+        counts[i] = len(ks)
+        keys.append(np.asarray(ks, dtype=np.int32))
+        owners.append(np.asarray([own[j] for j in ks], dtype=np.int32))
+    return counts, keys, owners
+
+
 # ---------------------------------------------------------------------------
 # Dense-table form: the definition, for finite inputs
 # ---------------------------------------------------------------------------

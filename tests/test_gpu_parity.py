@@ -392,3 +392,43 @@ def test_error_statuses_launch_nothing():
     assert torch.all(out == 7.0) and torch.all(lse == 7.0)
     with pytest.raises(qsa.QSAError):
         qsa.forward(q, k, v, routes, scale=float("nan"))
+
+
+# ---------------------------------------------------------------------------
+# query-union lists (the forward's key lists): bit-exact
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name,T", [("tiny", None), ("seq4k", 512), ("thd16k", 1024), ("seq32k", 768),
+                                    ("cp128k", 256)])
+def test_union_plan_bitexact(name, T):
+    wl = W.WORKLOADS[name] if T is None else W.WORKLOADS[name].scaled(T)
+    routes = W.make_routes(wl)
+    if name == "tiny":
+        routes = np.array(routes)
+        routes[10] = routes[11]                    # two rows of one group with the same set
+        routes[13, :5] = [7, 7, -1, wl.T_kv, 200]  # duplicates and invalid IDs
+    r = torch.from_numpy(np.array(routes, dtype=np.int32)).to(DEV)
+    group, ucnt, ukey, uown = qsa.union_plan(r, wl.T_kv)
+    torch.cuda.synchronize()
+    cnt, keys, owners = oracle.query_union_lists(routes, wl.T_kv, group)
+    np.testing.assert_array_equal(ucnt.cpu().numpy(), cnt)
+    ukey, uown = ukey.cpu().numpy(), uown.cpu().numpy()
+    for i in range(len(cnt)):
+        np.testing.assert_array_equal(ukey[i, :cnt[i]], keys[i])
+        np.testing.assert_array_equal(uown[i, :cnt[i]], owners[i])
+
+
+def test_union_plan_long_rows_fall_back_to_single_rows():
+    # rows of more than 4096 slots are not merged (groups of one row)
+    rng = np.random.default_rng(5)
+    T, T_kv, n_sel = 20, 50000, 5000
+    routes = rng.integers(-10, T_kv, size=(T, n_sel)).astype(np.int32)
+    r = torch.from_numpy(routes).to(DEV)
+    group, ucnt, ukey, uown = qsa.union_plan(r, T_kv)
+    torch.cuda.synchronize()
+    assert group == 1
+    cnt, keys, owners = oracle.query_union_lists(routes, T_kv, 1)
+    np.testing.assert_array_equal(ucnt.cpu().numpy(), cnt)
+    for i in range(T):
+        np.testing.assert_array_equal(ukey[i, :cnt[i]].cpu().numpy(), keys[i])
+        assert np.all(uown[i, :cnt[i]].cpu().numpy() == 1)

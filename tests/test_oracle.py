@@ -365,3 +365,31 @@ def test_key_tile_lists_refine_quads():
     np.testing.assert_array_equal(qptr, tptr)
     np.testing.assert_array_equal(qq, tq)
     np.testing.assert_array_equal([bin(int(m)).count("1") for m in qm], tn)
+
+
+@pytest.mark.parametrize("group", [1, 2, 4])
+def test_query_union_lists(group):
+    # brute force from the membership table: per group of adjacent rows, the
+    # keys any of them selects (ascending) and, per key, which of them did
+    rng = np.random.default_rng(37)
+    T, T_kv = 42, 211                                  # the last group is short for group 4
+    routes = _random_routes(rng, T, T_kv, 30)
+    routes[9] = -1                                     # a padding row inside a group
+    routes[10] = routes[11]                            # two rows with the same set
+    M = oracle.routes_to_membership(routes, T_kv)
+    counts, keys, owners = oracle.query_union_lists(routes, T_kv, group)
+    n_groups = (T + group - 1) // group
+    assert len(counts) == len(keys) == len(owners) == n_groups
+    for i in range(n_groups):
+        rows = range(group * i, min(T, group * (i + 1)))
+        want = np.nonzero(M[list(rows)].any(axis=0))[0]
+        assert counts[i] == len(want)
+        np.testing.assert_array_equal(keys[i], want)
+        for j, m in zip(keys[i], owners[i]):
+            assert m == sum(1 << q for q, t in enumerate(rows) if M[t, j])
+    if group == 1:                                     # a group of one row is the row's set
+        cnt, cols = oracle.route_rows_csr(routes, T_kv)
+        np.testing.assert_array_equal(counts, cnt)
+        for t in range(T):
+            np.testing.assert_array_equal(keys[t], cols[t, :cnt[t]])
+            assert np.all(owners[t] == 1)

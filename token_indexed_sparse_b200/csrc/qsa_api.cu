@@ -327,6 +327,22 @@ qsa_status_t qsa_route_plan(const int32_t* routes, int64_t T, int64_t T_kv, int 
   return QSA_OK;
 }
 
+int qsa_union_group(int n_sel) { return n_sel < 1 || n_sel > kMaxSel ? 0 : qsa::union_group(n_sel); }
+
+qsa_status_t qsa_union_plan(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel, int32_t* row_cnt,
+                            int32_t* row_cols, int32_t* ucnt, int32_t* ukey, uint8_t* uown, qsa_stream_t stream) {
+  if (!routes || !row_cnt || !row_cols || !ucnt || !ukey || !uown) return QSA_ERR_INVALID_ARGUMENT;
+  const qsa_status_t st = check_sizes(T, T_kv, qsa::kHeadsPerGroup, 1, n_sel);
+  if (st != QSA_OK) return st;
+  if (!aligned(routes, 4) || !aligned(row_cnt, 4) || !aligned(row_cols, 4) || !aligned(ucnt, 4) || !aligned(ukey, 4))
+    return QSA_ERR_MISALIGNED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 0, nullptr, nullptr, nullptr,
+                                 nullptr, qsa::kHeadsPerGroup, s));
+  QSA_TRY(qsa::launch_union_lists(row_cnt, row_cols, T, n_sel, qsa::union_group(n_sel), ucnt, ukey, uown, s));
+  return QSA_OK;
+}
+
 size_t qsa_tile_plan_scratch_size(int64_t T, int64_t T_kv) {
   if (T < 1 || T_kv < 1 || T_kv > INT32_MAX) return 0;
   const size_t nt = static_cast<size_t>((T_kv + 127) / 128);

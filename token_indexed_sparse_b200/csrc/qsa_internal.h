@@ -47,6 +47,17 @@ cudaError_t launch_tile_worklist(const int32_t* tile_ptr, const void* scratch, i
                                  int64_t T_kv, int G, int P, int C, int32_t* wl_cnt, int4* wl, void* dk, void* dv,
                                  bool f32_out, cudaStream_t s);
 
+// Union lists of groups of `group` adjacent query rows (qsa_routes.cu): per
+// group gi, the ascending union of the rows' route sets in ukey[gi * group *
+// n_sel, + ucnt[gi]) and per key a mask of the rows that selected it (uown).
+// group * n_sel <= kUnionSortCap; union_group(n_sel) is the group size the
+// forward uses (kUnionGroup rows, or 1 for rows too long to merge in shared memory).
+constexpr int kUnionGroup = 4;
+constexpr int kUnionSortCap = 16384;
+int union_group(int n_sel);
+cudaError_t launch_union_lists(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel, int group,
+                               int32_t* ucnt, int32_t* ukey, uint8_t* uown, cudaStream_t s);
+
 // Attention kernels (qsa_forward.cu, qsa_backward.cu, qsa_dkdv_union.cu).
 cudaError_t launch_forward(const void* q, const void* k, const void* v, const int32_t* row_cnt,
                            const int32_t* row_cols, int64_t T, int G, int n_sel, float scale,

@@ -24,6 +24,7 @@ namespace {
 constexpr int kRowThreads = 256;
 constexpr int kSortThreads = 256;
 constexpr int kSortCap = 4096;  // int64 entries sorted in shared memory (32 KB)
+constexpr int kMaxUnionGroup = 8;  // rows per union group at most
 
 // Ascending bitonic sort of s[0, n2) where n2 is a power of two and elements at
 // or beyond `len` are treated as +infinity (never read or written).  Every
@@ -506,6 +507,82 @@ __global__ void __launch_bounds__(512, 2) tile_fill_kernel(const int32_t* __rest
   }
 }
 
+// Union lists of groups of `group` adjacent query rows (the paired-query gather
+// of the "Query Sparse Attention (QSA)" page, "Selection and components":
+// adjacent queries gather the union of their selected keys once, owner bits
+// keeping each query's own set).  One CTA per group.  The rows are sorted
+// already, so their merge needs no sort: key x at position k of row q goes to
+// k + (keys of the rows below q that are <= x) + (keys of the rows above q
+// that are < x) (binary searches in shared memory), a stable merge in which
+// equal keys end up adjacent in row order.  Every distinct key is then placed
+// by a CTA scan over "first of its key" flags, with the OR of its owners.
+// Group gi's list is ukey / uown [gi * group * n_sel, ...), its length ucnt[gi].
+__device__ __forceinline__ int count_below(const int32_t* a, int n, int32_t x, bool or_equal) {
+  int lo = 0, hi = n;  // the number of a[0 .. n) that are < x (or <= x)
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] < x || (or_equal && a[mid] == x)) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(kRowThreads) union_lists_kernel(
+    const int32_t* __restrict__ row_cnt, const int32_t* __restrict__ row_cols, int64_t T, int n_sel, int group,
+    int32_t* __restrict__ ucnt, int32_t* __restrict__ ukey, uint8_t* __restrict__ uown) {
+  extern __shared__ int32_t us[];  // the rows' keys [total], then the merged (key, row) pairs [total] as int64
+  __shared__ int scratch[32];
+  __shared__ int off[kMaxUnionGroup + 1];
+  const int64_t gi = blockIdx.x, t0 = gi * group;
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int q = 0; q < group; ++q) {
+      off[q] = acc;
+      acc += t0 + q < T ? row_cnt[t0 + q] : 0;
+    }
+    off[group] = acc;
+  }
+  __syncthreads();
+  const int total = off[group];
+  int64_t* mv = reinterpret_cast<int64_t*>(us + ((total + 1) & ~1));
+  for (int i = threadIdx.x; i < total; i += blockDim.x) {
+    int q = 0;
+    while (i >= off[q + 1]) ++q;
+    us[i] = row_cols[(t0 + q) * n_sel + (i - off[q])];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < total; i += blockDim.x) {
+    int q = 0;
+    while (i >= off[q + 1]) ++q;
+    const int32_t x = us[i];
+    int pos = i - off[q];
+    for (int q2 = 0; q2 < group; ++q2)
+      if (q2 != q) pos += count_below(us + off[q2], off[q2 + 1] - off[q2], x, q2 < q);
+    mv[pos] = (static_cast<int64_t>(x) << 8) | q;
+  }
+  __syncthreads();
+  const int per = (total + blockDim.x - 1) / blockDim.x;
+  const int lo = min(total, static_cast<int>(threadIdx.x) * per), hi = min(total, lo + per);
+  int mine = 0;
+  for (int i = lo; i < hi; ++i)
+    if (i == 0 || (mv[i] >> 8) != (mv[i - 1] >> 8)) ++mine;
+  int cnt;
+  int pos = block_exclusive_scan(mine, scratch, &cnt);
+  const int64_t cap = static_cast<int64_t>(group) * n_sel;
+  int32_t* kd = ukey + gi * cap;
+  uint8_t* od = uown + gi * cap;
+  for (int i = lo; i < hi; ++i) {
+    if (i > 0 && (mv[i] >> 8) == (mv[i - 1] >> 8)) continue;
+    const int64_t key = mv[i] >> 8;
+    uint32_t own = 0;
+    for (int k = i; k < total && (mv[k] >> 8) == key; ++k) own |= 1u << (mv[k] & 0xff);
+    kd[pos] = static_cast<int32_t>(key);
+    od[pos] = static_cast<uint8_t>(own);
+    ++pos;
+  }
+  if (threadIdx.x == 0) ucnt[gi] = cnt;
+}
+
 // One warp per tile: lane 0 appends the tile's non-empty phase ranges to the
 // per-phase work lists, wl[p][*] = (tile, first entry, end entry, flags), flags
 // bit 0: no entries of the tile before this range, bit 1: none after it, bits
@@ -600,6 +677,25 @@ cudaError_t launch_quad_fill(const int32_t* row_cnt, const int32_t* row_cols, in
 cudaError_t launch_quad_sort(const int32_t* quad_ptr, int64_t n_quads, int64_t* quad_ent, int P, int C,
                              int32_t* phase_ptr, cudaStream_t s) {
   quad_sort_kernel<<<static_cast<unsigned>(n_quads), kSortThreads, 0, s>>>(quad_ptr, quad_ent, P, C, phase_ptr);
+  return cudaGetLastError();
+}
+
+int union_group(int n_sel) { return n_sel <= kUnionSortCap / kUnionGroup ? kUnionGroup : 1; }
+
+cudaError_t launch_union_lists(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel, int group,
+                               int32_t* ucnt, int32_t* ukey, uint8_t* uown, cudaStream_t s) {
+  if (group < 1 || group > kMaxUnionGroup || static_cast<int64_t>(group) * n_sel > kUnionSortCap)
+    return cudaErrorInvalidValue;
+  const int cap = group * n_sel;
+  const size_t smem = static_cast<size_t>((cap + 1) & ~1) * 4 + static_cast<size_t>(cap) * 8;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(union_lists_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t n_groups = (T + group - 1) / group;
+  union_lists_kernel<<<static_cast<unsigned>(n_groups), kRowThreads, smem, s>>>(row_cnt, row_cols, T, n_sel, group,
+                                                                               ucnt, ukey, uown);
   return cudaGetLastError();
 }
 

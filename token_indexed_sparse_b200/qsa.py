@@ -73,6 +73,10 @@ def library() -> ctypes.CDLL:
     lib.qsa_tile_plan_scratch_size.argtypes = [i64, i64]
     lib.qsa_tile_plan.restype = i32
     lib.qsa_tile_plan.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp, vp, sz, vp]
+    lib.qsa_union_group.restype = i32
+    lib.qsa_union_group.argtypes = [i32]
+    lib.qsa_union_plan.restype = i32
+    lib.qsa_union_plan.argtypes = [vp, i64, i64, i32, vp, vp, vp, vp, vp, vp]
     lib.qsa_cast_f32_to_bf16.restype = i32
     lib.qsa_cast_f32_to_bf16.argtypes = [vp, vp, i64, vp]
     _lib = lib
@@ -226,6 +230,28 @@ def backward(grad_out, q, k, v, out, lse, routes, scale: float = 1.0 / 16.0, *,
                                  _ptr(ws), ws.numel(), _stream(q.device), ev, n_ev)
     _check(st, "qsa_backward")
     return dq, dk, dv
+
+
+def union_plan(routes, T_kv: int):
+    """qsa_union_plan: ``(group, ucnt, ukey, uown)`` of the forward's query
+    groups (route rows first, as qsa_route_plan); ``ukey`` / ``uown`` are
+    ``[n_groups, group * n_sel]``, row i valid up to ``ucnt[i]``."""
+    lib = library()
+    routes = _prep(routes, torch.int32, "routes")
+    T, n_sel = routes.shape
+    group = lib.qsa_union_group(n_sel)
+    if group < 1:
+        raise ValueError("n_sel outside 1..16384")
+    n_groups = (T + group - 1) // group
+    dev = routes.device
+    row_cnt = torch.empty(T, dtype=torch.int32, device=dev)
+    row_cols = torch.empty(T, n_sel, dtype=torch.int32, device=dev)
+    ucnt = torch.empty(n_groups, dtype=torch.int32, device=dev)
+    ukey = torch.empty(n_groups, group * n_sel, dtype=torch.int32, device=dev)
+    uown = torch.empty(n_groups, group * n_sel, dtype=torch.uint8, device=dev)
+    _check(lib.qsa_union_plan(_ptr(routes), T, T_kv, n_sel, _ptr(row_cnt), _ptr(row_cols), _ptr(ucnt), _ptr(ukey),
+                              _ptr(uown), _stream(dev)), "qsa_union_plan")
+    return group, ucnt, ukey, uown
 
 
 def cast_f32_to_bf16(x, out=None):
