@@ -47,6 +47,8 @@ ATTENTION_PINS = [
     ("tile lists, 8 keys", lambda: pins.test_key_tile_lists(8)),
     ("tile lists, 128 keys", lambda: pins.test_key_tile_lists(128)),
     ("tiles of 4 = quads", pins.test_key_tile_lists_refine_quads),
+    ("query unions, groups of 4", lambda: pins.test_query_union_lists(4)),
+    ("query unions, groups of 1", lambda: pins.test_query_union_lists(1)),
 ]
 
 # name -> (text in the oracle, its mistaken form); every occurrence is replaced,
@@ -81,6 +83,11 @@ ATTENTION_MUTANTS = {
     "sampled-key dV from dS": ("dv[dst, g, :] += P[:, n] @ do[t, hs, :]", "dv[dst, g, :] += dS[:, n] @ do[t, hs, :]"),
     "sampled-key dK unscaled": ("dk[dst, g, :] += scale * (dS[:, n] @ q[t, hs, :])", "dk[dst, g, :] += dS[:, n] @ q[t, hs, :]"),
     "tile run one key long": ("int(pos.size)", "int(pos.size) + 1"),
+    "union owner bits shifted": ("own[int(j)] = own.get(int(j), 0) | (1 << q)",
+                                 "own[int(j)] = own.get(int(j), 0) | (1 << (q + 1))"),
+    "union drops a group's last row": ("for q in range(group):\n            t = group * i + q",
+                                       "for q in range(group - 1):\n            t = group * i + q"),
+    "union keys unsorted": ("ks = sorted(own)", "ks = list(own)"),
 }
 
 # ---------------------------------------------------------------------------
