@@ -160,11 +160,13 @@ qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k,
 
 /*
  * Number of kernels one qsa_forward (backward = 0) or qsa_backward (backward = 1)
- * call enqueues for these sizes, not counting the cudaMemsetAsync node of the
- * backward (one).  The forward launches 2 (route rows, attention); the backward
- * 8 (route rows, tile counts, tile scan, tile fill, tile sort, work lists, dQ,
- * dK/dV).  Returns 0 for sizes the calls reject.  For instrumentation and for
- * sizing CUDA graphs; the pages have no counterpart.
+ * call enqueues for these sizes, not counting the backward's cudaMemsetAsync
+ * nodes (one for its counters, and a second one for the tile masks when T_kv
+ * exceeds 8192 tiles of 128 keys).  The forward launches 2 (route rows,
+ * attention); the backward 8 (route rows, tile masks, column scans of the
+ * masks, tile-pointer scan, tile fill, work lists, dQ, dK/dV).  Returns 0 for
+ * sizes the calls reject.  For instrumentation and for sizing CUDA graphs; the
+ * pages have no counterpart.
  */
 int qsa_launch_count(int64_t T, int64_t T_kv, int H, int G, int n_sel, int backward);
 
