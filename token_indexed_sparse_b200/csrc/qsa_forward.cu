@@ -14,10 +14,15 @@
 // shape).  Rows past the end of R_t are zero-filled, so unselected K/V
 // values never reach an output.  Per chunk, warp w forms S = Q K^T for keys
 // 8w..8w+7 (mma.sync m16n8k16 BF16, FP32 accumulate, Q fragments held in
-// registers for the whole item), the chunk's row maxima are combined across the
-// warps in shared memory, P = exp2(S*scale*log2e - m) is written as BF16, and
-// warp w accumulates O[:, DPW w : DPW (w + 1)] += P V (DPW = 256 / warps, 128 at
-// the launch shape) with running-max rescaling.
+// registers for the whole item), P = exp2(S*scale*log2e - m) is written as BF16
+// against the running row maximum m, and warp w accumulates
+// O[:, DPW w : DPW (w + 1)] += P V (DPW = 256 / warps, 128 at the launch shape).
+// m may lag the true maximum by up to 2^8 (P < 256): only a chunk in which some
+// score passes m by more than that exchanges the warps' maxima, rescales O and
+// the sums and rewrites P, so most chunks take one barrier between S and P V.
+// Each lane keeps its part of the row sums; they are combined once per item.
+// (seq32k forward: 3.80 ms with a maximum exchange and a sum exchange in every
+// chunk, 3.53 ms with the lag.)
 #include "qsa_internal.h"
 #include "qsa_pipe.cuh"
 
@@ -42,11 +47,17 @@ struct FwdShape {
   static constexpr int kOffMax = kOffP + kRowTile * kPStride * 2;
   static constexpr int kOffSum = kOffMax + NW * kRowTile * 4;
   static constexpr int kOffDesc = kOffSum + NW * kRowTile * 4;
-  static constexpr int kSmemBytes = kOffDesc + STAGES * 16;
+  static constexpr int kOffJump = kOffDesc + STAGES * 16;       // one flag per warp
+  static constexpr int kSmemBytes = kOffJump + ((NW * 4 + 15) / 16) * 16;
   static_assert(kSmemBytes * CPS + 1024 * CPS <= 233472, "shared memory per SM");
   static_assert(kKs >= 1 && kNt % 2 == 0, "shape");
 };
 constexpr int kFirst = 1, kLast = 2;
+// The running maximum of a row may lag its true maximum by up to kLag (log2
+// units): P stays below 2^kLag, and O and the sums are rescaled only when a
+// score passes the maximum by more than that.
+constexpr float kLag = 8.f;
+__device__ __forceinline__ float p_of(float s, float m) { return s == -INFINITY ? 0.f : exp2f(s - m); }
 
 template <int NW, int STAGES, int CPS>
 __global__ void __launch_bounds__(NW * 32, CPS)
@@ -66,6 +77,7 @@ fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict_
   __nv_bfloat16* sP = reinterpret_cast<__nv_bfloat16*>(smem + S_::kOffP);
   float* sMax = reinterpret_cast<float*>(smem + S_::kOffMax);
   float* sSum = reinterpret_cast<float*>(smem + S_::kOffSum);
+  int* sJump = reinterpret_cast<int*>(smem + S_::kOffJump);
   if (tid < 32) reinterpret_cast<uint4*>(smem + S_::kOffZero)[tid] = make_uint4(0, 0, 0, 0);
 
   Cursor cur;
@@ -151,6 +163,15 @@ fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict_
     s[1] = v1 ? s[1] * scale_log2 : -INFINITY;
     s[2] = v0 ? s[2] * scale_log2 : -INFINITY;
     s[3] = v1 ? s[3] * scale_log2 : -INFINITY;
+    // P against the running maximum as it stands; it is replaced only when a
+    // score exceeds it by more than kLag (then every warp rescales together)
+    const bool jump = fmaxf(s[0], s[1]) > m0 + kLag || fmaxf(s[2], s[3]) > m1 + kLag;
+    const unsigned any_jump = __any_sync(0xffffffffu, jump);
+    float p0 = p_of(s[0], m0), p1 = p_of(s[1], m0), p2 = p_of(s[2], m1), p3 = p_of(s[3], m1);
+    if (!any_jump) {
+      *reinterpret_cast<uint32_t*>(sP + gq * kPStride + key0) = pack_bf16(p0, p1);
+      *reinterpret_cast<uint32_t*>(sP + (gq + 8) * kPStride + key0) = pack_bf16(p2, p3);
+    }
     float x0 = fmaxf(s[0], s[1]), x1 = fmaxf(s[2], s[3]);
     x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 1));
     x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 2));
@@ -160,45 +181,40 @@ fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict_
       sMax[warp * kRowTile + gq] = x0;
       sMax[warp * kRowTile + gq + 8] = x1;
     }
+    if (lane == 0) sJump[warp] = any_jump ? 1 : 0;
     __syncthreads();
-    float n0 = m0, n1 = m1;
+    bool rescale = false;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      n0 = fmaxf(n0, sMax[w * kRowTile + gq]);
-      n1 = fmaxf(n1, sMax[w * kRowTile + gq + 8]);
-    }
-    const float p0 = exp2f(s[0] - n0), p1 = exp2f(s[1] - n0);
-    const float p2 = exp2f(s[2] - n1), p3 = exp2f(s[3] - n1);
-    *reinterpret_cast<uint32_t*>(sP + gq * kPStride + key0) = pack_bf16(p0, p1);
-    *reinterpret_cast<uint32_t*>(sP + (gq + 8) * kPStride + key0) = pack_bf16(p2, p3);
-    float ps0 = p0 + p1, ps1 = p2 + p3;
-    ps0 += __shfl_xor_sync(0xffffffffu, ps0, 1);
-    ps0 += __shfl_xor_sync(0xffffffffu, ps0, 2);
-    ps1 += __shfl_xor_sync(0xffffffffu, ps1, 1);
-    ps1 += __shfl_xor_sync(0xffffffffu, ps1, 2);
-    if (cq == 0) {
-      sSum[warp * kRowTile + gq] = ps0;
-      sSum[warp * kRowTile + gq + 8] = ps1;
-    }
-    const float a0 = exp2f(m0 - n0), a1 = exp2f(m1 - n1);
-    m0 = n0;
-    m1 = n1;
-    __syncthreads();
-    float c0 = 0.f, c1 = 0.f;
+    for (int w = 0; w < NW; ++w) rescale |= sJump[w] != 0;
+    if (rescale) {  // CTA-uniform
+      float n0 = m0, n1 = m1;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      c0 += sSum[w * kRowTile + gq];
-      c1 += sSum[w * kRowTile + gq + 8];
-    }
-    l0 = l0 * a0 + c0;
-    l1 = l1 * a1 + c1;
+      for (int w = 0; w < NW; ++w) {
+        n0 = fmaxf(n0, sMax[w * kRowTile + gq]);
+        n1 = fmaxf(n1, sMax[w * kRowTile + gq + 8]);
+      }
+      const float a0 = n0 == -INFINITY ? 1.f : exp2f(m0 - n0), a1 = n1 == -INFINITY ? 1.f : exp2f(m1 - n1);
+      m0 = n0;
+      m1 = n1;
+      l0 *= a0;
+      l1 *= a1;
 #pragma unroll
-    for (int nt = 0; nt < kNt; ++nt) {
-      o[nt][0] *= a0;
-      o[nt][1] *= a0;
-      o[nt][2] *= a1;
-      o[nt][3] *= a1;
+      for (int nt = 0; nt < kNt; ++nt) {
+        o[nt][0] *= a0;
+        o[nt][1] *= a0;
+        o[nt][2] *= a1;
+        o[nt][3] *= a1;
+      }
+      p0 = p_of(s[0], m0);
+      p1 = p_of(s[1], m0);
+      p2 = p_of(s[2], m1);
+      p3 = p_of(s[3], m1);
+      *reinterpret_cast<uint32_t*>(sP + gq * kPStride + key0) = pack_bf16(p0, p1);
+      *reinterpret_cast<uint32_t*>(sP + (gq + 8) * kPStride + key0) = pack_bf16(p2, p3);
+      __syncthreads();
     }
+    l0 += p0 + p1;  // this lane's part of the row sums
+    l1 += p2 + p3;
     // O[:, DPW*w : DPW*(w+1)] += P V over the chunk's keys
 #pragma unroll
     for (int ks = 0; ks < kKs; ++ks) {
@@ -212,8 +228,24 @@ fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict_
         mma_16816(o[nt + 1], pa, b[2], b[3]);
       }
     }
-    if (d.w & kLast) {
-      const float i0 = 1.f / l0, i1 = 1.f / l1;
+    if (d.w & kLast) {  // CTA-uniform
+      float c0 = l0, c1 = l1;
+      c0 += __shfl_xor_sync(0xffffffffu, c0, 1);
+      c0 += __shfl_xor_sync(0xffffffffu, c0, 2);
+      c1 += __shfl_xor_sync(0xffffffffu, c1, 1);
+      c1 += __shfl_xor_sync(0xffffffffu, c1, 2);
+      if (cq == 0) {
+        sSum[warp * kRowTile + gq] = c0;
+        sSum[warp * kRowTile + gq + 8] = c1;
+      }
+      __syncthreads();
+      float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        t0 += sSum[w * kRowTile + gq];
+        t1 += sSum[w * kRowTile + gq + 8];
+      }
+      const float i0 = 1.f / t0, i1 = 1.f / t1;
       __nv_bfloat16* orow = out + qrow0 * kHeadDim;
 #pragma unroll
       for (int nt = 0; nt < kNt; ++nt) {
@@ -223,8 +255,8 @@ fwd_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict_
           *reinterpret_cast<uint32_t*>(orow + (gq + 8) * kHeadDim + dim) = pack_bf16(o[nt][2] * i1, o[nt][3] * i1);
       }
       if (warp == 0 && cq == 0) {
-        lse[qrow0 + gq] = (m0 + log2f(l0)) * kLn2;
-        if (gq + 8 < kHeadsPerGroup) lse[qrow0 + gq + 8] = (m1 + log2f(l1)) * kLn2;
+        lse[qrow0 + gq] = (m0 + log2f(t0)) * kLn2;
+        if (gq + 8 < kHeadsPerGroup) lse[qrow0 + gq + 8] = (m1 + log2f(t1)) * kLn2;
       }
     }
   }
