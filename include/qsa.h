@@ -138,8 +138,9 @@ qsa_status_t qsa_backward_fp32kv(const void* grad_out, const void* q, const void
  * `stage_events` may be NULL when n_stage_events is 0.  The pages have no
  * counterpart: this is an instrumentation hook of this library.
  *   forward stages : 0 route rows (sort/dedup), 1 attention forward
- *   backward stages: 0 route rows (+ delta), 1 tile lists (masks, column scans,
- *                    tile scan, fill), 2 work lists, 3 dQ (+ P/dS records), 4 dK/dV
+ *   backward stages: 0 route rows (+ delta, tile masks), 1 tile lists (column
+ *                    scans, tile-pointer scan, fill), 2 work lists, 3 dQ (+ P/dS
+ *                    records), 4 dK/dV
  * A failed eventRecord returns QSA_ERR_CUDA.
  */
 typedef struct CUevent_st* qsa_event_t; /* same type as cudaEvent_t */
@@ -159,14 +160,40 @@ qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k,
                              const qsa_event_t* stage_events, int n_stage_events);
 
 /*
+ * Same as qsa_forward_ex / qsa_backward_ex (dk / dv FP32 as in
+ * qsa_backward_fp32kv when kv_fp32 is nonzero), with K/V that may still be in
+ * flight: `kv_ready` (a cudaEvent_t, or NULL for none) is an event the caller
+ * records once k and v hold their values, for instance on the stream of a K/V
+ * all-gather.  The call enqueues its route work (which reads neither) first,
+ * then makes `stream` wait for kv_ready before the first kernel that reads k or
+ * v (the forward attention; the backward's dQ), so that the gather runs under
+ * the route kernels.  The wait is a cudaStreamWaitEvent on `stream`: the host
+ * never blocks.  Stage events as in the _ex calls; the wait follows stage 0 of
+ * the forward and stage 2 of the backward.  The context-parallel layout of the
+ * "flex_qsa" and "fa4_qsa" pages (local queries against gathered global K/V)
+ * is what it serves; the pages have no such call.  A failed wait returns
+ * QSA_ERR_CUDA.
+ */
+qsa_status_t qsa_forward_kvwait(const void* q, const void* k, const void* v, const int32_t* routes,
+                                int64_t T, int64_t T_kv, int H, int G, int n_sel, float scale,
+                                void* out, float* lse,
+                                void* workspace, size_t workspace_bytes, qsa_stream_t stream,
+                                qsa_event_t kv_ready, const qsa_event_t* stage_events, int n_stage_events);
+qsa_status_t qsa_backward_kvwait(const void* grad_out, const void* q, const void* k, const void* v,
+                                 const void* out, const float* lse, const int32_t* routes,
+                                 int64_t T, int64_t T_kv, int H, int G, int n_sel, float scale,
+                                 void* dq, void* dk, void* dv, int kv_fp32,
+                                 void* workspace, size_t workspace_bytes, qsa_stream_t stream,
+                                 qsa_event_t kv_ready, const qsa_event_t* stage_events, int n_stage_events);
+
+/*
  * Number of kernels one qsa_forward (backward = 0) or qsa_backward (backward = 1)
- * call enqueues for these sizes, not counting the backward's cudaMemsetAsync
- * nodes (one for its counters, and a second one for the tile masks when T_kv
- * exceeds 8192 tiles of 128 keys).  The forward launches 2 (route rows,
- * attention); the backward 8 (route rows, tile masks, column scans of the
- * masks, tile-pointer scan, tile fill, work lists, dQ, dK/dV).  Returns 0 for
- * sizes the calls reject.  For instrumentation and for sizing CUDA graphs; the
- * pages have no counterpart.
+ * call enqueues for these sizes, not counting the backward's one cudaMemsetAsync
+ * node (its counters and tile masks).  The forward launches 2 (route rows,
+ * attention); the backward 7 (route rows with the tile masks, column scans of
+ * the masks, tile-pointer scan, tile fill, work lists, dQ, dK/dV).  Returns 0
+ * for sizes the calls reject.  For instrumentation and for sizing CUDA graphs;
+ * the pages have no counterpart.
  */
 int qsa_launch_count(int64_t T, int64_t T_kv, int H, int G, int n_sel, int backward);
 

@@ -52,4 +52,4 @@ def test_program_against_the_library(lib_built, tmp_path, compiler, flags, suffi
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, (r.stdout, r.stderr)
     version, status, launches = r.stdout.strip().split("|")
-    assert "sm_100a" in version and status == "QSA_ERR_MISALIGNED" and int(launches) == 8
+    assert "sm_100a" in version and status == "QSA_ERR_MISALIGNED" and int(launches) == 7

@@ -67,6 +67,41 @@ def test_cp_single_rank_reproduces_plain_calls():
         dist.destroy_process_group()
 
 
+@pytest.mark.parametrize("kv_fp32", [False, True])
+def test_kv_ready_event_orders_the_kv_reads(kv_fp32):
+    """K/V written on another stream behind a long wait: calls given the
+    writer's event return exactly what calls on ready K/V return (a call that
+    read K/V before the event would see the zero-filled buffers)."""
+    wl, routes, q, k, v, do = _inputs("thd16k", 1024)
+    out, lse = qsa.forward(q, k, v, routes, wl.scale)
+    ref = qsa.backward(do, q, k, v, out, lse, routes, wl.scale, kv_fp32=kv_fp32)
+    torch.cuda.synchronize()
+    main = torch.cuda.current_stream()
+
+    def late_kv():
+        kb, vb = torch.zeros_like(k), torch.zeros_like(v)
+        side = torch.cuda.Stream()
+        side.wait_stream(main)
+        with torch.cuda.stream(side):
+            torch.cuda._sleep(100_000_000)  # a bounded spin, tens of milliseconds
+            kb.copy_(k)
+            vb.copy_(v)
+            ready = torch.cuda.Event()
+            ready.record(side)
+        kb.record_stream(main)
+        vb.record_stream(main)
+        return kb, vb, ready
+
+    kb, vb, ready = late_kv()
+    o2, l2 = qsa.forward(q, kb, vb, routes, wl.scale, kv_ready=ready)
+    kb, vb, ready = late_kv()
+    got = qsa.backward(do, q, kb, vb, out, lse, routes, wl.scale, kv_fp32=kv_fp32, kv_ready=ready)
+    torch.cuda.synchronize()
+    assert torch.equal(o2, out) and torch.equal(l2, lse)
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
+
+
 def _rne_bf16_bits(x32: np.ndarray) -> np.ndarray:
     """Round-to-nearest-even of FP32 to BF16, as bit patterns: add half an ulp of
     the BF16 result (minus one when the kept part is even, so that exact ties go

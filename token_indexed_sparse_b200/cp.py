@@ -18,8 +18,12 @@ local queries.  Backward: all-gather again, run the backward with FP32 dK/dV
 reduce-scatter those FP32 partials so that every rank receives the summed
 gradients of its own K/V slice, rounded to BF16 once.  The collectives are
 ``torch.distributed`` (NCCL over NVLink on GPUs); the attention itself is the
-library's CUDA path.  The local compute is a parameter only so that the
-collective plumbing can be exercised on CPU processes.
+library's CUDA path.  With NCCL the all-gathers run on a side stream and the
+library calls get their completion as an event: the route preprocessing, which
+reads no K/V, runs under the gather, and only the first kernel that reads K/V
+waits (qsa_forward_kvwait / qsa_backward_kvwait).  The local compute is a
+parameter only so that the collective plumbing can be exercised on CPU
+processes.
 """
 
 from __future__ import annotations
@@ -81,6 +85,30 @@ def _reduce_scatter_rows(x: torch.Tensor, group=None) -> torch.Tensor:
     return y[rank * n:(rank + 1) * n].clone()
 
 
+def _streamed(group, x: torch.Tensor) -> bool:
+    """Whether the collectives run on CUDA streams (NCCL, device tensors)."""
+    return x.is_cuda and dist.get_backend(group) == "nccl"
+
+
+def _gather_kv_async(k_local, v_local, group=None):
+    """All-gathers K and V on a side stream; returns ``(k, v, ready)`` where the
+    event ``ready`` fires once both are complete.  Nothing on the current
+    stream waits for it: the caller hands it to the library call."""
+    main = torch.cuda.current_stream(k_local.device)
+    side = torch.cuda.Stream(device=k_local.device)
+    side.wait_stream(main)  # the local slices are written on the current stream
+    with torch.cuda.stream(side):
+        k = _all_gather_rows(k_local, group)
+        v = _all_gather_rows(v_local, group)
+        ready = torch.cuda.Event()
+        ready.record(side)
+    for t in (k, v):  # allocated on the side stream, read on the current one
+        t.record_stream(main)
+    for t in (k_local, v_local):
+        t.record_stream(side)
+    return k, v, ready
+
+
 def cp_forward(q, k_local, v_local, routes, scale: float, group=None, local_forward=None):
     """Forward of this rank's query rows against the gathered global K/V.
 
@@ -90,6 +118,9 @@ def cp_forward(q, k_local, v_local, routes, scale: float, group=None, local_forw
     """
     if local_forward is None:
         from . import qsa
+        if _streamed(group, k_local):
+            k, v, ready = _gather_kv_async(k_local, v_local, group)
+            return qsa.forward(q, k, v, routes, scale, kv_ready=ready)
         local_forward = qsa.forward
     k = _all_gather_rows(k_local, group)
     v = _all_gather_rows(v_local, group)
@@ -109,14 +140,19 @@ def cp_backward(grad_out, q, k_local, v_local, out, lse, routes, scale: float, g
     """
     if local_backward is None or final_cast is None:
         from . import qsa
-    if local_backward is None:
-        def local_backward(go, q_, k_, v_, o_, l_, r_, s_):
-            return qsa.backward(go, q_, k_, v_, o_, l_, r_, s_, kv_fp32=True)
     if final_cast is None:
         final_cast = qsa.cast_f32_to_bf16
-    k = _all_gather_rows(k_local, group)
-    v = _all_gather_rows(v_local, group)
-    dq, dk_part, dv_part = local_backward(grad_out, q, k, v, out, lse, routes, scale)
+    if local_backward is None and _streamed(group, k_local):
+        k, v, ready = _gather_kv_async(k_local, v_local, group)
+        dq, dk_part, dv_part = qsa.backward(grad_out, q, k, v, out, lse, routes, scale, kv_fp32=True,
+                                            kv_ready=ready)
+    else:
+        if local_backward is None:
+            def local_backward(go, q_, k_, v_, o_, l_, r_, s_):
+                return qsa.backward(go, q_, k_, v_, o_, l_, r_, s_, kv_fp32=True)
+        k = _all_gather_rows(k_local, group)
+        v = _all_gather_rows(v_local, group)
+        dq, dk_part, dv_part = local_backward(grad_out, q, k, v, out, lse, routes, scale)
     if dk_part.dtype not in (torch.float32, torch.float64) or dv_part.dtype != dk_part.dtype:
         raise TypeError("local_backward must return FP32 (or FP64) dK/dV partials")
     dk = final_cast(_reduce_scatter_rows(dk_part, group))

@@ -73,12 +73,12 @@ Layout make_layout(int64_t T, int64_t T_kv, int H, int G, int n_sel, bool backwa
   if (backward) {
     dkdv_phases(T, H, &L.P, &L.C);
     L.tile_ctr = take(tile_ctr_ints(static_cast<int64_t>(nt), L.P, G) * 4);
+    L.lists = take(qsa::tile_lists_bytes(T, T_kv));  // tile masks first (zeroed with the counters), block bases
     L.tile_ptr = take((nt + 1) * 4);
     L.tile_fill = take(nt * 4);
     L.tile_ent = take(pairs * 8);  // at most one entry per routed pair
     L.delta = take(static_cast<size_t>(T) * H * 4);
     L.pds = take(pairs * G * 48);  // BF16 [P | dS] of every routed pair, 12 heads each
-    L.lists = take(qsa::tile_lists_bytes(T, T_kv));  // masks and block bases of the tile lists
     L.wl = take(static_cast<size_t>(L.P) * nt * 16);
     L.partial = take(nt * G * 2 * 128 * 256 * 4);  // FP32 dK and dV of every (tile, group)
   }
@@ -110,12 +110,41 @@ struct StageEvents {
 
 }  // namespace
 
+// The forward sequence.
+static qsa_status_t forward_impl(const void* q, const void* k, const void* v, const int32_t* routes, int64_t T,
+                                 int64_t T_kv, int H, int G, int n_sel, float scale, void* out, float* lse,
+                                 void* workspace, size_t workspace_bytes, qsa_stream_t stream,
+                                 const qsa_event_t* stage_events, int n_stage_events, qsa_event_t kv_ready) {
+  if (!q || !k || !v || !routes || !out || !lse || !workspace) return QSA_ERR_INVALID_ARGUMENT;
+  const qsa_status_t st = check_sizes(T, T_kv, H, G, n_sel);
+  if (st != QSA_OK) return st;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return QSA_ERR_INVALID_ARGUMENT;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(routes, 4) ||
+      !aligned(lse, 4) || !aligned(workspace, 256))
+    return QSA_ERR_MISALIGNED;
+  const Layout L = make_layout(T, T_kv, H, G, n_sel, false);
+  if (workspace_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* status = at<int>(workspace, L.status);
+  int32_t* row_cnt = at<int32_t>(workspace, L.row_cnt);
+  int32_t* row_cols = at<int32_t>(workspace, L.row_cols);
+  const StageEvents ev{stage_events, n_stage_events, s};
+  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 2, status, nullptr, nullptr,
+                                 nullptr, H, nullptr, s));
+  QSA_TRY(ev.mark(0));
+  // k and v are read from here on; the route work above ran without them
+  if (kv_ready != nullptr) QSA_TRY(cudaStreamWaitEvent(s, reinterpret_cast<cudaEvent_t>(kv_ready), 0));
+  QSA_TRY(qsa::launch_forward(q, k, v, row_cnt, row_cols, T, G, n_sel, scale, out, lse, status, s));
+  QSA_TRY(ev.mark(1));
+  return QSA_OK;
+}
+
 // The backward sequence; dk / dv are BF16, or FP32 when kv_f32.
 static qsa_status_t backward_impl(const void* grad_out, const void* q, const void* k, const void* v, const void* out,
                            const float* lse, const int32_t* routes, int64_t T, int64_t T_kv, int H, int G, int n_sel,
                            float scale, void* dq, void* dk, void* dv, bool kv_f32, void* workspace,
                            size_t workspace_bytes, qsa_stream_t stream, const qsa_event_t* stage_events,
-                           int n_stage_events) {
+                           int n_stage_events, qsa_event_t kv_ready) {
   if (!grad_out || !q || !k || !v || !out || !lse || !routes || !dq || !dk || !dv || !workspace)
     return QSA_ERR_INVALID_ARGUMENT;
   const qsa_status_t st = check_sizes(T, T_kv, H, G, n_sel);
@@ -145,14 +174,17 @@ static qsa_status_t backward_impl(const void* grad_out, const void* q, const voi
   int4* wl = at<int4>(workspace, L.wl);
   float* partial = at<float>(workspace, L.partial);
   const StageEvents ev{stage_events, n_stage_events, s};
-  QSA_TRY(cudaMemsetAsync(tile_cnt, 0, tile_ctr_ints(nt, L.P, G) * 4, s));
+  // one memset: the counters and the tile masks after them
+  QSA_TRY(cudaMemsetAsync(tile_cnt, 0, L.lists - L.tile_ctr + qsa::tile_masks_bytes(T, T_kv), s));
   QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 0, status, grad_out, out, delta,
-                                 H, s));
+                                 H, static_cast<unsigned long long*>(lists), s));
   QSA_TRY(ev.mark(0));
   QSA_TRY(qsa::launch_tile_lists(row_cnt, row_cols, T, n_sel, nt, lists, tile_cnt, tile_ptr, tile_fill, tile_ent, s));
   QSA_TRY(ev.mark(1));
   QSA_TRY(qsa::launch_tile_worklist(tile_ptr, lists, T, nt, T_kv, G, L.P, L.C, wl_cnt, wl, dk, dv, kv_f32, s));
   QSA_TRY(ev.mark(2));
+  // k and v are read from here on; the route work above ran without them
+  if (kv_ready != nullptr) QSA_TRY(cudaStreamWaitEvent(s, reinterpret_cast<cudaEvent_t>(kv_ready), 0));
   QSA_TRY(qsa::launch_backward_dq(grad_out, q, k, v, lse, delta, row_cnt, row_cols, T, G, n_sel, scale, dq, pds,
                                   s));
   QSA_TRY(ev.mark(3));
@@ -199,26 +231,16 @@ qsa_status_t qsa_forward_ex(const void* q, const void* k, const void* v, const i
                             int64_t T_kv, int H, int G, int n_sel, float scale, void* out, float* lse,
                             void* workspace, size_t workspace_bytes, qsa_stream_t stream,
                             const qsa_event_t* stage_events, int n_stage_events) {
-  if (!q || !k || !v || !routes || !out || !lse || !workspace) return QSA_ERR_INVALID_ARGUMENT;
-  const qsa_status_t st = check_sizes(T, T_kv, H, G, n_sel);
-  if (st != QSA_OK) return st;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return QSA_ERR_INVALID_ARGUMENT;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(routes, 4) ||
-      !aligned(lse, 4) || !aligned(workspace, 256))
-    return QSA_ERR_MISALIGNED;
-  const Layout L = make_layout(T, T_kv, H, G, n_sel, false);
-  if (workspace_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  int* status = at<int>(workspace, L.status);
-  int32_t* row_cnt = at<int32_t>(workspace, L.row_cnt);
-  int32_t* row_cols = at<int32_t>(workspace, L.row_cols);
-  const StageEvents ev{stage_events, n_stage_events, s};
-  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 2, status, nullptr, nullptr,
-                                 nullptr, H, s));
-  QSA_TRY(ev.mark(0));
-  QSA_TRY(qsa::launch_forward(q, k, v, row_cnt, row_cols, T, G, n_sel, scale, out, lse, status, s));
-  QSA_TRY(ev.mark(1));
-  return QSA_OK;
+  return forward_impl(q, k, v, routes, T, T_kv, H, G, n_sel, scale, out, lse, workspace, workspace_bytes, stream,
+                      stage_events, n_stage_events, nullptr);
+}
+
+qsa_status_t qsa_forward_kvwait(const void* q, const void* k, const void* v, const int32_t* routes, int64_t T,
+                                int64_t T_kv, int H, int G, int n_sel, float scale, void* out, float* lse,
+                                void* workspace, size_t workspace_bytes, qsa_stream_t stream, qsa_event_t kv_ready,
+                                const qsa_event_t* stage_events, int n_stage_events) {
+  return forward_impl(q, k, v, routes, T, T_kv, H, G, n_sel, scale, out, lse, workspace, workspace_bytes, stream,
+                      stage_events, n_stage_events, kv_ready);
 }
 
 qsa_status_t qsa_backward(const void* grad_out, const void* q, const void* k, const void* v, const void* out,
@@ -235,7 +257,16 @@ qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k,
                              size_t workspace_bytes, qsa_stream_t stream, const qsa_event_t* stage_events,
                              int n_stage_events) {
   return backward_impl(grad_out, q, k, v, out, lse, routes, T, T_kv, H, G, n_sel, scale, dq, dk, dv, false, workspace,
-                       workspace_bytes, stream, stage_events, n_stage_events);
+                       workspace_bytes, stream, stage_events, n_stage_events, nullptr);
+}
+
+qsa_status_t qsa_backward_kvwait(const void* grad_out, const void* q, const void* k, const void* v, const void* out,
+                                 const float* lse, const int32_t* routes, int64_t T, int64_t T_kv, int H, int G,
+                                 int n_sel, float scale, void* dq, void* dk, void* dv, int kv_fp32, void* workspace,
+                                 size_t workspace_bytes, qsa_stream_t stream, qsa_event_t kv_ready,
+                                 const qsa_event_t* stage_events, int n_stage_events) {
+  return backward_impl(grad_out, q, k, v, out, lse, routes, T, T_kv, H, G, n_sel, scale, dq, dk, dv, kv_fp32 != 0,
+                       workspace, workspace_bytes, stream, stage_events, n_stage_events, kv_ready);
 }
 
 qsa_status_t qsa_backward_fp32kv(const void* grad_out, const void* q, const void* k, const void* v, const void* out,
@@ -243,13 +274,13 @@ qsa_status_t qsa_backward_fp32kv(const void* grad_out, const void* q, const void
                                  int n_sel, float scale, void* dq, float* dk, float* dv, void* workspace,
                                  size_t workspace_bytes, qsa_stream_t stream) {
   return backward_impl(grad_out, q, k, v, out, lse, routes, T, T_kv, H, G, n_sel, scale, dq, dk, dv, true, workspace,
-                       workspace_bytes, stream, nullptr, 0);
+                       workspace_bytes, stream, nullptr, 0, nullptr);
 }
 
 int qsa_launch_count(int64_t T, int64_t T_kv, int H, int G, int n_sel, int backward) {
   if (check_sizes(T, T_kv, H, G, n_sel) != QSA_OK) return 0;
-  // backward: route rows, tile masks, column scans, tile scan, tile fill, work lists, dQ, dK/dV
-  return backward ? 8 : 2;
+  // backward: route rows (+ tile masks), column scans, tile-pointer scan, tile fill, work lists, dQ, dK/dV
+  return backward ? 7 : 2;
 }
 
 qsa_status_t qsa_bitmap_routes(const uint8_t* sel_blocks, const int32_t* lo, const int32_t* hi,
@@ -320,7 +351,7 @@ qsa_status_t qsa_route_plan(const int32_t* routes, int64_t T, int64_t T_kv, int 
   int32_t* phase_ptr = at<int32_t>(scratch, 2 * align256(static_cast<size_t>(nq) * 4));
   QSA_TRY(cudaMemsetAsync(quad_cnt, 0, static_cast<size_t>(nq) * 4, s));
   QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, quad_cnt, 2, nullptr, nullptr, nullptr,
-                                 nullptr, qsa::kHeadsPerGroup, s));
+                                 nullptr, qsa::kHeadsPerGroup, nullptr, s));
   QSA_TRY(qsa::launch_quad_scan(quad_cnt, nq, quad_ptr, quad_fill, s));
   QSA_TRY(qsa::launch_quad_fill(row_cnt, row_cols, T, n_sel, quad_fill, quad_ent, s));
   QSA_TRY(qsa::launch_quad_sort(quad_ptr, nq, quad_ent, 1, static_cast<int>(T), phase_ptr, s));
@@ -338,7 +369,7 @@ qsa_status_t qsa_union_plan(const int32_t* routes, int64_t T, int64_t T_kv, int 
     return QSA_ERR_MISALIGNED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 0, nullptr, nullptr, nullptr,
-                                 nullptr, qsa::kHeadsPerGroup, s));
+                                 nullptr, qsa::kHeadsPerGroup, nullptr, s));
   QSA_TRY(qsa::launch_union_lists(row_cnt, row_cols, T, n_sel, qsa::union_group(n_sel), ucnt, ukey, uown, s));
   return QSA_OK;
 }
@@ -364,8 +395,9 @@ qsa_status_t qsa_tile_plan(const int32_t* routes, int64_t T, int64_t T_kv, int n
   int32_t* tile_cnt = static_cast<int32_t*>(scratch);
   int32_t* tile_fill = at<int32_t>(scratch, align256(static_cast<size_t>(nt) * 4));
   void* lists = at<void>(scratch, 2 * align256(static_cast<size_t>(nt) * 4));
+  QSA_TRY(cudaMemsetAsync(lists, 0, qsa::tile_masks_bytes(T, T_kv), s));
   QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 0, nullptr, nullptr, nullptr,
-                                 nullptr, qsa::kHeadsPerGroup, s));
+                                 nullptr, qsa::kHeadsPerGroup, static_cast<unsigned long long*>(lists), s));
   QSA_TRY(qsa::launch_tile_lists(row_cnt, row_cols, T, n_sel, nt, lists, tile_cnt, tile_ptr, tile_fill, tile_ent, s));
   return QSA_OK;
 }

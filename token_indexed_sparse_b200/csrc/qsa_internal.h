@@ -8,15 +8,18 @@ namespace qsa {
 
 // Route preprocessing (qsa_routes.cu).
 // Per-row ascending, de-duplicated valid route IDs; optionally counts, per
-// bucket of 2^cnt_shift consecutive keys (2: quads, 7: 128-key tiles), the rows
-// that meet it (bucket_cnt must be zeroed by the caller).
+// bucket of 2^cnt_shift consecutive keys (2: quads), the rows that meet it
+// (bucket_cnt must be zeroed by the caller).
 // `status` (nullable) is zeroed by this kernel, the first of every call.  With
 // `delta` non-null it also writes delta[t, h] = sum_d dO[t,h,d] * out[t,h,d]
-// (FP32 from the BF16 tensors, [T, H]).
+// (FP32 from the BF16 tensors, [T, H]).  With `tile_masks` non-null (the first
+// tile_masks_bytes of a tile-lists scratch, zeroed by the caller) it sets row
+// t's bit in the mask of (t / 64, tile) for every 128-key tile the row meets,
+// the input of launch_tile_lists.
 cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel,
                               int32_t* row_cnt, int32_t* row_cols, int32_t* bucket_cnt, int cnt_shift,
                               int* status, const void* dout, const void* out, float* delta, int H,
-                              cudaStream_t s);
+                              unsigned long long* tile_masks, cudaStream_t s);
 // quad_cnt -> quad_ptr (exclusive scan, n_quads+1 entries) and quad_fill (copy
 // of quad_ptr used as fill cursors).
 cudaError_t launch_quad_scan(const int32_t* quad_cnt, int64_t n_quads, int32_t* quad_ptr,
@@ -31,10 +34,12 @@ cudaError_t launch_quad_sort(const int32_t* quad_ptr, int64_t n_quads, int64_t* 
 // The key->query transpose over 128-key tiles: one entry per (row, tile) pair,
 // (t << 32) | (i0 << 8) | (n - 1) with row_cols[t][i0, i0 + n) the row's keys in
 // the tile, every list in ascending query order without a sort: per block of 64
-// rows a mask of the rows meeting each tile, block bases from a scan down each
-// tile's column, ranks from mask popcounts.  `scratch` holds the masks and the
-// block bases (tile_lists_bytes); tile_cnt, tile_ptr (n_tiles + 1) and
-// tile_fill (n_tiles) are written.
+// rows a mask of the rows meeting each tile (set by launch_route_rows), block
+// bases from a scan down each tile's column, ranks from mask popcounts.
+// `scratch` holds the masks (its first tile_masks_bytes) and the block bases
+// (tile_lists_bytes in all); tile_cnt, tile_ptr (n_tiles + 1) and tile_fill
+// (n_tiles) are written.
+size_t tile_masks_bytes(int64_t T, int64_t T_kv);
 size_t tile_lists_bytes(int64_t T, int64_t T_kv);
 cudaError_t launch_tile_lists(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel,
                               int64_t n_tiles, void* scratch, int32_t* tile_cnt, int32_t* tile_ptr,

@@ -120,7 +120,7 @@ extern "C" qsa_status_t qsa_forward_noalloc(const void* q, const void* k, const 
   int32_t* row_cols = reinterpret_cast<int32_t*>(base + 256 + align256(static_cast<size_t>(T) * 4));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 2, status, nullptr, nullptr, nullptr,
-                             H, s) != cudaSuccess)
+                             H, nullptr, s) != cudaSuccess)
     return QSA_ERR_CUDA;
   if (qsa::launch_forward(q, k, v, row_cnt, row_cols, T, G, n_sel, scale, out, lse, status, s) != cudaSuccess)
     return QSA_ERR_CUDA;

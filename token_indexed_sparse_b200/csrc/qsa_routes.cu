@@ -149,24 +149,66 @@ __device__ __forceinline__ void warp_sort(int32_t (&v)[NPL], int lane) {
   }
 }
 
+// Keys per 128-key tile: 2^kTileShift.  Query rows form blocks of kBlockRows
+// for the tile masks (one 64-bit mask per block and tile).
+constexpr int kTileShift = 7;
+constexpr int kBlockRows = 64;
+constexpr int kRowWarps = 8;  // rows (warps) per CTA of route_rows_warp_kernel
+
+// Sets row t's bit in the mask of (its 64-row block, 128-key tile tl); the
+// masks [ceil(T / 64), n_tiles] are zeroed by the caller.
+__device__ __forceinline__ void mark_tile(unsigned long long* masks, int64_t n_tiles, int64_t t, int32_t tl) {
+  static_assert(kBlockRows == 64, "one 64-bit mask per block of rows");
+  atomicOr(masks + (t / kBlockRows) * n_tiles + tl, 1ull << (t % kBlockRows));
+}
+
+// delta[t, h] = rowsum(dO * out) for heads h0 .. h0 + 3 of row t, h0 = first,
+// first + step, ... below H (H a multiple of 4), by one warp with the four
+// heads' loads in flight together.
+__device__ __forceinline__ void row_delta(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out,
+                                          float* __restrict__ delta, int64_t t, int H, int lane, int first, int step) {
+  for (int h0 = first; h0 < H; h0 += step) {
+    uint4 a[4], b[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t off = (t * H + h0 + j) * kHeadDim + lane * 8;
+      a[j] = __ldg(reinterpret_cast<const uint4*>(dout + off));
+      b[j] = __ldg(reinterpret_cast<const uint4*>(out + off));
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float x = bf16_lo(a[j].x) * bf16_lo(b[j].x) + bf16_hi(a[j].x) * bf16_hi(b[j].x) +
+                bf16_lo(a[j].y) * bf16_lo(b[j].y) + bf16_hi(a[j].y) * bf16_hi(b[j].y) +
+                bf16_lo(a[j].z) * bf16_lo(b[j].z) + bf16_hi(a[j].z) * bf16_hi(b[j].z) +
+                bf16_lo(a[j].w) * bf16_lo(b[j].w) + bf16_hi(a[j].w) * bf16_hi(b[j].w);
+      x = warp_sum(x);
+      if (lane == 0) delta[t * H + h0 + j] = x;
+    }
+  }
+}
+
 // One warp per query row (rows of up to 32*NPL route slots): filter, sort in
-// registers, de-duplicate, compact; optional per-bucket row counts (a bucket is
-// 2^cnt_shift consecutive keys: a quad or a 128-key tile) and delta.
+// registers, de-duplicate, compact; optionally per-bucket row counts (a bucket
+// is 2^cnt_shift consecutive keys), the row's bits in the tile masks, and delta.
+// (A shared-memory bitmap of the row's key range in place of the sort, with
+// word popcounts scanned across the warp, ran the seq32k rows in 0.30 ms
+// against 0.25 ms for this sort: the bit-by-bit read-back diverges across lanes.)
 template <int NPL>
-__global__ void __launch_bounds__(256) route_rows_warp_kernel(
+__global__ void __launch_bounds__(kRowWarps * 32, 3) route_rows_warp_kernel(
     const int32_t* __restrict__ routes, int64_t T, int32_t T_kv, int n_sel, int32_t* __restrict__ row_cnt,
     int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt, int cnt_shift, int* __restrict__ status,
     const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out, float* __restrict__ delta,
-    int H) {
+    int H, unsigned long long* __restrict__ masks, int64_t n_tiles) {
   const int lane = threadIdx.x & 31;
   const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
   if (t >= T) return;
   const int32_t* row = routes + t * n_sel;
+  int32_t* dst = row_cols + t * n_sel;
   int32_t v[NPL];
 #pragma unroll
-  for (int r = 0; r < NPL; ++r) {
-    const int i = lane * NPL + r;
+  for (int r = 0; r < NPL; ++r) {  // coalesced: the sort does not care where a value starts
+    const int i = r * 32 + lane;
     int32_t x = INT_MAX;
     if (i < n_sel) {
       const int32_t y = __ldg(row + i);
@@ -175,7 +217,8 @@ __global__ void __launch_bounds__(256) route_rows_warp_kernel(
     v[r] = x;
   }
   warp_sort<NPL>(v, lane);
-  // previous element of v[0] lives in the previous lane's v[NPL - 1]
+  // element e = lane * NPL + r; the previous element of v[0] is the previous
+  // lane's v[NPL - 1]
   int32_t prev = __shfl_up_sync(0xffffffffu, v[NPL - 1], 1);
   if (lane == 0) prev = INT_MIN;
   int mine = 0;
@@ -187,6 +230,8 @@ __global__ void __launch_bounds__(256) route_rows_warp_kernel(
       ++mine;
       if (quad_cnt != nullptr && (p == INT_MIN || (p >> cnt_shift) != (x >> cnt_shift)))
         atomicAdd(quad_cnt + (x >> cnt_shift), 1);
+      if (masks != nullptr && (p == INT_MIN || (p >> kTileShift) != (x >> kTileShift)))
+        mark_tile(masks, n_tiles, t, x >> kTileShift);
     }
   }
   int incl = mine;
@@ -196,27 +241,15 @@ __global__ void __launch_bounds__(256) route_rows_warp_kernel(
     if (lane >= o) incl += y;
   }
   int pos = incl - mine;
-  int32_t* dst = row_cols + t * n_sel;
 #pragma unroll
   for (int r = 0; r < NPL; ++r) {
     const int32_t p = r == 0 ? prev : v[r - 1];
     const int32_t x = v[r];
     if (x != INT_MAX && x != p) dst[pos++] = x;
   }
-  if (lane == 31) row_cnt[t] = incl;
-
-  if (delta != nullptr) {  // delta[t, h] = rowsum(dO * out)
-    for (int h = 0; h < H; ++h) {
-      const int64_t off = (t * H + h) * kHeadDim + lane * 8;
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(dout + off));
-      const uint4 b = __ldg(reinterpret_cast<const uint4*>(out + off));
-      float x = bf16_lo(a.x) * bf16_lo(b.x) + bf16_hi(a.x) * bf16_hi(b.x) + bf16_lo(a.y) * bf16_lo(b.y) +
-                bf16_hi(a.y) * bf16_hi(b.y) + bf16_lo(a.z) * bf16_lo(b.z) + bf16_hi(a.z) * bf16_hi(b.z) +
-                bf16_lo(a.w) * bf16_lo(b.w) + bf16_hi(a.w) * bf16_hi(b.w);
-      x = warp_sum(x);
-      if (lane == 0) delta[t * H + h] = x;
-    }
-  }
+  const int cnt = __shfl_sync(0xffffffffu, incl, 31);
+  if (lane == 0) row_cnt[t] = cnt;
+  if (delta != nullptr) row_delta(dout, out, delta, t, H, lane, 0, 4);
 }
 
 // One block per query row: filter invalid IDs, sort, de-duplicate, compact.
@@ -224,7 +257,7 @@ __global__ void __launch_bounds__(kRowThreads) route_rows_kernel(
     const int32_t* __restrict__ routes, int32_t T_kv, int n_sel, int n2,
     int32_t* __restrict__ row_cnt, int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt, int cnt_shift,
     int* __restrict__ status, const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out,
-    float* __restrict__ delta, int H) {
+    float* __restrict__ delta, int H, unsigned long long* __restrict__ masks, int64_t n_tiles) {
   extern __shared__ int32_t sv[];  // n2 values, then 32 ints of scan scratch
   int* scratch = sv + n2;
   const int64_t t = blockIdx.x;
@@ -251,6 +284,8 @@ __global__ void __launch_bounds__(kRowThreads) route_rows_kernel(
       ++mine;
       if (quad_cnt != nullptr && (i == 0 || (sv[i - 1] >> cnt_shift) != (x >> cnt_shift)))
         atomicAdd(quad_cnt + (x >> cnt_shift), 1);
+      if (masks != nullptr && (i == 0 || (sv[i - 1] >> kTileShift) != (x >> kTileShift)))
+        mark_tile(masks, n_tiles, t, x >> kTileShift);
     }
   }
   int total;
@@ -261,20 +296,7 @@ __global__ void __launch_bounds__(kRowThreads) route_rows_kernel(
     if (x != INT_MAX && (i == 0 || sv[i - 1] != x)) dst[pos++] = x;
   }
   if (threadIdx.x == 0) row_cnt[t] = total;
-
-  if (delta != nullptr) {  // delta[t, h] = rowsum(dO * out), one warp per head row
-    const int lane = threadIdx.x & 31;
-    for (int h = threadIdx.x >> 5; h < H; h += blockDim.x >> 5) {
-      const int64_t off = (t * H + h) * kHeadDim + lane * 8;
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(dout + off));
-      const uint4 b = __ldg(reinterpret_cast<const uint4*>(out + off));
-      float x = bf16_lo(a.x) * bf16_lo(b.x) + bf16_hi(a.x) * bf16_hi(b.x) + bf16_lo(a.y) * bf16_lo(b.y) +
-                bf16_hi(a.y) * bf16_hi(b.y) + bf16_lo(a.z) * bf16_lo(b.z) + bf16_hi(a.z) * bf16_hi(b.z) +
-                bf16_lo(a.w) * bf16_lo(b.w) + bf16_hi(a.w) * bf16_hi(b.w);
-      x = warp_sum(x);
-      if (lane == 0) delta[t * H + h] = x;
-    }
-  }
+  if (delta != nullptr) row_delta(dout, out, delta, t, H, threadIdx.x & 31, 4 * (threadIdx.x >> 5), 4 * (blockDim.x >> 5));
 }
 
 // Single block: exclusive scan of quad counts (n_quads + 1 offsets).
@@ -371,65 +393,15 @@ __global__ void __launch_bounds__(kSortThreads) quad_sort_kernel(const int32_t* 
 // Entry of a (query row, tile) pair, the "union" of the row's keys in the tile:
 // (t << 32) | (i0 << 8) | (n - 1), where row_cols[t][i0, i0 + n) are the row's
 // keys inside the tile (ascending, so one contiguous run of the sorted row).
-constexpr int kTileShift = 7;
 
 // Rows come in blocks of 64 (kBlockRows).  Per block and tile, a 64-bit mask of
-// the block's rows that meet the tile; a scan down each tile's column of mask
+// the block's rows that meet the tile (set by the route-rows kernels, which see
+// each row's tiles as they sort it); a scan down each tile's column of mask
 // popcounts gives every block its first slot in the tile's list; an entry's
 // place inside its block is the popcount of the mask below its row.  So every
 // (row, tile) entry is written straight to its place in ascending query order,
 // with no sort and no atomics on the list, and a query phase (a multiple of 64
-// rows) starts at a block's first slot.  With at most kTileBins tiles a block
-// builds its masks in shared memory and writes each one once.
-constexpr int kBlockRows = 64;
-constexpr int kTileBins = 8192;
-
-// Calls f(t, cols, cnt, tile, i) for every i where row t's sorted keys enter a
-// new tile, for the 64 rows of block blockIdx.x spread over the CTA's warps.  A
-// warp reads its row 32 keys at a time, the previous key of each lane coming
-// from its neighbour.
-template <typename F>
-__device__ __forceinline__ void for_block_runs(const int32_t* __restrict__ row_cnt,
-                                               const int32_t* __restrict__ row_cols, int64_t T, int n_sel, F f) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const int rpw = kBlockRows / nw;
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kBlockRows + static_cast<int64_t>(warp) * rpw;
-  for (int r = 0; r < rpw; ++r) {
-    const int64_t t = t0 + r;
-    if (t >= T) return;
-    const int cnt = row_cnt[t];
-    const int32_t* cols = row_cols + t * n_sel;
-    int32_t carry = -1;  // tile of the last key of the previous 32 (none: -1)
-    for (int base = 0; base < cnt; base += 32) {
-      const int i = base + lane;
-      const int32_t tl = i < cnt ? (cols[i] >> kTileShift) : INT_MAX;
-      int32_t prev = __shfl_up_sync(0xffffffffu, tl, 1);
-      if (lane == 0) prev = carry;
-      carry = __shfl_sync(0xffffffffu, tl, 31);
-      if (i < cnt && tl != prev) f(t, cols, cnt, tl, i);
-    }
-  }
-}
-
-// masks[block * n_tiles + tile]: bit (t mod 64) set when row t meets the tile
-// (zeroed by the caller when n_tiles > kTileBins).
-__global__ void __launch_bounds__(512) tile_mask_kernel(const int32_t* __restrict__ row_cnt,
-                                                        const int32_t* __restrict__ row_cols, int64_t T, int n_sel,
-                                                        int64_t n_tiles, unsigned long long* __restrict__ masks) {
-  extern __shared__ unsigned long long msk[];
-  const bool local = n_tiles <= kTileBins;
-  if (local) {
-    for (int64_t j = threadIdx.x; j < n_tiles; j += blockDim.x) msk[j] = 0ull;
-    __syncthreads();
-  }
-  unsigned long long* dst = masks + static_cast<int64_t>(blockIdx.x) * n_tiles;
-  for_block_runs(row_cnt, row_cols, T, n_sel, [&](int64_t t, const int32_t*, int, int32_t tl, int) {
-    atomicOr(local ? msk + tl : dst + tl, 1ull << (t & 63));
-  });
-  if (!local) return;
-  __syncthreads();
-  for (int64_t j = threadIdx.x; j < n_tiles; j += blockDim.x) dst[j] = msk[j];
-}
+// rows) starts at a block's first slot.
 
 // One warp per tile: exclusive scan of the blocks' mask popcounts down the
 // tile's column (blk_base), and the tile's row count.
@@ -634,14 +606,16 @@ static int next_pow2(int x) {
 
 cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, int n_sel, int32_t* row_cnt,
                               int32_t* row_cols, int32_t* bucket_cnt, int cnt_shift, int* status, const void* dout,
-                              const void* out, float* delta, int H, cudaStream_t s) {
+                              const void* out, float* delta, int H, unsigned long long* tile_masks, cudaStream_t s) {
   const auto* dq = static_cast<const __nv_bfloat16*>(dout);
   const auto* o = static_cast<const __nv_bfloat16*>(out);
-  const unsigned wblocks = static_cast<unsigned>((T + 7) / 8);
+  const unsigned wblocks = static_cast<unsigned>((T + kRowWarps - 1) / kRowWarps);
   const int32_t tkv = static_cast<int32_t>(T_kv);
-#define QSA_ROWS_WARP(NPL)                                                                                       \
-  route_rows_warp_kernel<NPL><<<wblocks, 256, 0, s>>>(routes, T, tkv, n_sel, row_cnt, row_cols, bucket_cnt,     \
-                                                      cnt_shift, status, dq, o, delta, H);                       \
+  const int64_t n_tiles = (T_kv + 127) >> kTileShift;
+#define QSA_ROWS_WARP(NPL)                                                                                         \
+  route_rows_warp_kernel<NPL><<<wblocks, kRowWarps * 32, 0, s>>>(routes, T, tkv, n_sel, row_cnt, row_cols,        \
+                                                                 bucket_cnt, cnt_shift, status, dq, o, delta, H, \
+                                                                 tile_masks, n_tiles);                            \
   return cudaGetLastError()
   if (n_sel <= 64) { QSA_ROWS_WARP(2); }
   if (n_sel <= 128) { QSA_ROWS_WARP(4); }
@@ -657,7 +631,7 @@ cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, in
     if (e != cudaSuccess) return e;
   }
   route_rows_kernel<<<static_cast<unsigned>(T), kRowThreads, smem, s>>>(
-      routes, tkv, n_sel, n2, row_cnt, row_cols, bucket_cnt, cnt_shift, status, dq, o, delta, H);
+      routes, tkv, n_sel, n2, row_cnt, row_cols, bucket_cnt, cnt_shift, status, dq, o, delta, H, tile_masks, n_tiles);
   return cudaGetLastError();
 }
 
@@ -699,33 +673,26 @@ cudaError_t launch_union_lists(const int32_t* row_cnt, const int32_t* row_cols, 
   return cudaGetLastError();
 }
 
-size_t tile_lists_bytes(int64_t T, int64_t T_kv) {
+size_t tile_masks_bytes(int64_t T, int64_t T_kv) {
   const size_t nb = static_cast<size_t>((T + kBlockRows - 1) / kBlockRows);
   const size_t nt = static_cast<size_t>((T_kv + 127) / 128);
-  return nb * nt * 12;  // a mask (8 bytes) and a block base (4 bytes) per (block, tile)
+  return nb * nt * 8;
+}
+
+size_t tile_lists_bytes(int64_t T, int64_t T_kv) {
+  return tile_masks_bytes(T, T_kv) / 8 * 12;  // a mask (8 bytes) and a block base (4 bytes) per (block, tile)
 }
 
 cudaError_t launch_tile_lists(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel,
                               int64_t n_tiles, void* scratch, int32_t* tile_cnt, int32_t* tile_ptr,
                               int32_t* tile_fill, int64_t* tile_ent, cudaStream_t s) {
   const int64_t nb = (T + kBlockRows - 1) / kBlockRows;
-  auto* masks = static_cast<unsigned long long*>(scratch);
-  auto* blk_base = reinterpret_cast<int32_t*>(masks + nb * n_tiles);
+  const auto* masks = static_cast<const unsigned long long*>(scratch);
+  auto* blk_base = reinterpret_cast<int32_t*>(static_cast<unsigned long long*>(scratch) + nb * n_tiles);
   const int threads = n_sel <= 1024 ? 256 : 512;  // 8 rows per warp, or 4 for long rows
-  const bool local = n_tiles <= kTileBins;
-  cudaError_t e;
-  if (!local) {
-    e = cudaMemsetAsync(masks, 0, static_cast<size_t>(nb * n_tiles) * 8, s);
-  } else {
-    e = cudaFuncSetAttribute(tile_mask_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kTileBins * 8));
-  }
-  if (e != cudaSuccess) return e;
-  tile_mask_kernel<<<static_cast<unsigned>(nb), threads, local ? static_cast<size_t>(n_tiles) * 8 : 0, s>>>(
-      row_cnt, row_cols, T, n_sel, n_tiles, masks);
   tile_scan_kernel<<<static_cast<unsigned>((n_tiles * 32 + 255) / 256), 256, 0, s>>>(masks, nb, n_tiles, blk_base,
                                                                                     tile_cnt);
-  e = launch_quad_scan(tile_cnt, n_tiles, tile_ptr, tile_fill, s);
+  cudaError_t e = launch_quad_scan(tile_cnt, n_tiles, tile_ptr, tile_fill, s);
   if (e != cudaSuccess) return e;
   tile_fill_kernel<<<static_cast<unsigned>(nb), threads, 0, s>>>(row_cnt, row_cols, T, n_sel, n_tiles, masks,
                                                                  blk_base, tile_ptr, tile_ent);

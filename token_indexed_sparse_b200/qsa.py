@@ -55,6 +55,11 @@ def library() -> ctypes.CDLL:
     lib.qsa_forward_ex.argtypes = lib.qsa_forward.argtypes + [vp, i32]
     lib.qsa_backward_ex.restype = i32
     lib.qsa_backward_ex.argtypes = lib.qsa_backward.argtypes + [vp, i32]
+    lib.qsa_forward_kvwait.restype = i32
+    lib.qsa_forward_kvwait.argtypes = lib.qsa_forward.argtypes + [vp, vp, i32]
+    lib.qsa_backward_kvwait.restype = i32
+    lib.qsa_backward_kvwait.argtypes = lib.qsa_backward.argtypes[:16] + [i32] + lib.qsa_backward.argtypes[16:] + [
+        vp, vp, i32]
     lib.qsa_launch_count.restype = i32
     lib.qsa_launch_count.argtypes = [i64, i64, i32, i32, i32, i32]
     lib.qsa_bitmap_routes.restype = i32
@@ -168,12 +173,23 @@ def _events(stage_events):
     return (ctypes.c_void_p * len(handles))(*handles), len(handles)
 
 
+def _event_handle(e):
+    """Raw cudaEvent_t of a recorded torch.cuda.Event, or None."""
+    if e is None:
+        return None
+    if e.cuda_event == 0:
+        raise ValueError("kv_ready must be a recorded torch.cuda.Event")
+    return e.cuda_event
+
+
 def forward(q, k, v, routes, scale: float = 1.0 / 16.0, *, out=None, lse=None, workspace=None,
-            stage_events=None):
+            stage_events=None, kv_ready=None):
     """qsa_forward: returns ``(out [T,H,256] bf16, lse [T,H] float32)``.
 
     ``stage_events`` (optional list of torch.cuda.Event) are recorded after the
-    route-sort and attention stages (qsa_forward_ex)."""
+    route-sort and attention stages.  ``kv_ready`` (optional recorded
+    torch.cuda.Event): k and v may still be being written until it fires; the
+    route work runs first and the attention waits for it (qsa_forward_kvwait)."""
     lib = library()
     q = _prep(q, torch.bfloat16, "q")
     k = _prep(k, torch.bfloat16, "k")
@@ -186,20 +202,24 @@ def forward(q, k, v, routes, scale: float = 1.0 / 16.0, *, out=None, lse=None, w
     ws_bytes = lib.qsa_forward_workspace_size(T, T_kv, H, G, n_sel)
     ws = _workspace(ws_bytes, q.device, workspace)
     ev, n_ev = _events(stage_events)
-    st = lib.qsa_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(routes), T, T_kv, H, G, n_sel, float(scale),
-                            _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device), ev, n_ev)
+    st = lib.qsa_forward_kvwait(_ptr(q), _ptr(k), _ptr(v), _ptr(routes), T, T_kv, H, G, n_sel, float(scale),
+                                _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(q.device),
+                                _event_handle(kv_ready), ev, n_ev)
     _check(st, "qsa_forward")
     return out, lse
 
 
 def backward(grad_out, q, k, v, out, lse, routes, scale: float = 1.0 / 16.0, *,
-             dq=None, dk=None, dv=None, workspace=None, stage_events=None, kv_fp32: bool = False):
+             dq=None, dk=None, dv=None, workspace=None, stage_events=None, kv_fp32: bool = False,
+             kv_ready=None):
     """qsa_backward: returns ``(dq, dk, dv)`` (bf16, shapes of q, k, v).
 
     ``stage_events`` (optional, up to 5 torch.cuda.Event) are recorded after
-    each backward stage (qsa_backward_ex).  With ``kv_fp32`` dk and dv are FP32
-    (qsa_backward_fp32kv: the sums before the BF16 rounding, for adding partials
-    from several calls)."""
+    each backward stage.  With ``kv_fp32`` dk and dv are FP32 (the sums before
+    the BF16 rounding, for adding partials from several calls).  ``kv_ready``
+    (optional recorded torch.cuda.Event): k and v may still be being written
+    until it fires; the route work runs first and dQ waits for it
+    (qsa_backward_kvwait)."""
     lib = library()
     grad_out = _prep(grad_out, torch.bfloat16, "grad_out")
     q = _prep(q, torch.bfloat16, "q")
@@ -217,17 +237,11 @@ def backward(grad_out, q, k, v, out, lse, routes, scale: float = 1.0 / 16.0, *,
           else _out(dv, v.shape, kv_dtype, v.device, "dv"))
     ws_bytes = lib.qsa_backward_workspace_size(T, T_kv, H, G, n_sel)
     ws = _workspace(ws_bytes, q.device, workspace)
-    if kv_fp32:
-        if stage_events:
-            raise ValueError("stage events are not recorded by the FP32 dK/dV backward")
-        st = lib.qsa_backward_fp32kv(_ptr(grad_out), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(routes),
-                                     T, T_kv, H, G, n_sel, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
-                                     _ptr(ws), ws.numel(), _stream(q.device))
-    else:
-        ev, n_ev = _events(stage_events)
-        st = lib.qsa_backward_ex(_ptr(grad_out), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(routes),
+    ev, n_ev = _events(stage_events)
+    st = lib.qsa_backward_kvwait(_ptr(grad_out), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(routes),
                                  T, T_kv, H, G, n_sel, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
-                                 _ptr(ws), ws.numel(), _stream(q.device), ev, n_ev)
+                                 1 if kv_fp32 else 0, _ptr(ws), ws.numel(), _stream(q.device),
+                                 _event_handle(kv_ready), ev, n_ev)
     _check(st, "qsa_backward")
     return dq, dk, dv
 
