@@ -7,7 +7,9 @@ A step is one full pass of the hot path on one sequence of the seq32k workload
 (T = 32768 tokens, 24 query heads / 2 KV heads, d = 256, 128 four-token blocks
 = 512 unique routed keys per query, 564 route slots with 10% duplicates):
 route sort/dedup + forward + route transpose + dQ + dK/dV, every kernel of the
-library, inputs resident in HBM.  The metric is selected (query, key) token
+library, inputs resident in HBM.  The backward reuses the forward's sorted route
+lists from the forward's workspace (qsa_backward_saved), as a training step
+keeps them for its backward.  The metric is selected (query, key) token
 pairs per second, N = sum_t |R_t| per step (the two KV groups share the routes).
 
 With N GPUs (torchrun), every rank runs its own sequence (independent problems,
@@ -48,11 +50,11 @@ SPEC_BF16_TFLOPS = 2250.0              # B200 dense BF16 tensor peak (NVIDIA spe
 TRAFFIC = {
     # the timed step's dK/dV launch on seq32k: ncu dram__bytes_read.sum + dram__bytes_write.sum
     # (the dK/dV summary under profiles/); the kernel and the phase sizing of its launch
-    "bwd_dkdv": (13687003648, {
+    "bwd_dkdv": (15083029760, {
         "token_indexed_sparse_b200/csrc/qsa_dkdv_union.cu":
-            "3f17ce8a839d435e88248da8cc1c3393eaa0c76bbf7b119ec93fce2f9c41a17b",
+            "1ebd1ab736b167e165bf20277e70b378f50e0b542b063957dcbdd386bf5619ae",
         "token_indexed_sparse_b200/csrc/qsa_api.cu":
-            "f1767b0adbc801a1f6652ad5362ca555cd832431f6d8ca6a868e67697100fa32",
+            "5d19978cca318f395bf266024013af302738c42098e39431964f7bf1ba901abf",
     }),
 }
 
@@ -70,7 +72,7 @@ def stage_traffic(stage):
 
 
 FWD_STAGES = ["fwd_route_rows", "fwd_attention"]
-BWD_STAGES = ["bwd_route_rows", "bwd_tile_lists", "bwd_tile_worklist", "bwd_dq", "bwd_dkdv"]
+BWD_STAGES = ["bwd_delta_masks", "bwd_tile_lists", "bwd_tile_worklist", "bwd_dq", "bwd_dkdv"]
 
 
 def pass_ms(stage_ms):
@@ -323,8 +325,9 @@ def run_ours(args):
 
     def step(fwd_ev=None, bwd_ev=None):
         qsa.forward(q, k, v, routes, wl.scale, out=out, lse=lse, workspace=ws_f, stage_events=fwd_ev)
+        # the backward reuses the forward's route lists (kept in ws_f) instead of sorting again
         qsa.backward(do, q, k, v, out, lse, routes, wl.scale, dq=dq, dk=dk, dv=dv, workspace=ws_b,
-                     stage_events=bwd_ev)
+                     stage_events=bwd_ev, saved_workspace=ws_f)
 
     for _ in range(args.warmup):
         step()
@@ -409,7 +412,8 @@ def run_ours(args):
                 q_, k_, v_, do_, r_ = d_in[b]
                 o_, l_, dq_, dk_, dv_ = d_res[b]
                 qsa.forward(q_, k_, v_, r_, wl.scale, out=o_, lse=l_, workspace=ws_f)
-                qsa.backward(do_, q_, k_, v_, o_, l_, r_, wl.scale, dq=dq_, dk=dk_, dv=dv_, workspace=ws_b)
+                qsa.backward(do_, q_, k_, v_, o_, l_, r_, wl.scale, dq=dq_, dk=dk_, dv=dv_, workspace=ws_b,
+                             saved_workspace=ws_f)
                 ev_cmp[b].record(stream)
             kk = i - 2
             if 0 <= kk < n_steps:

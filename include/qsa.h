@@ -39,7 +39,8 @@
  *     scratch: nothing needs to be initialised, nothing survives the call,
  *     except the first int32 of the workspace, a status word: once the call's
  *     work has completed on the stream it is 0, or nonzero if a kernel gave up
- *     on a bounded wait (its outputs are then invalid).  Every wait inside the
+ *     on a bounded wait (its outputs are then invalid), and, after a forward
+ *     call, the route lists that qsa_backward_saved can reuse.  Every wait inside the
  *     kernels is bounded, so a fault in the pipeline ends the kernel instead of
  *     hanging the GPU.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
@@ -185,6 +186,31 @@ qsa_status_t qsa_backward_kvwait(const void* grad_out, const void* q, const void
                                  void* dq, void* dk, void* dv, int kv_fp32,
                                  void* workspace, size_t workspace_bytes, qsa_stream_t stream,
                                  qsa_event_t kv_ready, const qsa_event_t* stage_events, int n_stage_events);
+
+/*
+ * Backward that reuses the forward's route lists instead of sorting the routes
+ * again.  Every forward call (qsa_forward, _ex, _kvwait, with a workspace of at
+ * least qsa_forward_workspace_size bytes) leaves the per-row ascending,
+ * de-duplicated route lists it computed in its workspace, after the status
+ * word; `fwd_workspace` / `fwd_workspace_bytes` name that workspace, which must
+ * still hold them: the forward ran with the same routes and sizes, and nothing
+ * has written the workspace since (the backward's own `workspace` may be the
+ * same buffer, if it is large enough for the backward).  The backward then
+ * runs only delta and the tile masks as its route work.  Results are bit for
+ * bit those of qsa_backward_kvwait on the same routes; other arguments, checks
+ * and stage events as there (routes are not an argument).  A forward workspace
+ * that does not hold the lists of the same routes gives wrong gradients: the
+ * library cannot check it without reading device memory.  The pages have no
+ * counterpart (training keeps a forward's index structures for its backward as
+ * it keeps the LSE).
+ */
+qsa_status_t qsa_backward_saved(const void* grad_out, const void* q, const void* k, const void* v,
+                                const void* out, const float* lse,
+                                const void* fwd_workspace, size_t fwd_workspace_bytes,
+                                int64_t T, int64_t T_kv, int H, int G, int n_sel, float scale,
+                                void* dq, void* dk, void* dv, int kv_fp32,
+                                void* workspace, size_t workspace_bytes, qsa_stream_t stream,
+                                qsa_event_t kv_ready, const qsa_event_t* stage_events, int n_stage_events);
 
 /*
  * Number of kernels one qsa_forward (backward = 0) or qsa_backward (backward = 1)

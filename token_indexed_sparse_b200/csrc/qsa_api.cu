@@ -144,23 +144,29 @@ static qsa_status_t backward_impl(const void* grad_out, const void* q, const voi
                            const float* lse, const int32_t* routes, int64_t T, int64_t T_kv, int H, int G, int n_sel,
                            float scale, void* dq, void* dk, void* dv, bool kv_f32, void* workspace,
                            size_t workspace_bytes, qsa_stream_t stream, const qsa_event_t* stage_events,
-                           int n_stage_events, qsa_event_t kv_ready) {
-  if (!grad_out || !q || !k || !v || !out || !lse || !routes || !dq || !dk || !dv || !workspace)
+                           int n_stage_events, qsa_event_t kv_ready, const void* fwd_workspace,
+                           size_t fwd_workspace_bytes) {
+  // with fwd_workspace the route lists come from a forward call's workspace, and routes is not read
+  const bool saved = fwd_workspace != nullptr;
+  if (!grad_out || !q || !k || !v || !out || !lse || (!routes && !saved) || !dq || !dk || !dv || !workspace)
     return QSA_ERR_INVALID_ARGUMENT;
   const qsa_status_t st = check_sizes(T, T_kv, H, G, n_sel);
   if (st != QSA_OK) return st;
   if (!(scale > 0.f) || !std::isfinite(scale)) return QSA_ERR_INVALID_ARGUMENT;
   if (!aligned(grad_out, 16) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
-      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) || !aligned(routes, 4) ||
-      !aligned(workspace, 256))
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4) ||
+      (!saved && !aligned(routes, 4)) || !aligned(workspace, 256) || (saved && !aligned(fwd_workspace, 256)))
     return QSA_ERR_MISALIGNED;
   const Layout L = make_layout(T, T_kv, H, G, n_sel, true);
   if (workspace_bytes < L.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
+  const Layout LF = make_layout(T, T_kv, H, G, n_sel, false);
+  if (saved && fwd_workspace_bytes < LF.total) return QSA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int64_t nt = (T_kv + 127) / 128;
   int* status = at<int>(workspace, L.status);
-  int32_t* row_cnt = at<int32_t>(workspace, L.row_cnt);
-  int32_t* row_cols = at<int32_t>(workspace, L.row_cols);
+  void* rows_ws = saved ? const_cast<void*>(fwd_workspace) : workspace;  // read only when saved
+  int32_t* row_cnt = at<int32_t>(rows_ws, saved ? LF.row_cnt : L.row_cnt);
+  int32_t* row_cols = at<int32_t>(rows_ws, saved ? LF.row_cols : L.row_cols);
   int32_t* tile_cnt = at<int32_t>(workspace, L.tile_ctr);
   int32_t* wl_cnt = tile_cnt + nt;
   int32_t* claim = wl_cnt + L.P;
@@ -176,8 +182,12 @@ static qsa_status_t backward_impl(const void* grad_out, const void* q, const voi
   const StageEvents ev{stage_events, n_stage_events, s};
   // one memset: the counters and the tile masks after them
   QSA_TRY(cudaMemsetAsync(tile_cnt, 0, L.lists - L.tile_ctr + qsa::tile_masks_bytes(T, T_kv), s));
-  QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 0, status, grad_out, out, delta,
-                                 H, static_cast<unsigned long long*>(lists), s));
+  if (saved)
+    QSA_TRY(qsa::launch_row_delta_masks(row_cnt, row_cols, T, T_kv, n_sel, status, grad_out, out, delta, H,
+                                        static_cast<unsigned long long*>(lists), s));
+  else
+    QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 0, status, grad_out, out,
+                                   delta, H, static_cast<unsigned long long*>(lists), s));
   QSA_TRY(ev.mark(0));
   QSA_TRY(qsa::launch_tile_lists(row_cnt, row_cols, T, n_sel, nt, lists, tile_cnt, tile_ptr, tile_fill, tile_ent, s));
   QSA_TRY(ev.mark(1));
@@ -257,7 +267,7 @@ qsa_status_t qsa_backward_ex(const void* grad_out, const void* q, const void* k,
                              size_t workspace_bytes, qsa_stream_t stream, const qsa_event_t* stage_events,
                              int n_stage_events) {
   return backward_impl(grad_out, q, k, v, out, lse, routes, T, T_kv, H, G, n_sel, scale, dq, dk, dv, false, workspace,
-                       workspace_bytes, stream, stage_events, n_stage_events, nullptr);
+                       workspace_bytes, stream, stage_events, n_stage_events, nullptr, nullptr, 0);
 }
 
 qsa_status_t qsa_backward_kvwait(const void* grad_out, const void* q, const void* k, const void* v, const void* out,
@@ -266,7 +276,18 @@ qsa_status_t qsa_backward_kvwait(const void* grad_out, const void* q, const void
                                  size_t workspace_bytes, qsa_stream_t stream, qsa_event_t kv_ready,
                                  const qsa_event_t* stage_events, int n_stage_events) {
   return backward_impl(grad_out, q, k, v, out, lse, routes, T, T_kv, H, G, n_sel, scale, dq, dk, dv, kv_fp32 != 0,
-                       workspace, workspace_bytes, stream, stage_events, n_stage_events, kv_ready);
+                       workspace, workspace_bytes, stream, stage_events, n_stage_events, kv_ready, nullptr, 0);
+}
+
+qsa_status_t qsa_backward_saved(const void* grad_out, const void* q, const void* k, const void* v, const void* out,
+                                const float* lse, const void* fwd_workspace, size_t fwd_workspace_bytes, int64_t T,
+                                int64_t T_kv, int H, int G, int n_sel, float scale, void* dq, void* dk, void* dv,
+                                int kv_fp32, void* workspace, size_t workspace_bytes, qsa_stream_t stream,
+                                qsa_event_t kv_ready, const qsa_event_t* stage_events, int n_stage_events) {
+  if (!fwd_workspace) return QSA_ERR_INVALID_ARGUMENT;
+  return backward_impl(grad_out, q, k, v, out, lse, nullptr, T, T_kv, H, G, n_sel, scale, dq, dk, dv, kv_fp32 != 0,
+                       workspace, workspace_bytes, stream, stage_events, n_stage_events, kv_ready, fwd_workspace,
+                       fwd_workspace_bytes);
 }
 
 qsa_status_t qsa_backward_fp32kv(const void* grad_out, const void* q, const void* k, const void* v, const void* out,
@@ -274,7 +295,7 @@ qsa_status_t qsa_backward_fp32kv(const void* grad_out, const void* q, const void
                                  int n_sel, float scale, void* dq, float* dk, float* dv, void* workspace,
                                  size_t workspace_bytes, qsa_stream_t stream) {
   return backward_impl(grad_out, q, k, v, out, lse, routes, T, T_kv, H, G, n_sel, scale, dq, dk, dv, true, workspace,
-                       workspace_bytes, stream, nullptr, 0, nullptr);
+                       workspace_bytes, stream, nullptr, 0, nullptr, nullptr, 0);
 }
 
 int qsa_launch_count(int64_t T, int64_t T_kv, int H, int G, int n_sel, int backward) {

@@ -20,6 +20,11 @@ cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, in
                               int32_t* row_cnt, int32_t* row_cols, int32_t* bucket_cnt, int cnt_shift,
                               int* status, const void* dout, const void* out, float* delta, int H,
                               unsigned long long* tile_masks, cudaStream_t s);
+// The backward's route work from row lists sorted already (a forward's, same
+// routes): delta and the tile masks as launch_route_rows would set them.
+cudaError_t launch_row_delta_masks(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int64_t T_kv,
+                                   int n_sel, int* status, const void* dout, const void* out, float* delta, int H,
+                                   unsigned long long* tile_masks, cudaStream_t s);
 // quad_cnt -> quad_ptr (exclusive scan, n_quads+1 entries) and quad_fill (copy
 // of quad_ptr used as fill cursors).
 cudaError_t launch_quad_scan(const int32_t* quad_cnt, int64_t n_quads, int32_t* quad_ptr,

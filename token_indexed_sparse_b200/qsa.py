@@ -57,6 +57,9 @@ def library() -> ctypes.CDLL:
     lib.qsa_backward_ex.argtypes = lib.qsa_backward.argtypes + [vp, i32]
     lib.qsa_forward_kvwait.restype = i32
     lib.qsa_forward_kvwait.argtypes = lib.qsa_forward.argtypes + [vp, vp, i32]
+    lib.qsa_backward_saved.restype = i32
+    lib.qsa_backward_saved.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, i64, i64, i32, i32, i32, f32, vp, vp, vp, i32,
+                                       vp, sz, vp, vp, vp, i32]
     lib.qsa_backward_kvwait.restype = i32
     lib.qsa_backward_kvwait.argtypes = lib.qsa_backward.argtypes[:16] + [i32] + lib.qsa_backward.argtypes[16:] + [
         vp, vp, i32]
@@ -211,7 +214,7 @@ def forward(q, k, v, routes, scale: float = 1.0 / 16.0, *, out=None, lse=None, w
 
 def backward(grad_out, q, k, v, out, lse, routes, scale: float = 1.0 / 16.0, *,
              dq=None, dk=None, dv=None, workspace=None, stage_events=None, kv_fp32: bool = False,
-             kv_ready=None):
+             kv_ready=None, saved_workspace=None):
     """qsa_backward: returns ``(dq, dk, dv)`` (bf16, shapes of q, k, v).
 
     ``stage_events`` (optional, up to 5 torch.cuda.Event) are recorded after
@@ -219,7 +222,10 @@ def backward(grad_out, q, k, v, out, lse, routes, scale: float = 1.0 / 16.0, *,
     the BF16 rounding, for adding partials from several calls).  ``kv_ready``
     (optional recorded torch.cuda.Event): k and v may still be being written
     until it fires; the route work runs first and dQ waits for it
-    (qsa_backward_kvwait)."""
+    (qsa_backward_kvwait).  ``saved_workspace``: the workspace tensor of the
+    forward call on the same routes (still holding its route lists, which
+    are then reused instead of sorting the routes again: qsa_backward_saved);
+    ``routes`` then only gives n_sel."""
     lib = library()
     grad_out = _prep(grad_out, torch.bfloat16, "grad_out")
     q = _prep(q, torch.bfloat16, "q")
@@ -238,6 +244,14 @@ def backward(grad_out, q, k, v, out, lse, routes, scale: float = 1.0 / 16.0, *,
     ws_bytes = lib.qsa_backward_workspace_size(T, T_kv, H, G, n_sel)
     ws = _workspace(ws_bytes, q.device, workspace)
     ev, n_ev = _events(stage_events)
+    if saved_workspace is not None:
+        fws = _workspace(0, q.device, saved_workspace)
+        st = lib.qsa_backward_saved(_ptr(grad_out), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(fws),
+                                    fws.numel(), T, T_kv, H, G, n_sel, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
+                                    1 if kv_fp32 else 0, _ptr(ws), ws.numel(), _stream(q.device),
+                                    _event_handle(kv_ready), ev, n_ev)
+        _check(st, "qsa_backward_saved")
+        return dq, dk, dv
     st = lib.qsa_backward_kvwait(_ptr(grad_out), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(routes),
                                  T, T_kv, H, G, n_sel, float(scale), _ptr(dq), _ptr(dk), _ptr(dv),
                                  1 if kv_fp32 else 0, _ptr(ws), ws.numel(), _stream(q.device),
