@@ -208,6 +208,24 @@ def test_route_plan_edge_rows():
     _check_plan(routes, T_kv)
 
 
+@pytest.mark.parametrize("n_sel", [2, 33, 64, 65, 300, 512, 513, 544, 545, 576, 577, 640, 641, 700, 768, 769,
+                                   1024, 1025, 2048])
+def test_route_rows_every_kernel_width(n_sel):
+    # the route-row kernels change with n_sel (register networks of 64 .. 1024
+    # slots, 512 + 32 .. 512 + 256 split sorts merged in shared memory, and the
+    # CTA sort above 1024): rows with duplicates, invalid IDs, empty rows and
+    # rows that fill every slot with distinct keys
+    rng = np.random.default_rng(n_sel)
+    T, T_kv = 96, 3000
+    routes = rng.integers(-40, T_kv + 40, size=(T, n_sel)).astype(np.int32)
+    routes[0] = -1
+    routes[1] = rng.permutation(T_kv)[:n_sel] if n_sel <= T_kv else routes[1]
+    routes[2] = 7
+    routes[3, : n_sel // 2] = routes[3, n_sel - n_sel // 2:] if n_sel > 1 else routes[3, :0]
+    routes[4] = np.sort(routes[4])[::-1]
+    _check_plan(routes, T_kv)
+
+
 def test_route_plan_long_quad_list():
     # 5000 queries share one quad: its list is longer than the in-shared-memory sort
     T, T_kv = 5000, 16

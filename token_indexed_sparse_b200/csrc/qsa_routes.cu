@@ -114,6 +114,10 @@ __device__ __forceinline__ void warp_sort(int32_t (&v)[NPL], int lane) {
       // k-block (bit k/2 of the element index clear) keeps the minimum
       const int m = k / NPL - 1;
       const bool lower = (lane & (k / (2 * NPL))) == 0;
+      if (NPL == 1) {  // register 0 pairs with register 0 of lane ^ m
+        const int32_t t = __shfl_xor_sync(0xffffffffu, v[0], m);
+        v[0] = lower ? min(v[0], t) : max(v[0], t);
+      }
 #pragma unroll
       for (int r = 0; r < NPL / 2; ++r) {
         const int r2 = NPL - 1 - r;
@@ -187,38 +191,15 @@ __device__ __forceinline__ void row_delta(const __nv_bfloat16* __restrict__ dout
   }
 }
 
-// One warp per query row (rows of up to 32*NPL route slots): filter, sort in
-// registers, de-duplicate, compact; optionally per-bucket row counts (a bucket
-// is 2^cnt_shift consecutive keys), the row's bits in the tile masks, and delta.
-// (A shared-memory bitmap of the row's key range in place of the sort, with
-// word popcounts scanned across the warp, ran the seq32k rows in 0.30 ms
-// against 0.25 ms for this sort: the bit-by-bit read-back diverges across lanes.)
+// Emits a warp's sorted values (element e = lane * NPL + r in v[r], +infinity
+// as INT_MAX at the end): de-duplicates and compacts them to dst, and
+// optionally adds per-bucket row counts (a bucket is 2^cnt_shift consecutive
+// keys) and sets the row's bits in the tile masks.  Returns the row's count.
 template <int NPL>
-__global__ void __launch_bounds__(kRowWarps * 32, 3) route_rows_warp_kernel(
-    const int32_t* __restrict__ routes, int64_t T, int32_t T_kv, int n_sel, int32_t* __restrict__ row_cnt,
-    int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt, int cnt_shift, int* __restrict__ status,
-    const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out, float* __restrict__ delta,
-    int H, unsigned long long* __restrict__ masks, int64_t n_tiles) {
-  const int lane = threadIdx.x & 31;
-  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
-  if (t >= T) return;
-  const int32_t* row = routes + t * n_sel;
-  int32_t* dst = row_cols + t * n_sel;
-  int32_t v[NPL];
-#pragma unroll
-  for (int r = 0; r < NPL; ++r) {  // coalesced: the sort does not care where a value starts
-    const int i = r * 32 + lane;
-    int32_t x = INT_MAX;
-    if (i < n_sel) {
-      const int32_t y = __ldg(row + i);
-      if (y >= 0 && y < T_kv) x = y;
-    }
-    v[r] = x;
-  }
-  warp_sort<NPL>(v, lane);
-  // element e = lane * NPL + r; the previous element of v[0] is the previous
-  // lane's v[NPL - 1]
+__device__ __forceinline__ int emit_sorted(const int32_t (&v)[NPL], int lane, int64_t t, int32_t* __restrict__ dst,
+                                           int32_t* __restrict__ quad_cnt, int cnt_shift,
+                                           unsigned long long* __restrict__ masks, int64_t n_tiles) {
+  // the previous element of v[0] is the previous lane's v[NPL - 1]
   int32_t prev = __shfl_up_sync(0xffffffffu, v[NPL - 1], 1);
   if (lane == 0) prev = INT_MIN;
   int mine = 0;
@@ -247,7 +228,109 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3) route_rows_warp_kernel(
     const int32_t x = v[r];
     if (x != INT_MAX && x != p) dst[pos++] = x;
   }
-  const int cnt = __shfl_sync(0xffffffffu, incl, 31);
+  return __shfl_sync(0xffffffffu, incl, 31);
+}
+
+// Loads slots [first, first + 32 * NPL) of a route row into registers
+// (coalesced: slot first + r * 32 + lane in v[r]; the sort does not care where
+// a value starts), invalid IDs and slots past n_sel as INT_MAX.
+template <int NPL>
+__device__ __forceinline__ void load_slots(int32_t (&v)[NPL], const int32_t* __restrict__ row, int first, int n_sel,
+                                           int32_t T_kv, int lane) {
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) {
+    const int i = first + r * 32 + lane;
+    int32_t x = INT_MAX;
+    if (i < n_sel) {
+      const int32_t y = __ldg(row + i);
+      if (y >= 0 && y < T_kv) x = y;
+    }
+    v[r] = x;
+  }
+}
+
+// One warp per query row (rows of up to 32*NPL route slots): filter, sort in
+// registers, de-duplicate, compact; optionally per-bucket row counts, the
+// row's bits in the tile masks, and delta.
+// (A shared-memory bitmap of the row's key range in place of the sort, with
+// word popcounts scanned across the warp, ran the seq32k rows in 0.30 ms
+// against 0.25 ms for this sort: the bit-by-bit read-back diverges across lanes.)
+template <int NPL>
+__global__ void __launch_bounds__(kRowWarps * 32, 3) route_rows_warp_kernel(
+    const int32_t* __restrict__ routes, int64_t T, int32_t T_kv, int n_sel, int32_t* __restrict__ row_cnt,
+    int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt, int cnt_shift, int* __restrict__ status,
+    const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out, float* __restrict__ delta,
+    int H, unsigned long long* __restrict__ masks, int64_t n_tiles) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+  if (t >= T) return;
+  int32_t v[NPL];
+  load_slots<NPL>(v, routes + t * n_sel, 0, n_sel, T_kv, lane);
+  warp_sort<NPL>(v, lane);
+  const int cnt = emit_sorted<NPL>(v, lane, t, row_cols + t * n_sel, quad_cnt, cnt_shift, masks, n_tiles);
+  if (lane == 0) row_cnt[t] = cnt;
+  if (delta != nullptr) row_delta(dout, out, delta, t, H, lane, 0, 4);
+}
+
+// Rows of 513 .. 512 + 32 * NB slots (NB <= 8): the first 512 slots and the
+// rest are sorted apart in registers (bitonic networks of 512 and 32 NB
+// elements, about 40-95 % fewer compare-exchanges than one network of 1024),
+// stored to shared memory and merged: lane l produces the merged elements
+// l * (16 + NB) ... of the stable merge (ties from the first part first), its
+// split of the two parts found by a binary search on its diagonal.
+constexpr int kSplitA = 512;
+template <int NB>
+__global__ void __launch_bounds__(kRowWarps * 32, 3) route_rows_split_kernel(
+    const int32_t* __restrict__ routes, int64_t T, int32_t T_kv, int n_sel, int32_t* __restrict__ row_cnt,
+    int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt, int cnt_shift, int* __restrict__ status,
+    const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out, float* __restrict__ delta,
+    int H, unsigned long long* __restrict__ masks, int64_t n_tiles) {
+  constexpr int NA = kSplitA / 32, kLenB = 32 * NB, kPer = NA + NB;
+  __shared__ int32_t parts[kRowWarps][kSplitA + kLenB];
+  const int lane = threadIdx.x & 31;
+  int32_t* sa = parts[threadIdx.x >> 5];
+  int32_t* sb = sa + kSplitA;
+  const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+  if (t >= T) return;
+  const int32_t* row = routes + t * n_sel;
+  {
+    int32_t a[NA];
+    load_slots<NA>(a, row, 0, n_sel, T_kv, lane);
+    warp_sort<NA>(a, lane);
+#pragma unroll
+    for (int r = 0; r < NA; ++r) sa[lane * NA + r] = a[r];
+  }
+  {
+    int32_t b[NB];
+    load_slots<NB>(b, row, kSplitA, n_sel, T_kv, lane);
+    warp_sort<NB>(b, lane);
+#pragma unroll
+    for (int r = 0; r < NB; ++r) sb[lane * NB + r] = b[r];
+  }
+  __syncwarp();
+  // merge path: the first d merged elements take i from the first part and
+  // d - i from the second, i the least value with sa[i] > sb[d - i - 1]
+  const int d = lane * kPer;
+  int lo = d > kLenB ? d - kLenB : 0, hi = d < kSplitA ? d : kSplitA;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (sa[mid] <= sb[d - mid - 1]) lo = mid + 1;
+    else hi = mid;
+  }
+  int ia = lo, ib = d - lo;
+  int32_t v[kPer];
+#pragma unroll
+  for (int r = 0; r < kPer; ++r) {
+    const int32_t x = ia < kSplitA ? sa[ia] : INT_MAX;
+    const int32_t y = ib < kLenB ? sb[ib] : INT_MAX;
+    const bool take_a = ib >= kLenB || (ia < kSplitA && x <= y);
+    v[r] = take_a ? x : y;
+    ia += take_a ? 1 : 0;
+    ib += take_a ? 0 : 1;
+  }
+  const int cnt = emit_sorted<kPer>(v, lane, t, row_cols + t * n_sel, quad_cnt, cnt_shift, masks, n_tiles);
   if (lane == 0) row_cnt[t] = cnt;
   if (delta != nullptr) row_delta(dout, out, delta, t, H, lane, 0, 4);
 }
@@ -646,6 +729,22 @@ cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, in
   if (n_sel <= 128) { QSA_ROWS_WARP(4); }
   if (n_sel <= 256) { QSA_ROWS_WARP(8); }
   if (n_sel <= 512) { QSA_ROWS_WARP(16); }
+#undef QSA_ROWS_WARP
+#define QSA_ROWS_SPLIT(NB)                                                                                        \
+  route_rows_split_kernel<NB><<<wblocks, kRowWarps * 32, 0, s>>>(routes, T, tkv, n_sel, row_cnt, row_cols,         \
+                                                                 bucket_cnt, cnt_shift, status, dq, o, delta, H, \
+                                                                 tile_masks, n_tiles);                            \
+  return cudaGetLastError()
+  if (n_sel <= kSplitA + 32) { QSA_ROWS_SPLIT(1); }
+  if (n_sel <= kSplitA + 64) { QSA_ROWS_SPLIT(2); }
+  if (n_sel <= kSplitA + 128) { QSA_ROWS_SPLIT(4); }
+  if (n_sel <= kSplitA + 256) { QSA_ROWS_SPLIT(8); }
+#undef QSA_ROWS_SPLIT
+#define QSA_ROWS_WARP(NPL)                                                                                         \
+  route_rows_warp_kernel<NPL><<<wblocks, kRowWarps * 32, 0, s>>>(routes, T, tkv, n_sel, row_cnt, row_cols,        \
+                                                                 bucket_cnt, cnt_shift, status, dq, o, delta, H, \
+                                                                 tile_masks, n_tiles);                            \
+  return cudaGetLastError()
   if (n_sel <= 1024) { QSA_ROWS_WARP(32); }
 #undef QSA_ROWS_WARP
   const int n2 = next_pow2(n_sel);
