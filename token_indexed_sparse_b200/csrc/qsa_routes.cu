@@ -361,27 +361,68 @@ __global__ void __launch_bounds__(256) row_delta_masks_kernel(
   row_delta(dout, out, delta, t, H, lane, 0, 4);
 }
 
-// One block per query row: filter invalid IDs, sort, de-duplicate, compact.
+// Sorts a row of n2 slots (n2 a power of two >= 2048, slots past n_sel and
+// invalid IDs as INT_MAX) with the CTA's 8 warps: every 256-slot chunk is
+// sorted in registers by one warp (warp_sort), then rounds of pairwise merges
+// double the sorted runs until one remains, each thread producing n2 / 256
+// consecutive outputs of its pair of runs after a binary search on its
+// diagonal (merge path).  b0 and b1 are n2 ints each of shared memory; returns
+// the one holding the sorted row.  All threads of the CTA must call it.
+__device__ int32_t* block_merge_sort(int32_t* b0, int32_t* b1, const int32_t* __restrict__ row, int n_sel,
+                                     int32_t T_kv, int n2) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int c = warp; c < n2 / 256; c += nw) {
+    int32_t v[8];
+    load_slots<8>(v, row, c * 256, n_sel, T_kv, lane);
+    warp_sort<8>(v, lane);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) b0[c * 256 + lane * 8 + r] = v[r];
+  }
+  __syncthreads();
+  const int per = n2 / static_cast<int>(blockDim.x);
+  int32_t* src = b0;
+  int32_t* dst = b1;
+  for (int len = 256; len < n2; len <<= 1) {
+    const int o0 = static_cast<int>(threadIdx.x) * per;
+    const int base = o0 & ~(2 * len - 1);  // the pair of runs [base, base + len), [base + len, base + 2 len)
+    const int32_t* a = src + base;
+    const int32_t* b = a + len;
+    const int d = o0 - base;
+    int lo = d > len ? d - len : 0, hi = d < len ? d : len;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (a[mid] <= b[d - mid - 1]) lo = mid + 1;
+      else hi = mid;
+    }
+    int ia = lo, ib = d - lo;
+    for (int r = 0; r < per; ++r) {
+      const int32_t x = ia < len ? a[ia] : INT_MAX;
+      const int32_t y = ib < len ? b[ib] : INT_MAX;
+      const bool take_a = ib >= len || (ia < len && x <= y);
+      dst[o0 + r] = take_a ? x : y;
+      ia += take_a ? 1 : 0;
+      ib += take_a ? 0 : 1;
+    }
+    __syncthreads();
+    int32_t* tmp = src;
+    src = dst;
+    dst = tmp;
+  }
+  return src;
+}
+
+// One block per query row (rows of more than 1024 slots): filter invalid IDs,
+// sort (block_merge_sort), de-duplicate, compact.
 __global__ void __launch_bounds__(kRowThreads) route_rows_kernel(
     const int32_t* __restrict__ routes, int32_t T_kv, int n_sel, int n2,
     int32_t* __restrict__ row_cnt, int32_t* __restrict__ row_cols, int32_t* __restrict__ quad_cnt, int cnt_shift,
     int* __restrict__ status, const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out,
     float* __restrict__ delta, int H, unsigned long long* __restrict__ masks, int64_t n_tiles) {
-  extern __shared__ int32_t sv[];  // n2 values, then 32 ints of scan scratch
-  int* scratch = sv + n2;
+  extern __shared__ int32_t smem_rows[];  // two buffers of n2 values, then 32 ints of scan scratch
+  int* scratch = smem_rows + 2 * n2;
   const int64_t t = blockIdx.x;
   if (status != nullptr && t == 0 && threadIdx.x == 0) *status = 0;
-  const int32_t* row = routes + t * n_sel;
-  for (int i = threadIdx.x; i < n2; i += blockDim.x) {
-    int32_t x = INT_MAX;
-    if (i < n_sel) {
-      const int32_t r = row[i];
-      if (r >= 0 && r < T_kv) x = r;
-    }
-    sv[i] = x;
-  }
-  __syncthreads();
-  block_sort<int32_t>(sv, n2, n2);
+  const int32_t* sv = block_merge_sort(smem_rows, smem_rows + n2, routes + t * n_sel, n_sel, T_kv, n2);
 
   // Each thread owns a contiguous run of the sorted values.
   const int per = (n2 + blockDim.x - 1) / blockDim.x;
@@ -748,7 +789,7 @@ cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, in
   if (n_sel <= 1024) { QSA_ROWS_WARP(32); }
 #undef QSA_ROWS_WARP
   const int n2 = next_pow2(n_sel);
-  const size_t smem = static_cast<size_t>(n2 + 32) * sizeof(int32_t);
+  const size_t smem = static_cast<size_t>(2 * n2 + 32) * sizeof(int32_t);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(route_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
