@@ -551,9 +551,11 @@ def run_cp(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    ws_f = torch.empty(qsa.forward_workspace_size(e - s, wl.T_kv, wl.H, wl.G, wl.W), dtype=torch.uint8, device=dev)
+
     def step(q_, k_, v_, do_, r_):
-        out, lse = cp.cp_forward(q_, k_, v_, r_, wl.scale)
-        return (out, lse, *cp.cp_backward(do_, q_, k_, v_, out, lse, r_, wl.scale))
+        out, lse = cp.cp_forward(q_, k_, v_, r_, wl.scale, workspace=ws_f)
+        return (out, lse, *cp.cp_backward(do_, q_, k_, v_, out, lse, r_, wl.scale, saved_workspace=ws_f))
 
     for _ in range(args.warmup):
         step(q, k, v, do, routes)
