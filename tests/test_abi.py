@@ -106,6 +106,37 @@ def test_host_validation_before_any_launch(lib):
     assert lib.qsa_tile_plan_scratch_size(16, 300) == 2 * 256 + 256
 
 
+def test_saved_and_kvwait_host_validation(lib):
+    # the backward that reuses a forward's route lists checks the forward
+    # workspace (present, 256-byte aligned, large enough) before any launch;
+    # routes are not an argument there.  These return before touching CUDA.
+    P = ctypes.c_void_p
+    big = 1 << 30
+
+    def saved(fws=4096, fws_bytes=big, ws=8192, ws_bytes=big, dv=256):
+        return lib.qsa_backward_saved(P(256), P(256), P(256), P(256), P(256), P(256), P(fws), fws_bytes, 16, 16,
+                                      12, 1, 4, 0.0625, P(256), P(256), P(dv), 0, P(ws), ws_bytes, None, None,
+                                      None, 0)
+    assert saved(fws=0) == 1
+    assert saved(dv=0) == 1
+    assert saved(fws=4096 + 16) == 3
+    assert saved(fws_bytes=8) == 4
+    assert saved(ws_bytes=8) == 4
+    fwd_need = lib.qsa_forward_workspace_size(16, 16, 12, 1, 4)
+    assert saved(fws_bytes=fwd_need - 1) == 4
+
+    def kvwait_fwd(q=256, ws_bytes=big):
+        return lib.qsa_forward_kvwait(P(q), P(256), P(256), P(256), 16, 16, 12, 1, 4, 0.0625, P(256), P(256),
+                                      P(4096), ws_bytes, None, None, None, 0)
+    assert kvwait_fwd(q=0) == 1 and kvwait_fwd(q=264) == 3 and kvwait_fwd(ws_bytes=8) == 4
+
+    def kvwait_bwd(routes=256, kv_fp32=0, ws_bytes=big):
+        return lib.qsa_backward_kvwait(P(256), P(256), P(256), P(256), P(256), P(256), P(routes), 16, 16, 12, 1,
+                                       4, 0.0625, P(256), P(256), P(256), kv_fp32, P(4096), ws_bytes, None, None,
+                                       None, 0)
+    assert kvwait_bwd(routes=0) == 1 and kvwait_bwd(routes=258) == 3 and kvwait_bwd(kv_fp32=1, ws_bytes=8) == 4
+
+
 def _fwd_noalloc(lib, q=256, T=16, n_sel=4):
     P = ctypes.c_void_p
     f = lib.qsa_forward_noalloc
