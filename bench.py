@@ -50,11 +50,11 @@ SPEC_BF16_TFLOPS = 2250.0              # B200 dense BF16 tensor peak (NVIDIA spe
 TRAFFIC = {
     # the timed step's dK/dV launch on seq32k: ncu dram__bytes_read.sum + dram__bytes_write.sum
     # (the dK/dV summary under profiles/); the kernel and the phase sizing of its launch
-    "bwd_dkdv": (15083029760, {
+    "bwd_dkdv": (15447996672, {
         "token_indexed_sparse_b200/csrc/qsa_dkdv_union.cu":
             "1ebd1ab736b167e165bf20277e70b378f50e0b542b063957dcbdd386bf5619ae",
         "token_indexed_sparse_b200/csrc/qsa_api.cu":
-            "5d19978cca318f395bf266024013af302738c42098e39431964f7bf1ba901abf",
+            "c7e2ca56d7da2243780efbeaf0ba3b7f06f4b3ce3b7e152b150908afcdec826e",
     }),
 }
 
