@@ -40,7 +40,8 @@
  *     except the first int32 of the workspace, a status word: once the call's
  *     work has completed on the stream it is 0, or nonzero if a kernel gave up
  *     on a bounded wait (its outputs are then invalid), and, after a forward
- *     call, the route lists that qsa_backward_saved can reuse.  Every wait inside the
+ *     call, the route lists that qsa_backward_saved can reuse, with their tag
+ *     in int32 words 4..7.  Every wait inside the
  *     kernels is bounded, so a fault in the pipeline ends the kernel instead of
  *     hanging the GPU.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
@@ -198,11 +199,14 @@ qsa_status_t qsa_backward_kvwait(const void* grad_out, const void* q, const void
  * same buffer, if it is large enough for the backward).  The backward then
  * runs only delta and the tile masks as its route work.  Results are bit for
  * bit those of qsa_backward_kvwait on the same routes; other arguments, checks
- * and stage events as there (routes are not an argument).  A forward workspace
- * that does not hold the lists of the same routes gives wrong gradients: the
- * library cannot check it without reading device memory.  The pages have no
- * counterpart (training keeps a forward's index structures for its backward as
- * it keeps the LSE).
+ * and stage events as there (routes are not an argument).  The forward also
+ * leaves a tag of the sizes it sorted for (int32 words 4..7 of its workspace);
+ * when fwd_workspace lacks the tag of rows of these sizes (no forward wrote it,
+ * or one of other sizes), the status word of `workspace` reads 2 after the
+ * call, no kernel reads the lists, and dq, dk and dv are invalid.  Lists of
+ * other routes with the same sizes cannot be told apart on the device: they
+ * give wrong gradients.  The pages have no counterpart (training keeps a
+ * forward's index structures for its backward as it keeps the LSE).
  */
 qsa_status_t qsa_backward_saved(const void* grad_out, const void* q, const void* k, const void* v,
                                 const void* out, const float* lse,

@@ -51,3 +51,25 @@ def test_saved_rows_in_the_backward_workspace_itself():
     for a, b in zip(got, ref):
         assert torch.equal(a, b)
     assert int(ws[:4].view(torch.int32).item()) == 0  # status word: no wait gave up
+
+
+def test_saved_rows_without_a_forward_report_a_bad_status():
+    # a forward workspace that no forward wrote (zero-filled here, so that even
+    # an unguarded read would see empty rows) lacks the route-list tag: the
+    # status word reports it and no kernel reads the lists
+    wl, routes, q, k, v, do = _inputs("thd16k", 1024)
+    H, G, n_sel = wl.H, wl.G, routes.shape[1]
+    out, lse = qsa.forward(q, k, v, routes, wl.scale)
+    fws = torch.zeros(qsa.forward_workspace_size(wl.T, wl.T_kv, H, G, n_sel), dtype=torch.uint8, device=DEV)
+    ws = torch.empty(qsa.backward_workspace_size(wl.T, wl.T_kv, H, G, n_sel), dtype=torch.uint8, device=DEV)
+    qsa.backward(do, q, k, v, out, lse, routes, wl.scale, workspace=ws, saved_workspace=fws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 2
+    # a forward on the same buffer writes the tag: the same call then succeeds
+    qsa.forward(q, k, v, routes, wl.scale, workspace=fws)
+    ref = qsa.backward(do, q, k, v, out, lse, routes, wl.scale)
+    got = qsa.backward(do, q, k, v, out, lse, routes, wl.scale, workspace=ws, saved_workspace=fws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)

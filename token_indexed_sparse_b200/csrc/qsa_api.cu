@@ -183,20 +183,21 @@ static qsa_status_t backward_impl(const void* grad_out, const void* q, const voi
   // one memset: the counters and the tile masks after them
   QSA_TRY(cudaMemsetAsync(tile_cnt, 0, L.lists - L.tile_ctr + qsa::tile_masks_bytes(T, T_kv), s));
   if (saved)
-    QSA_TRY(qsa::launch_row_delta_masks(row_cnt, row_cols, T, T_kv, n_sel, status, grad_out, out, delta, H,
-                                        static_cast<unsigned long long*>(lists), s));
+    QSA_TRY(qsa::launch_row_delta_masks(row_cnt, row_cols, T, T_kv, n_sel, at<int>(rows_ws, LF.status), status,
+                                        grad_out, out, delta, H, static_cast<unsigned long long*>(lists), s));
   else
     QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 0, status, grad_out, out,
                                    delta, H, static_cast<unsigned long long*>(lists), s));
   QSA_TRY(ev.mark(0));
-  QSA_TRY(qsa::launch_tile_lists(row_cnt, row_cols, T, n_sel, nt, lists, tile_cnt, tile_ptr, tile_fill, tile_ent, s));
+  QSA_TRY(qsa::launch_tile_lists(row_cnt, row_cols, T, n_sel, nt, lists, tile_cnt, tile_ptr, tile_fill, tile_ent,
+                                 status, s));
   QSA_TRY(ev.mark(1));
   QSA_TRY(qsa::launch_tile_worklist(tile_ptr, lists, T, nt, T_kv, G, L.P, L.C, wl_cnt, wl, dk, dv, kv_f32, s));
   QSA_TRY(ev.mark(2));
   // k and v are read from here on; the route work above ran without them
   if (kv_ready != nullptr) QSA_TRY(cudaStreamWaitEvent(s, reinterpret_cast<cudaEvent_t>(kv_ready), 0));
   QSA_TRY(qsa::launch_backward_dq(grad_out, q, k, v, lse, delta, row_cnt, row_cols, T, G, n_sel, scale, dq, pds,
-                                  s));
+                                  status, s));
   QSA_TRY(ev.mark(3));
   QSA_TRY(qsa::launch_backward_dkdv_union(grad_out, q, pds, row_cols, tile_ent, wl_cnt, wl, claim, done,
                                           L.P, nt, T_kv, G, n_sel, scale, partial, dk, dv, kv_f32, status, s));
@@ -419,7 +420,8 @@ qsa_status_t qsa_tile_plan(const int32_t* routes, int64_t T, int64_t T_kv, int n
   QSA_TRY(cudaMemsetAsync(lists, 0, qsa::tile_masks_bytes(T, T_kv), s));
   QSA_TRY(qsa::launch_route_rows(routes, T, T_kv, n_sel, row_cnt, row_cols, nullptr, 0, nullptr, nullptr, nullptr,
                                  nullptr, qsa::kHeadsPerGroup, static_cast<unsigned long long*>(lists), s));
-  QSA_TRY(qsa::launch_tile_lists(row_cnt, row_cols, T, n_sel, nt, lists, tile_cnt, tile_ptr, tile_fill, tile_ent, s));
+  QSA_TRY(qsa::launch_tile_lists(row_cnt, row_cols, T, n_sel, nt, lists, tile_cnt, tile_ptr, tile_fill, tile_ent,
+                                 nullptr, s));
   return QSA_OK;
 }
 

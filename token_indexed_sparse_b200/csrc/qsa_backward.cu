@@ -70,7 +70,7 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
           const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
           const float* __restrict__ lse, const float* __restrict__ delta, const int32_t* __restrict__ row_cnt,
           const int32_t* __restrict__ row_cols, int64_t n_items, int G, int n_sel, float scale, float scale_log2,
-          __nv_bfloat16* __restrict__ dq, uint16_t* __restrict__ pds) {
+          __nv_bfloat16* __restrict__ dq, uint16_t* __restrict__ pds, const int* __restrict__ status) {
   using S_ = DqShape<NW, STAGES, CPS>;
   constexpr int KEYS = S_::kKeys, kTile = S_::kTile, kStageBytes = S_::kStageBytes, kDsStride = S_::kDsStride;
   constexpr int kNt = S_::kNt, kKs = S_::kKs, kItemBytes = S_::kItemBytes, kThreads = S_::kThreads;
@@ -83,6 +83,9 @@ dq_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restric
   __nv_bfloat16* sDS = reinterpret_cast<__nv_bfloat16*>(smem + S_::kOffDS);
   uint16_t* sRec = reinterpret_cast<uint16_t*>(smem + S_::kOffRec);
   const uint32_t sDSa = smem_u32(sDS);
+  // route lists that failed their tag check are not read (the status word
+  // already reports it; dq is left unwritten)
+  if (status != nullptr && *status == kStatusBadPlan) return;
   if (tid < 32) reinterpret_cast<uint4*>(smem + S_::kOffZero)[tid] = make_uint4(0, 0, 0, 0);
 
   Cursor cur;
@@ -264,7 +267,7 @@ constexpr int kDqWarps = 4, kDqStages = 2, kDqCtasPerSm = 2;
 cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* k, const void* v,
                                const float* lse, const float* delta, const int32_t* row_cnt,
                                const int32_t* row_cols, int64_t T, int G, int n_sel, float scale, void* dq,
-                               uint16_t* pds, cudaStream_t s) {
+                               uint16_t* pds, const int* status, cudaStream_t s) {
   using S_ = DqShape<kDqWarps, kDqStages, kDqCtasPerSm>;
   auto kern = dq_kernel<kDqWarps, kDqStages, kDqCtasPerSm>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S_::kSmemBytes);
@@ -275,7 +278,7 @@ cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* 
   kern<<<static_cast<unsigned>(grid), S_::kThreads, S_::kSmemBytes, s>>>(
       static_cast<const __nv_bfloat16*>(grad_out), static_cast<const __nv_bfloat16*>(q),
       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), lse, delta, row_cnt, row_cols,
-      n_items, G, n_sel, scale, scale * kLog2e, static_cast<__nv_bfloat16*>(dq), pds);
+      n_items, G, n_sel, scale, scale * kLog2e, static_cast<__nv_bfloat16*>(dq), pds, status);
   return cudaGetLastError();
 }
 

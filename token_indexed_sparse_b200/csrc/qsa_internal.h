@@ -22,9 +22,12 @@ cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, in
                               unsigned long long* tile_masks, cudaStream_t s);
 // The backward's route work from row lists sorted already (a forward's, same
 // routes): delta and the tile masks as launch_route_rows would set them.
+// plan_tag: the status slot of the call that wrote the lists; `status` is set
+// to kStatusBadPlan unless it carries the route-list tag of rows of these sizes.
+constexpr int kStatusBadPlan = 2;
 cudaError_t launch_row_delta_masks(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int64_t T_kv,
-                                   int n_sel, int* status, const void* dout, const void* out, float* delta, int H,
-                                   unsigned long long* tile_masks, cudaStream_t s);
+                                   int n_sel, const int* plan_tag, int* status, const void* dout, const void* out,
+                                   float* delta, int H, unsigned long long* tile_masks, cudaStream_t s);
 // quad_cnt -> quad_ptr (exclusive scan, n_quads+1 entries) and quad_fill (copy
 // of quad_ptr used as fill cursors).
 cudaError_t launch_quad_scan(const int32_t* quad_cnt, int64_t n_quads, int32_t* quad_ptr,
@@ -48,7 +51,7 @@ size_t tile_masks_bytes(int64_t T, int64_t T_kv);
 size_t tile_lists_bytes(int64_t T, int64_t T_kv);
 cudaError_t launch_tile_lists(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel,
                               int64_t n_tiles, void* scratch, int32_t* tile_cnt, int32_t* tile_ptr,
-                              int32_t* tile_fill, int64_t* tile_ent, cudaStream_t s);
+                              int32_t* tile_fill, int64_t* tile_ent, const int* status, cudaStream_t s);
 // Per-phase work lists of non-empty (tile, entry range) items (wl_cnt zeroed by
 // the caller), phase p = rows [p C, (p + 1) C) with C a multiple of 64, its
 // start in a tile's list read from the block bases in `scratch` (written by
@@ -77,7 +80,7 @@ cudaError_t launch_forward(const void* q, const void* k, const void* v, const in
 cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* k, const void* v,
                                const float* lse, const float* delta, const int32_t* row_cnt,
                                const int32_t* row_cols, int64_t T, int G, int n_sel, float scale,
-                               void* dq, uint16_t* pds, cudaStream_t s);
+                               void* dq, uint16_t* pds, const int* status, cudaStream_t s);
 // SM count of the current device (cached).
 int sm_count();
 // dK/dV over 128-key tiles on the tensor cores, all P query phases in one

@@ -159,6 +159,19 @@ constexpr int kTileShift = 7;
 constexpr int kBlockRows = 64;
 constexpr int kRowWarps = 8;  // rows (warps) per CTA of route_rows_warp_kernel
 
+// Route-list tag: a route kernel that zeroes a call's status word also writes,
+// in words 4..7 of the same 256-byte slot, {kPlanMagic, T, T_kv, n_sel}, so a
+// later call that reuses the route lists (qsa_backward_saved) can check, on the
+// device, that they come from a route kernel run on rows of these sizes.
+constexpr int32_t kPlanMagic = 0x51534131;
+__device__ __forceinline__ void write_plan_tag(int* status, int64_t T, int32_t T_kv, int n_sel) {
+  status[0] = 0;
+  status[4] = kPlanMagic;
+  status[5] = static_cast<int32_t>(T);
+  status[6] = T_kv;
+  status[7] = n_sel;
+}
+
 // Sets row t's bit in the mask of (its 64-row block, 128-key tile tl); the
 // masks [ceil(T / 64), n_tiles] are zeroed by the caller.
 __device__ __forceinline__ void mark_tile(unsigned long long* masks, int64_t n_tiles, int64_t t, int32_t tl) {
@@ -263,7 +276,7 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3) route_rows_warp_kernel(
     int H, unsigned long long* __restrict__ masks, int64_t n_tiles) {
   const int lane = threadIdx.x & 31;
   const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+  if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) write_plan_tag(status, T, T_kv, n_sel);
   if (t >= T) return;
   int32_t v[NPL];
   load_slots<NPL>(v, routes + t * n_sel, 0, n_sel, T_kv, lane);
@@ -292,7 +305,7 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3) route_rows_split_kernel(
   int32_t* sa = parts[threadIdx.x >> 5];
   int32_t* sb = sa + kSplitA;
   const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+  if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) write_plan_tag(status, T, T_kv, n_sel);
   if (t >= T) return;
   const int32_t* row = routes + t * n_sel;
   {
@@ -340,13 +353,18 @@ __global__ void __launch_bounds__(kRowWarps * 32, 3) route_rows_split_kernel(
 // starting wherever a key's tile differs from the previous key's.  One warp
 // per row.
 __global__ void __launch_bounds__(256) row_delta_masks_kernel(
-    const int32_t* __restrict__ row_cnt, const int32_t* __restrict__ row_cols, int64_t T, int n_sel,
-    int* __restrict__ status, const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* __restrict__ out,
-    float* __restrict__ delta, int H, unsigned long long* __restrict__ masks, int64_t n_tiles) {
+    const int32_t* __restrict__ row_cnt, const int32_t* __restrict__ row_cols, int64_t T, int32_t T_kv, int n_sel,
+    const int* __restrict__ plan_tag, int* __restrict__ status, const __nv_bfloat16* __restrict__ dout,
+    const __nv_bfloat16* __restrict__ out, float* __restrict__ delta, int H, unsigned long long* __restrict__ masks,
+    int64_t n_tiles) {
   const int lane = threadIdx.x & 31;
   const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
-  if (t >= T) return;
+  // the lists must carry the tag of rows of these sizes; without it nothing
+  // reads them (here, in the tile fill or in dQ: those see the status word)
+  const bool ok = plan_tag[4] == kPlanMagic && plan_tag[5] == static_cast<int32_t>(T) && plan_tag[6] == T_kv &&
+                  plan_tag[7] == n_sel;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *status = ok ? 0 : kStatusBadPlan;
+  if (t >= T || !ok) return;
   const int cnt = row_cnt[t];
   const int32_t* cols = row_cols + t * n_sel;
   int32_t carry = -1;  // tile of the last key of the previous 32 (none: -1)
@@ -421,7 +439,7 @@ __global__ void __launch_bounds__(kRowThreads) route_rows_kernel(
   extern __shared__ int32_t smem_rows[];  // two buffers of n2 values, then 32 ints of scan scratch
   int* scratch = smem_rows + 2 * n2;
   const int64_t t = blockIdx.x;
-  if (status != nullptr && t == 0 && threadIdx.x == 0) *status = 0;
+  if (status != nullptr && t == 0 && threadIdx.x == 0) write_plan_tag(status, gridDim.x, T_kv, n_sel);
   const int32_t* sv = block_merge_sort(smem_rows, smem_rows + n2, routes + t * n_sel, n_sel, T_kv, n2);
 
   // Each thread owns a contiguous run of the sorted values.
@@ -600,10 +618,11 @@ __global__ void __launch_bounds__(256) tile_fill_kernel(const int32_t* __restric
                                                         const int32_t* __restrict__ row_cols, int64_t T, int n_sel,
                                                         int64_t n_tiles, const unsigned long long* __restrict__ masks,
                                                         const int32_t* __restrict__ blk_base,
-                                                        const int32_t* __restrict__ ptr, int64_t* __restrict__ ent) {
+                                                        const int32_t* __restrict__ ptr, int64_t* __restrict__ ent,
+                                                        const int* __restrict__ status) {
   const int lane = threadIdx.x & 31;
   const int64_t t = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (t >= T) return;
+  if (t >= T || (status != nullptr && *status == kStatusBadPlan)) return;
   const int cnt = row_cnt[t];
   const int32_t* cols = row_cols + t * n_sel;
   int32_t carry = -1;             // tile of the last key of the previous window (none: -1)
@@ -801,11 +820,12 @@ cudaError_t launch_route_rows(const int32_t* routes, int64_t T, int64_t T_kv, in
 }
 
 cudaError_t launch_row_delta_masks(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int64_t T_kv,
-                                   int n_sel, int* status, const void* dout, const void* out, float* delta, int H,
-                                   unsigned long long* tile_masks, cudaStream_t s) {
+                                   int n_sel, const int* plan_tag, int* status, const void* dout, const void* out,
+                                   float* delta, int H, unsigned long long* tile_masks, cudaStream_t s) {
   row_delta_masks_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, s>>>(
-      row_cnt, row_cols, T, n_sel, status, static_cast<const __nv_bfloat16*>(dout),
-      static_cast<const __nv_bfloat16*>(out), delta, H, tile_masks, (T_kv + 127) >> kTileShift);
+      row_cnt, row_cols, T, static_cast<int32_t>(T_kv), n_sel, plan_tag, status,
+      static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(out), delta, H, tile_masks,
+      (T_kv + 127) >> kTileShift);
   return cudaGetLastError();
 }
 
@@ -859,7 +879,7 @@ size_t tile_lists_bytes(int64_t T, int64_t T_kv) {
 
 cudaError_t launch_tile_lists(const int32_t* row_cnt, const int32_t* row_cols, int64_t T, int n_sel,
                               int64_t n_tiles, void* scratch, int32_t* tile_cnt, int32_t* tile_ptr,
-                              int32_t* tile_fill, int64_t* tile_ent, cudaStream_t s) {
+                              int32_t* tile_fill, int64_t* tile_ent, const int* status, cudaStream_t s) {
   const int64_t nb = (T + kBlockRows - 1) / kBlockRows;
   const auto* masks = static_cast<const unsigned long long*>(scratch);
   auto* blk_base = reinterpret_cast<int32_t*>(static_cast<unsigned long long*>(scratch) + nb * n_tiles);
@@ -868,7 +888,7 @@ cudaError_t launch_tile_lists(const int32_t* row_cnt, const int32_t* row_cols, i
   cudaError_t e = launch_quad_scan(tile_cnt, n_tiles, tile_ptr, tile_fill, s);
   if (e != cudaSuccess) return e;
   tile_fill_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, s>>>(row_cnt, row_cols, T, n_sel, n_tiles, masks,
-                                                                     blk_base, tile_ptr, tile_ent);
+                                                                     blk_base, tile_ptr, tile_ent, status);
   return cudaGetLastError();
 }
 
