@@ -49,12 +49,10 @@ SPEC_BF16_TFLOPS = 2250.0              # B200 dense BF16 tensor peak (NVIDIA spe
 # stage -> (bytes per step, {source file: sha256 of that file at capture time}).
 TRAFFIC = {
     # the timed step's dK/dV launch on seq32k: ncu dram__bytes_read.sum + dram__bytes_write.sum
-    # (the dK/dV summary under profiles/); the kernel and the phase sizing of its launch
+    # (the dK/dV summary under profiles/); the file holds the kernel and the phase sizing of its launch
     "bwd_dkdv": (15447996672, {
         "token_indexed_sparse_b200/csrc/qsa_dkdv_union.cu":
-            "1ebd1ab736b167e165bf20277e70b378f50e0b542b063957dcbdd386bf5619ae",
-        "token_indexed_sparse_b200/csrc/qsa_api.cu":
-            "c7e2ca56d7da2243780efbeaf0ba3b7f06f4b3ce3b7e152b150908afcdec826e",
+            "e2339e686c44d450f2050d467a25c5c8985473c25f9691d8053f4f61416bc43e",
     }),
 }
 

@@ -25,24 +25,6 @@ qsa_status_t check_sizes(int64_t T, int64_t T_kv, int H, int G, int n_sel) {
   return QSA_OK;
 }
 
-// Query phases of the dK/dV pass: each phase covers C consecutive queries, chosen
-// so that one phase's Q and dO rows (C * H * 1 KB; the pass reads one tensor at
-// a time) stay resident in L2 (48 MiB), but at least 4096 queries: every phase
-// boundary costs an FP32 partial read and write per (tile, group, tensor), and
-// with many heads the L2 bound alone makes phases so short that this dominates
-// (seq32k, 24 heads: 2048 queries per phase ran dK/dV in 7.7 ms, 4096 in 7.1 ms;
-// with 12 heads the bound is 4096 already).  At most 64 phases.
-void dkdv_phases(int64_t T, int H, int* P, int* C) {
-  int64_t c = (int64_t{48} << 20) / (static_cast<int64_t>(H) * 1024);
-  c = c < 4096 ? 4096 : (c / 256) * 256;
-  int64_t p = (T + c - 1) / c;
-  if (p > 64) {
-    c = (((T + 63) / 64) + 255) / 256 * 256;
-    p = (T + c - 1) / c;
-  }
-  *P = static_cast<int>(p);
-  *C = static_cast<int>(c);
-}
 
 struct Layout {
   size_t status = 0, row_cnt = 0, row_cols = 0, tile_ctr = 0, tile_ptr = 0, tile_fill = 0, tile_ent = 0, delta = 0,
@@ -71,7 +53,7 @@ Layout make_layout(int64_t T, int64_t T_kv, int H, int G, int n_sel, bool backwa
   L.row_cnt = take(static_cast<size_t>(T) * 4);
   L.row_cols = take(pairs * 4);
   if (backward) {
-    dkdv_phases(T, H, &L.P, &L.C);
+    qsa::dkdv_phases(T, H, &L.P, &L.C);
     L.tile_ctr = take(tile_ctr_ints(static_cast<int64_t>(nt), L.P, G) * 4);
     L.lists = take(qsa::tile_lists_bytes(T, T_kv));  // tile masks first (zeroed with the counters), block bases
     L.tile_ptr = take((nt + 1) * 4);

@@ -585,6 +585,26 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
 
 }  // namespace
 
+// Query phases of the dK/dV pass: each phase covers C consecutive queries, chosen
+// so that one phase's Q and dO rows (C * H * 1 KB; the pass reads one tensor at
+// a time) stay resident in L2 (48 MiB), but at least 4096 queries: every phase
+// boundary costs an FP32 partial read and write per (tile, group, tensor), and
+// with many heads the L2 bound alone makes phases so short that this dominates
+// (seq32k, 24 heads: 2048 queries per phase ran dK/dV in 7.7 ms, 4096 in 7.1 ms;
+// with 12 heads the bound is 4096 already).  At most 64 phases.  It lives with
+// the kernel because the launch's DRAM traffic depends on both.
+void dkdv_phases(int64_t T, int H, int* P, int* C) {
+  int64_t c = (int64_t{48} << 20) / (static_cast<int64_t>(H) * 1024);
+  c = c < 4096 ? 4096 : (c / 256) * 256;
+  int64_t p = (T + c - 1) / c;
+  if (p > 64) {
+    c = (((T + 63) / 64) + 255) / 256 * 256;
+    p = (T + c - 1) / c;
+  }
+  *P = static_cast<int>(p);
+  *C = static_cast<int>(c);
+}
+
 cudaError_t launch_backward_dkdv_union(const void* grad_out, const void* q, const uint16_t* pds,
                                        const int32_t* row_cols, const int64_t* tile_ent, const int32_t* wl_cnt,
                                        const int4* wl, int* claim_ctr, int* done, int P, int64_t n_tiles,

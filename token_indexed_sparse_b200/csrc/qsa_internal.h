@@ -83,6 +83,9 @@ cudaError_t launch_backward_dq(const void* grad_out, const void* q, const void* 
                                void* dq, uint16_t* pds, const int* status, cudaStream_t s);
 // SM count of the current device (cached).
 int sm_count();
+// Query phases of the dK/dV pass for T queries of H heads: P phases of C
+// queries each (C a multiple of 256).
+void dkdv_phases(int64_t T, int H, int* P, int* C);
 // dK/dV over 128-key tiles on the tensor cores, all P query phases in one
 // launch: units (tile, group, tensor) of the per-phase work lists claimed from
 // *claim_ctr in phase order; the FP32 partial of a (tile, group, tensor) passes
