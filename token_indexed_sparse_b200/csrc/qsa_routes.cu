@@ -10,7 +10,13 @@
 //     list written directly in ascending query order (no sort), and the
 //     per-phase work lists the dK/dV kernel claims its units from, and
 //   * the same transpose over aligned key quads with 4-bit owner masks
-//     (quad_ptr, quad_ent), exposed by qsa_route_plan.
+//     (quad_ptr, quad_ent), exposed by qsa_route_plan, and
+//   * the query-union lists of adjacent rows (qsa_union_plan).
+// Rows are sorted by a warp in registers (bitonic networks over shfl.xor) up to
+// 1024 slots, 513-768 slots as 512 + the rest merged in shared memory, and by a
+// CTA above 1024 (register-sorted 256-slot chunks, merge-path rounds).  The
+// forward's lists stay in its workspace with a tag of their sizes, so that the
+// backward can reuse them (row_delta_masks_kernel) instead of sorting again.
 // A fixed list order makes the dK/dV summation order, and so its result bits,
 // independent of scheduling.
 #include <climits>
