@@ -50,9 +50,9 @@ SPEC_BF16_TFLOPS = 2250.0              # B200 dense BF16 tensor peak (NVIDIA spe
 TRAFFIC = {
     # the timed step's dK/dV launch on seq32k: ncu dram__bytes_read.sum + dram__bytes_write.sum
     # (the dK/dV summary under profiles/); the file holds the kernel and the phase sizing of its launch
-    "bwd_dkdv": (15447996672, {
+    "bwd_dkdv": (14818692864, {
         "token_indexed_sparse_b200/csrc/qsa_dkdv_union.cu":
-            "e2339e686c44d450f2050d467a25c5c8985473c25f9691d8053f4f61416bc43e",
+            "c650e98ff4ccfb8ca6e8c7eb14b8b19cdfce9b68cbfa355bd7b39c4da2064cbf",
     }),
 }
 

@@ -24,9 +24,10 @@
 // chunks of 8 entries, publishes each chunk's descriptor in a shared-memory ring
 // and prefetches its records and keys into L2); warps 0-11 fill the chunks,
 // warps s, s + 3, s + 6 and s + 9 every chunk of stage s of the 3-stage
-// shared-memory ring, each two of its unions (clear A, gather B rows with
-// cp.async, store the records into their A rows; a warp keeps only about eight
-// 512-byte copies in flight, so the rows of a chunk are split over four warps);
+// shared-memory ring, each two of its unions (clear A, copy the records' P or
+// dS halves straight into their A rows and gather the B rows, all with
+// cp.async; a warp keeps only about eight 512-byte copies in flight, so the
+// rows of a chunk are split over four warps);
 // warp 17 (one thread) issues the MMAs; warps 12-15 (tensor-memory lane
 // quarters 0-3) run the epilogue, thread = key row.  Units are claimed from one counter in
 // phase order (phase 0's units, then phase 1's, ...; inside a phase every dK
@@ -209,24 +210,27 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
 
   if (warp < kUWorkers) {
     // ------------------------------------------------------------ workers
-    // Warps s + 6 h (h < kUWorkersPerStage) fill chunks s, s + 6, s + 12, ...
-    // together, each taking kMy of the chunk's unions: each takes the chunk's descriptor from
-    // the scheduler's ring, waits for the chunk's stage to be free, clears its
-    // unions' A slots, gathers their 24 Q (or dO) rows into B with cp.async,
-    // stores their records into the A rows of their keys, waits for its copies
-    // and arrives on the stage's full barrier (complete when all have).  Up to
-    // kUStages chunks are in flight at once, with no barrier between stages.
+    // Warps s + 3 h (h < kUWorkersPerStage) fill chunks s, s + 3, s + 6, ...
+    // together, each taking kMy of the chunk's unions: each takes the chunk's
+    // descriptor from the scheduler's ring, loads its unions' keys, waits for
+    // the chunk's stage to be free, clears its unions' A slots, copies their
+    // records into the A rows of their keys and gathers their 24 Q (or dO) rows
+    // into B (cp.async, 8 and 16 bytes), waits for its copies and arrives on the
+    // stage's full barrier (complete when all have).  Up to kUStages chunks are
+    // in flight at once, with no barrier between stages.  (Records loaded into
+    // registers first and stored after the gather, with keys past 32 of a run
+    // loaded one after another, ran thd16k's dK/dV in 1.16 ms against 0.89 ms.)
     const int s = warp % kUStages, half = warp / kUStages;
     constexpr int kMy = kUUnions / kUWorkersPerStage;  // unions per warp
     const int u0 = kMy * half;                         // this warp's first union of a chunk
     // A rows this lane wrote in the warp's previous chunk (its stage still holds
-    // them): clearing those 24-byte slots restores zeros in this warp's unions'
-    // columns without rewriting the tile; they are cleared for all 128 rows on
-    // the stage's first use and after a chunk whose records were not all tracked
-    // (runs > 32 keys)
-    int prev_m[kMy];
+    // them; keys lane and lane + 32 of each union): clearing those 24-byte slots
+    // restores zeros in this warp's unions' columns without rewriting the tile;
+    // they are cleared for all 128 rows on the stage's first use and after a
+    // chunk whose records were not all tracked (runs > 64 keys)
+    int prev_m[kMy], prev_m2[kMy];  // A rows of keys 0..31 and 32..63 of the warp's unions
 #pragma unroll
-    for (int j = 0; j < kMy; ++j) prev_m[j] = -1;
+    for (int j = 0; j < kMy; ++j) prev_m[j] = prev_m2[j] = -1;
     bool zero_all = true;
     for (int c = s;; c += kUStages) {
       const int rs = c % kURing;
@@ -244,22 +248,19 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
       const bool end = hd.x < 0;
       if (end && hd.y == 0) break;  // an end marker for a stage whose chunk the MMA never reaches
       const int n = hd.z & 255, r = hd.z >> 10, g = r >> 1, tensor = r & 1, tile = hd.w;
-      // the records and keys of this warp's unions (j < 32), loaded first so
-      // that their latency overlaps the wait for the stage, the clearing and the
-      // row gather; record j of union u goes to A row (key - tile base), K
-      // columns 12 u .. 12 u + 11 (dK takes the record's dS half, dV its P half)
+      // the keys of this warp's unions (positions lane and lane + 32 of each
+      // run), loaded first so that their latency overlaps the wait for the
+      // stage; record i of union u goes to A row (key - tile base), K columns
+      // 12 u .. 12 u + 11 (dK takes the record's dS half, dV its P half)
       const int key0 = tile * kUKeys;
-      int32_t key[kMy];
-      uint2 val[kMy][3];
+      int32_t key[kMy], key2[kMy];
 #pragma unroll
       for (int j = 0; j < kMy; ++j) {
         const int64_t t = e[j] >> 32;
         const int i0 = static_cast<int>((e[j] >> 8) & 0x3fff), cnt = static_cast<int>(e[j] & 0x7f) + 1;
         const bool ok_j = u0 + j < n && lane < cnt;
-        const uint2* rec = reinterpret_cast<const uint2*>(pds + ((t * G + g) * n_sel + i0) * kURec) + (tensor ? 0 : 3);
         key[j] = ok_j ? __ldg(row_cols + t * n_sel + i0 + lane) : -1;
-#pragma unroll
-        for (int hq = 0; hq < 3; ++hq) val[j][hq] = ok_j ? __ldg(rec + lane * 6 + hq) : make_uint2(0, 0);
+        key2[j] = u0 + j < n && lane + 32 < cnt ? __ldg(row_cols + t * n_sel + i0 + 32 + lane) : -1;
       }
       // stage s is free once the MMAs of chunk c - kUStages completed
       if (c >= kUStages) {
@@ -293,6 +294,32 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
 #pragma unroll
             for (int hq = 0; hq < 3; ++hq) *slot(u0 + j, prev_m[j], hq) = make_uint2(0, 0);
           }
+#pragma unroll
+        for (int j = 0; j < kMy; ++j)
+          if (prev_m2[j] >= 0) {
+#pragma unroll
+            for (int hq = 0; hq < 3; ++hq) *slot(u0 + j, prev_m2[j], hq) = make_uint2(0, 0);
+          }
+      }
+      __syncwarp();  // the clearing above before the record copies below
+      // record i of union u (its P or dS half: 3 x 8 bytes) straight into the A
+      // row of its key; returns that row, or -1
+      auto copy_rec = [&](int j, int32_t k, int i) -> int {
+        const int m = k - key0;
+        if (k < 0 || static_cast<unsigned>(m) >= static_cast<unsigned>(kUKeys)) return -1;  // never for a well-formed list
+        const int64_t t = e[j] >> 32;
+        const int i0 = static_cast<int>((e[j] >> 8) & 0x3fff);
+        const uint2* rec = reinterpret_cast<const uint2*>(pds + ((t * G + g) * n_sel + i0 + i) * kURec) + (tensor ? 0 : 3);
+#pragma unroll
+        for (int hq = 0; hq < 3; ++hq)
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(smem_u32(slot(u0 + j, m, hq))), "l"(rec + hq)
+                       : "memory");
+        return m;
+      };
+#pragma unroll
+      for (int j = 0; j < kMy; ++j) {
+        prev_m[j] = copy_rec(j, key[j], lane);
+        prev_m2[j] = copy_rec(j, key2[j], lane + 32);
       }
       // B: the 12 head rows of each of this warp's unions (zero-filled for missing unions)
       {
@@ -311,7 +338,6 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
         }
       }
       cp_async_commit();
-      __syncwarp();  // the clearing above before the record stores below
       // stores record j of union u; returns its A row, or -1
       auto put = [&](int u, int32_t k, const uint2 (&v)[3]) -> int {
         const int m = k - key0;
@@ -320,9 +346,7 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
         for (int hq = 0; hq < 3; ++hq) *slot(u, m, hq) = v[hq];
         return m;
       };
-#pragma unroll
-      for (int j = 0; j < kMy; ++j) prev_m[j] = put(u0 + j, key[j], val[j]);
-      // unions with more than 32 keys in the tile (rare for sparse routes); their
+      // unions with more than 64 keys in the tile (rare for sparse routes); their
       // extra rows are not tracked, so the next chunk of this stage clears all
       // of this warp's slots
       zero_all = false;
@@ -330,10 +354,10 @@ dkdv_union_kernel(const __nv_bfloat16* __restrict__ dout, const __nv_bfloat16* _
       for (int j = 0; j < kMy; ++j) {
         const int64_t t = e[j] >> 32;
         const int i0 = static_cast<int>((e[j] >> 8) & 0x3fff), cnt = static_cast<int>(e[j] & 0x7f) + 1;
-        if (u0 + j >= n || cnt <= 32) continue;
+        if (u0 + j >= n || cnt <= 64) continue;
         zero_all = true;
         const uint2* rec = reinterpret_cast<const uint2*>(pds + ((t * G + g) * n_sel + i0) * kURec) + (tensor ? 0 : 3);
-        for (int jj = lane + 32; jj < cnt; jj += 32) {
+        for (int jj = lane + 64; jj < cnt; jj += 32) {
           const uint2 v[3] = {__ldg(rec + jj * 6), __ldg(rec + jj * 6 + 1), __ldg(rec + jj * 6 + 2)};
           put(u0 + j, __ldg(row_cols + t * n_sel + i0 + jj), v);
         }
