@@ -476,6 +476,7 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {**workload_config(wl), "pairs_per_step": pairs, "flops_per_step": flops,
                    "l2": "flushed (256 MiB write) before every timed step, outside its events",
+                   "backward": "on the forward's saved route lists (qsa_backward_saved)",
                    "parallelism": f"{world} independent sequences (one per GPU)" if world > 1 else "1 GPU"},
         "tflops": step_tflops * world,
         "step_roofline": {"flops": flops, "t_roof_ms": flops / (peaks["bf16_tflops"] * 1e12) * 1e3,
@@ -607,6 +608,7 @@ def run_cp(args):
         "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {**workload_config(wl), "pairs_per_step": pairs_total, "flops_per_step": flops,
                    "l2": "flushed (256 MiB write) before every timed step, outside its events",
+                   "backward": "on the forward's saved route lists (qsa_backward_saved)",
                    "parallelism": f"cp{world}: one sequence, query rows balanced by routed pairs, K/V "
                                   f"all-gather and FP32 dK/dV reduce-scatter over NCCL"},
         "tflops": flops * args.steps / (total_ms * 1e-3) / 1e12,
