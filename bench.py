@@ -423,8 +423,8 @@ def run_ours(args):
                 ev_out[b].record(s_out)
 
     # enough steps that the pipeline's fill (the first inputs) and drain (the
-    # last results) weigh little against the steady state
-    e2e_steps = max(10, args.steps)
+    # last results) weigh little against the steady state (about 1 s of copies)
+    e2e_steps = max(40, args.steps)
     e2e_run(2)
     torch.cuda.synchronize()
     e0, e1 = mk(), mk()
